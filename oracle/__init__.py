@@ -1,0 +1,235 @@
+"""CPU oracle for the BitNet b1.58 BitLinear forward path.
+
+TEST INFRASTRUCTURE ONLY.  The tests, the smoke check and the benchmark's CPU
+baseline leg are the only callers; the CUDA library never imports, links or
+executes anything here, and this package imports nothing from it.
+
+The arithmetic lives in ``bitlinear_oracle.c`` (plain scalar C, compiled with
+``-ffp-contract=off`` and no fast-math).  This module only compiles it, loads
+it with ctypes and marshals numpy arrays in and out.
+
+Page cited throughout as [MF]: "BitNet b1.58: Mathematical Foundations of
+1.58-Bit Ternary Quantization, Absmean Scaling, and Multiplication-Free LLM
+Architectures", section 2 (weight absmean quantisation, activation absmax
+quantisation, the linear transformation and rescaling) and section 6
+(vectorized ternary GEMV: sign/zero masks, masked addition).
+
+Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
+against closed forms, library routines, hand-worked fixtures and brute force;
+none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bitlinear_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+QB_MINUS_1 = 127  # [MF] §2: Q_b - 1, multiplier and clip bound of the activation codes
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc; returns the path of the shared object."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + ".tmp.%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+           "-fno-fast-math", "-fno-unsafe-math-optimizations", "-Wall", "-Wextra",
+           _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i64, f32, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_int
+        vp = ctypes.c_void_p
+        lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f32.restype = f32
+        lib.oracle_f32_to_bf16.argtypes = [f32]
+        lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        lib.oracle_abs_sum.argtypes = [vp, i64, i64]
+        lib.oracle_abs_sum.restype = ctypes.c_double
+        lib.oracle_absmean_gamma.argtypes = [vp, i64, i64]
+        lib.oracle_absmean_gamma.restype = f32
+        lib.oracle_ternarize.argtypes = [vp, i64, f32, f32, vp]
+        lib.oracle_ternarize.restype = None
+        lib.oracle_pack.argtypes = [vp, i64, i64, vp]
+        lib.oracle_pack.restype = i32
+        lib.oracle_unpack.argtypes = [vp, i64, i64, vp]
+        lib.oracle_unpack.restype = i32
+        lib.oracle_unpack_row.argtypes = [vp, i64, i64, i64, vp]
+        lib.oracle_unpack_row.restype = i32
+        lib.oracle_rms.argtypes = [vp, i64, f32]
+        lib.oracle_rms.restype = f32
+        lib.oracle_quant_act.argtypes = [vp, i64, i64, vp, i32, f32, f32, vp,
+                                         vp, vp, vp, vp]
+        lib.oracle_quant_act.restype = None
+        lib.oracle_int_matmul.argtypes = [vp, vp, i64, i64, i64, vp]
+        lib.oracle_int_matmul.restype = None
+        lib.oracle_dot_masked_add.argtypes = [vp, vp, i64]
+        lib.oracle_dot_masked_add.restype = ctypes.c_int32
+        lib.oracle_rescale.argtypes = [vp, i64, i64, f32, vp, vp]
+        lib.oracle_rescale.restype = None
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ------------------------------------------------------------------ bf16 ---
+
+def bf16_bits_to_f32(bits) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float32."""
+    lib = _load()
+    b = _c(bits, np.uint16).ravel()
+    return np.array([lib.oracle_bf16_to_f32(int(v)) for v in b],
+                    dtype=np.float32).reshape(np.shape(bits))
+
+
+def f32_to_bf16_bits(x) -> np.ndarray:
+    """float32 -> bf16 bit patterns, round to nearest even."""
+    lib = _load()
+    a = _c(x, np.float32).ravel()
+    return np.array([lib.oracle_f32_to_bf16(float(v)) for v in a],
+                    dtype=np.uint16).reshape(np.shape(x))
+
+
+# ---------------------------------------------------- weight quantisation ---
+
+def abs_sum(W) -> float:
+    W = _c(W, np.float32)
+    return _load().oracle_abs_sum(_ptr(W), W.shape[0], W.shape[1])
+
+
+def absmean_gamma(W) -> float:
+    """gamma = mean |W_ij| over the whole tensor ([MF] §2)."""
+    W = _c(W, np.float32)
+    return float(_load().oracle_absmean_gamma(_ptr(W), W.shape[0], W.shape[1]))
+
+
+def ternarize(W, gamma: float, eps: float = 1e-5) -> np.ndarray:
+    """W~ = RoundClip(W / (gamma + eps), -1, 1) in int8 ([MF] §2)."""
+    W = _c(W, np.float32)
+    out = np.empty(W.shape, dtype=np.int8)
+    _load().oracle_ternarize(_ptr(W), W.size, gamma, eps, _ptr(out))
+    return out
+
+
+def pack(wq) -> np.ndarray:
+    """Ternary codes [d_out][d_in] -> packed uint32 words (tile layout)."""
+    wq = _c(wq, np.int8)
+    n, k = wq.shape
+    out = np.empty(n * k // 16 if (n % 16 == 0 and k % 256 == 0) else 0,
+                   dtype=np.uint32)
+    rc = _load().oracle_pack(_ptr(wq), n, k, _ptr(out) if out.size else None)
+    if rc != 0:
+        raise ValueError("oracle_pack: shape not a whole number of 16x256 tiles "
+                         "or a code outside {-1,0,1}")
+    return out
+
+
+def unpack(packed, d_out: int, d_in: int) -> np.ndarray:
+    packed = _c(packed, np.uint32)
+    out = np.empty((d_out, d_in), dtype=np.int8)
+    rc = _load().oracle_unpack(_ptr(packed), d_out, d_in, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_unpack: invalid code 3 or bad shape")
+    return out
+
+
+def unpack_row(packed, d_out: int, d_in: int, o: int) -> np.ndarray:
+    packed = _c(packed, np.uint32)
+    out = np.empty(d_in, dtype=np.int8)
+    rc = _load().oracle_unpack_row(_ptr(packed), d_out, d_in, o, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_unpack_row: invalid code 3 or bad index")
+    return out
+
+
+# ------------------------------------------------ activation quantisation ---
+
+def rms(x_bf16_bits, norm_eps: float = 1e-5) -> float:
+    x = _c(x_bf16_bits, np.uint16)
+    return float(_load().oracle_rms(_ptr(x), x.size, norm_eps))
+
+
+def quant_act(X_bf16_bits, gain=None, rmsnorm: bool = True, eps: float = 1e-5,
+              norm_eps: float = 1e-5, rms_in=None):
+    """Per-token absmax int8 quantisation, optional RMSNorm first ([MF] §2).
+
+    Returns (xq int8 [T][K], beta f32 [T], rowsum int32 [T], rms f32 [T]).
+    """
+    X = _c(X_bf16_bits, np.uint16)
+    T, K = X.shape
+    g = None if gain is None else _c(gain, np.float32)
+    r_in = None if rms_in is None else _c(rms_in, np.float32)
+    xq = np.empty((T, K), dtype=np.int8)
+    beta = np.empty(T, dtype=np.float32)
+    rowsum = np.empty(T, dtype=np.int32)
+    rms_out = np.empty(T, dtype=np.float32)
+    _load().oracle_quant_act(_ptr(X), T, K, _ptr(g), int(bool(rmsnorm)), eps,
+                             norm_eps, _ptr(r_in), _ptr(xq), _ptr(beta),
+                             _ptr(rowsum), _ptr(rms_out))
+    return xq, beta, rowsum, rms_out
+
+
+# ----------------------------------------------------- product / rescale ---
+
+def int_matmul(wq, xq) -> np.ndarray:
+    """acc[t][o] = sum_k W~[o][k] X~[t][k] in int32 ([MF] §2)."""
+    wq = _c(wq, np.int8)
+    xq = _c(xq, np.int8)
+    N, K = wq.shape
+    T = xq.shape[0]
+    acc = np.empty((T, N), dtype=np.int32)
+    _load().oracle_int_matmul(_ptr(wq), _ptr(xq), T, N, K, _ptr(acc))
+    return acc
+
+
+def dot_masked_add(wrow, xrow) -> int:
+    """Sign-mask / zero-mask masked-add dot product ([MF] §6)."""
+    w = _c(wrow, np.int8)
+    x = _c(xrow, np.int8)
+    return int(_load().oracle_dot_masked_add(_ptr(w), _ptr(x), w.size))
+
+
+def rescale(acc, gamma: float, beta) -> np.ndarray:
+    """Y = acc * beta * gamma / (Q_b - 1), in float64 ([MF] §2)."""
+    acc = _c(acc, np.int32)
+    beta = _c(beta, np.float32)
+    T, N = acc.shape
+    y = np.empty((T, N), dtype=np.float64)
+    _load().oracle_rescale(_ptr(acc), T, N, gamma, _ptr(beta), _ptr(y))
+    return y
+
+
+def forward(W, X_bf16_bits, eps: float = 1e-5, norm_eps: float = 1e-5, gain=None,
+            rmsnorm: bool = True, gamma=None, rms_in=None):
+    """The whole BitLinear forward on the CPU: returns a dict of every stage."""
+    g = absmean_gamma(W) if gamma is None else float(gamma)
+    wq = ternarize(W, g, eps)
+    xq, beta, rowsum, r = quant_act(X_bf16_bits, gain, rmsnorm, eps, norm_eps,
+                                    rms_in)
+    acc = int_matmul(wq, xq)
+    y = rescale(acc, g, beta)
+    return dict(gamma=g, wq=wq, xq=xq, beta=beta, rowsum=rowsum, rms=r, acc=acc,
+                y=y)

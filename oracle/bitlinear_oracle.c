@@ -1,0 +1,294 @@
+/*
+ * bitlinear_oracle.c -- plain, slow, obviously-correct CPU statement of the
+ * BitNet b1.58 BitLinear forward computation.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header, table or helper with the CUDA
+ * library; the two meet only through the seeded synthetic inputs.
+ *
+ * Source of every step (cited as [MF]):
+ *   "BitNet b1.58: Mathematical Foundations of 1.58-Bit Ternary Quantization,
+ *    Absmean Scaling, and Multiplication-Free LLM Architectures" (llms.blog),
+ *   section 2 "Mathematical Formulation of the BitLinear b1.58 Layer" with its
+ *   three parts "Weight Quantization: Absmean Scaling", "Activation
+ *   Quantization: Absmax Scaling" and "The Linear Transformation and
+ *   Rescaling"; section 6 "Implementation Considerations and Inference
+ *   Engines", part "Vectorized Ternary GEMV with SIMD" (sign / zero masks,
+ *   masked addition, scale-factor fusion).
+ *
+ * Precision: reductions (the absmean sum, the RMS sum of squares) and the
+ * final rescale are carried in double.  The quantities that feed an integer
+ * code (z = W / (gamma + eps), n = x / rms, v = n * 127 / (beta + eps)) are
+ * formed in IEEE binary32, one correctly rounded operation at a time, because
+ * that is the precision in which the GPU kernels form them; the rounding
+ * floor(z + 0.5) itself is then evaluated exactly.  This file is compiled
+ * with -ffp-contract=off and without fast-math so no operation is fused.
+ *
+ * Readings taken where the page is silent or inconsistent:
+ *   - Q_b - 1 = 127 is both the activation multiplier and the clip bound; the
+ *     code range is the symmetric [-127, 127].
+ *   - The activation absmax beta is taken per token (one row of X).
+ *   - RMSNorm is x / sqrt(mean(x^2) + norm_eps) * g, with g = 1 unless a gain
+ *     vector is given; the page names RMSNorm but prints no formula.
+ *   - The rescale is the literal beta*gamma/(Q_b-1), without the epsilons used
+ *     inside the two quantisers.
+ *   - RoundClip rounds with floor(z + 0.5), i.e. halves go toward +infinity,
+ *     evaluated exactly on the binary32 value z.
+ *
+ * Packed weight layout (this library's own format; the page only says
+ * "packed 2-bit"): a d_out x d_in ternary matrix is cut into tiles of 16 rows
+ * by 256 columns, stored tile-row-major; inside a tile the 16 rows follow one
+ * another, each as 16 little-endian 32-bit words; word kw of a row holds
+ * columns 16*kw .. 16*kw+15 and the 2-bit code c = W~ + 1 of column
+ * 16*kw + 4*s + j sits at bits 8*j + 2*s.  Code 3 is never produced and is
+ * rejected on unpack.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_QB_MINUS_1 127
+
+/* ---------------------------------------------------------------- bf16 --- */
+
+/* bf16 -> binary32 is exact: the bf16 pattern is the top half of the float. */
+float oracle_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* binary32 -> bf16, round to nearest, ties to even (finite inputs). */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint32_t lower = u & 0xFFFFu;
+    uint32_t upper = u >> 16;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))
+        upper += 1u;
+    return (uint16_t)upper;
+}
+
+/* ------------------------------------------ weight quantisation ([MF] §2) */
+
+/* Sum over all entries of |W_ij|, in double, in index order. */
+double oracle_abs_sum(const float *W, int64_t n_out, int64_t n_in)
+{
+    double s = 0.0;
+    for (int64_t i = 0; i < n_out * n_in; ++i)
+        s += fabs((double)W[i]);
+    return s;
+}
+
+/* gamma = (1 / (d_out d_in)) * sum |W_ij|   ([MF] §2, absmean scale). */
+float oracle_absmean_gamma(const float *W, int64_t n_out, int64_t n_in)
+{
+    double s = oracle_abs_sum(W, n_out, n_in);
+    return (float)(s / ((double)n_out * (double)n_in));
+}
+
+/* RoundClip(z, a, b) = max(a, min(b, floor(z + 0.5)))   ([MF] §2).
+ * z arrives in binary32; floor(z + 0.5) is then taken exactly: the sum is
+ * formed in double, which holds z + 0.5 without rounding whenever it lies
+ * near an integer (|z| >= 0.5 there, so z has no bits below 2^-24 of its
+ * leading bit).  A binary32 sum would round 0.5 - 2^-25 + 0.5 up to 1. */
+static float round_clip_f32(float z, float a, float b)
+{
+    double u = (double)z + 0.5;
+    float r = (float)floor(u);
+    if (r > b) r = b;
+    if (r < a) r = a;
+    return r;
+}
+
+/* W~_ij = RoundClip(W_ij / (gamma + eps), -1, 1)   ([MF] §2). */
+void oracle_ternarize(const float *W, int64_t count, float gamma, float eps,
+                      int8_t *wq)
+{
+    float den = gamma + eps;   /* binary32 addition */
+    for (int64_t i = 0; i < count; ++i) {
+        float z = W[i] / den;  /* binary32 division */
+        wq[i] = (int8_t)round_clip_f32(z, -1.0f, 1.0f);
+    }
+}
+
+/* ------------------------------------------------------- packed layout --- */
+
+/* Index of the word holding weight (o, k) and the bit offset of its code. */
+static void packed_position(int64_t n_in, int64_t o, int64_t k,
+                            int64_t *word, int *shift)
+{
+    int64_t tiles_per_row = n_in / 256;
+    int64_t rb = o / 16, r = o % 16;
+    int64_t kb = k / 256, kw = (k % 256) / 16;
+    int s = (int)((k % 16) / 4), j = (int)(k % 4);
+    *word = ((rb * tiles_per_row + kb) * 16 + r) * 16 + kw;
+    *shift = 8 * j + 2 * s;
+}
+
+/* Returns 0, or -1 if a shape is not a whole number of tiles or a code is
+ * outside {-1, 0, 1}. */
+int oracle_pack(const int8_t *wq, int64_t n_out, int64_t n_in, uint32_t *packed)
+{
+    if (n_out % 16 != 0 || n_in % 256 != 0) return -1;
+    memset(packed, 0, (size_t)(n_out * n_in / 16) * sizeof(uint32_t));
+    for (int64_t o = 0; o < n_out; ++o) {
+        for (int64_t k = 0; k < n_in; ++k) {
+            int v = wq[o * n_in + k];
+            if (v < -1 || v > 1) return -1;
+            int64_t word;
+            int shift;
+            packed_position(n_in, o, k, &word, &shift);
+            packed[word] |= ((uint32_t)(v + 1)) << shift;
+        }
+    }
+    return 0;
+}
+
+/* Inverse of oracle_pack.  Returns -1 on the unused code 3. */
+int oracle_unpack(const uint32_t *packed, int64_t n_out, int64_t n_in, int8_t *wq)
+{
+    if (n_out % 16 != 0 || n_in % 256 != 0) return -1;
+    for (int64_t o = 0; o < n_out; ++o) {
+        for (int64_t k = 0; k < n_in; ++k) {
+            int64_t word;
+            int shift;
+            packed_position(n_in, o, k, &word, &shift);
+            uint32_t c = (packed[word] >> shift) & 3u;
+            if (c == 3u) return -1;
+            wq[o * n_in + k] = (int8_t)((int)c - 1);
+        }
+    }
+    return 0;
+}
+
+/* One row of codes read back out of the packed buffer (for sampled checks on
+ * matrices too large to unpack whole).  Returns -1 on code 3. */
+int oracle_unpack_row(const uint32_t *packed, int64_t n_out, int64_t n_in,
+                      int64_t o, int8_t *row)
+{
+    if (n_out % 16 != 0 || n_in % 256 != 0 || o < 0 || o >= n_out) return -1;
+    for (int64_t k = 0; k < n_in; ++k) {
+        int64_t word;
+        int shift;
+        packed_position(n_in, o, k, &word, &shift);
+        uint32_t c = (packed[word] >> shift) & 3u;
+        if (c == 3u) return -1;
+        row[k] = (int8_t)((int)c - 1);
+    }
+    return 0;
+}
+
+/* ---------------------------------------- activation quantisation ([MF] §2) */
+
+/* RMS of one token: sqrt(mean(x^2) + norm_eps), carried in double and
+ * rounded once to binary32. */
+float oracle_rms(const uint16_t *x, int64_t K, float norm_eps)
+{
+    double ss = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        double v = (double)oracle_bf16_to_f32(x[k]);
+        ss += v * v;
+    }
+    return (float)sqrt(ss / (double)K + (double)norm_eps);
+}
+
+/*
+ * Per-token absmax int8 quantisation with optional RMSNorm in front.
+ *   n_k   = x_k / rms (binary32 division), times g_k if a gain is given
+ *           (binary32 multiplication); n_k = x_k when rmsnorm == 0
+ *   beta  = max_k |n_k|
+ *   q_k   = RoundClip(n_k * 127 / (beta + eps), -127, 127) with the scale
+ *           127 / (beta + eps) formed first (binary32 add, then divide) and
+ *           applied with one binary32 multiplication
+ *   S     = sum_k q_k (the correction term of the offset-code product)
+ * rms_in, when not NULL, supplies the per-token rms instead of computing it
+ * (used to compare integer codes against a GPU that computed its own rms).
+ */
+void oracle_quant_act(const uint16_t *X, int64_t T, int64_t K, const float *gain,
+                      int rmsnorm, float eps, float norm_eps, const float *rms_in,
+                      int8_t *xq, float *beta, int32_t *rowsum, float *rms_out)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *x = X + t * K;
+        float rms = 1.0f;
+        if (rmsnorm)
+            rms = rms_in ? rms_in[t] : oracle_rms(x, K, norm_eps);
+        if (rms_out) rms_out[t] = rms;
+
+        float b = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float n = oracle_bf16_to_f32(x[k]);
+            if (rmsnorm) {
+                n = n / rms;
+                if (gain) n = n * gain[k];
+            }
+            float a = fabsf(n);
+            if (a > b) b = a;
+        }
+        beta[t] = b;
+
+        float scale = (float)ORACLE_QB_MINUS_1 / (b + eps);
+        int32_t S = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            float n = oracle_bf16_to_f32(x[k]);
+            if (rmsnorm) {
+                n = n / rms;
+                if (gain) n = n * gain[k];
+            }
+            float v = n * scale;
+            int q = (int)round_clip_f32(v, -(float)ORACLE_QB_MINUS_1,
+                                        (float)ORACLE_QB_MINUS_1);
+            xq[t * K + k] = (int8_t)q;
+            S += q;
+        }
+        rowsum[t] = S;
+    }
+}
+
+/* ---------------------------------- product and rescale ([MF] §2 and §6) */
+
+/* acc[t][o] = sum_k W~[o][k] * X~[t][k], exact in int32. */
+void oracle_int_matmul(const int8_t *wq, const int8_t *xq, int64_t T, int64_t N,
+                       int64_t K, int32_t *acc)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t o = 0; o < N; ++o) {
+            int32_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int32_t)wq[o * K + k] * (int32_t)xq[t * K + k];
+            acc[t * N + o] = s;
+        }
+}
+
+/* The same dot product written the multiplier-free way of [MF] §6: unpack a
+ * sign mask and a zero mask per weight and add (x XOR sign) - sign where the
+ * weight is non-zero.  sign is all ones (-1) for a -1 weight and 0 otherwise;
+ * on two's-complement int8 (x ^ -1) - (-1) = ~x + 1 = -x. */
+int32_t oracle_dot_masked_add(const int8_t *wrow, const int8_t *xrow, int64_t K)
+{
+    int32_t acc = 0;
+    for (int64_t k = 0; k < K; ++k) {
+        int32_t sign = (wrow[k] < 0) ? -1 : 0;
+        int nonzero = (wrow[k] != 0);
+        if (nonzero)
+            acc += ((int32_t)xrow[k] ^ sign) - sign;
+    }
+    return acc;
+}
+
+/* Y = (X~ W~^T) * beta * gamma / (Q_b - 1), in double ([MF] §2). */
+void oracle_rescale(const int32_t *acc, int64_t T, int64_t N, float gamma,
+                    const float *beta, double *y)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        double scale = (double)beta[t] * (double)gamma / (double)ORACLE_QB_MINUS_1;
+        for (int64_t o = 0; o < N; ++o)
+            y[t * N + o] = (double)acc[t * N + o] * scale;
+    }
+}

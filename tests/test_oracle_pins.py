@@ -1,0 +1,334 @@
+"""Pins of the CPU oracle to facts other than itself.
+
+Each test checks the oracle against something fixed by the page or by
+mathematics: a hand-worked example, a closed form, a statistical law, a
+library routine computing the same quantity another way, brute force on
+tiny inputs, or an identity printed on the page.  Page cited as [MF]:
+"BitNet b1.58: Mathematical Foundations of 1.58-Bit Ternary Quantization,
+Absmean Scaling, and Multiplication-Free LLM Architectures".
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import Problem, bf16_bits, draw
+
+RNG = np.random.default_rng(1234)
+
+
+def _bits(x):
+    return bf16_bits(torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16))
+
+
+# ------------------------------------------------------------- worked example
+
+def test_worked_example(golden_dir):
+    """Hand-derived example from the formulas of [MF] §2 (the page prints none)."""
+    ex = json.load(open(os.path.join(golden_dir, "worked_example.json")))
+    W = np.array(ex["W"], dtype=np.float32)
+    X = _bits(ex["X"])
+    out = oracle.forward(W, X, eps=ex["eps"], norm_eps=ex["norm_eps"])
+    assert out["gamma"] == ex["gamma"]
+    np.testing.assert_array_equal(out["wq"], np.array(ex["W_ternary"]))
+    assert abs(out["rms"][0] - ex["rms"]) < 2e-6
+    assert abs(out["beta"][0] - ex["beta"]) < 2e-6
+    np.testing.assert_array_equal(out["xq"], np.array(ex["X_int8"]))
+    np.testing.assert_array_equal(out["rowsum"], np.array(ex["rowsum"]))
+    np.testing.assert_array_equal(out["acc"], np.array(ex["acc"]))
+    np.testing.assert_allclose(out["y"], np.array(ex["Y"]), rtol=2e-6)
+
+
+# ------------------------------------------------------------------- bf16
+
+def test_bf16_conversions_match_torch():
+    x = np.concatenate([RNG.standard_normal(2000).astype(np.float32) * 10,
+                        np.array([0.0, -0.0, 1.0, 1.00390625, 1.0078125,
+                                  1.005859375, 1.001953125, 3.0e-39, 65504.0],
+                                 dtype=np.float32)])
+    mine = oracle.f32_to_bf16_bits(x)
+    ref = bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+    np.testing.assert_array_equal(mine, ref)
+    back = oracle.bf16_bits_to_f32(ref)
+    np.testing.assert_array_equal(
+        back, torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy())
+
+
+# ------------------------------------------------------------------ gamma
+
+def test_gamma_constant_magnitude():
+    """|W_ij| = c everywhere => gamma = c exactly ([MF] §2, absmean)."""
+    c = np.float32(0.0234375)  # exactly representable
+    signs = RNG.choice([-1.0, 1.0], size=(48, 256)).astype(np.float32)
+    assert oracle.absmean_gamma(signs * c) == float(c)
+
+
+def test_gamma_half_normal_mean():
+    """E|W| = sigma*sqrt(2/pi) for W ~ N(0, sigma^2) (half-normal mean)."""
+    for sigma, seed in ((0.02, 0), (0.015, 3)):
+        W = draw(Problem("h", 1024, 1024, 1, sigma, 0.0, 1.0, seed))[0].numpy()
+        g = oracle.absmean_gamma(W)
+        mean = sigma * math.sqrt(2 / math.pi)
+        se = sigma * math.sqrt(1 - 2 / math.pi) / math.sqrt(W.size)
+        assert abs(g - mean) < 5 * se, (g, mean, se)
+
+
+def test_gamma_sum_against_exact_sum():
+    """The double sum agrees with math.fsum (correctly rounded) to 1e-12."""
+    W = (RNG.standard_normal((64, 512)) * 0.02).astype(np.float32)
+    exact = math.fsum(abs(float(v)) for v in W.ravel())
+    assert abs(oracle.abs_sum(W) - exact) <= 1e-12 * exact
+    assert oracle.absmean_gamma(W) == np.float32(exact / W.size)
+
+
+def test_gamma_homogeneous_and_sign_free():
+    W = (RNG.standard_normal((32, 256)) * 0.02).astype(np.float32)
+    g = oracle.absmean_gamma(W)
+    assert oracle.absmean_gamma(-W) == g
+    assert oracle.absmean_gamma(W * np.float32(4.0)) == np.float32(4.0) * np.float32(g)
+    assert abs(oracle.absmean_gamma(np.ascontiguousarray(W.T)) - g) <= 1e-7 * g
+
+
+# ------------------------------------------------------------- ternarise
+
+def test_ternary_alphabet_and_gaussian_zero_fraction():
+    """W~ in {-1,0,1}; for Gaussian W the zero fraction is
+    P(|Z| < sqrt(2/pi)/2) = erf(1/(2 sqrt(pi))) = 0.3101 and +-1 split evenly."""
+    W = draw(Problem("z", 2048, 1024, 1, 0.02, 0.0, 1.0, 7))[0].numpy()
+    wq = oracle.ternarize(W, oracle.absmean_gamma(W))
+    assert set(np.unique(wq).tolist()) <= {-1, 0, 1}
+    p0 = math.erf(1 / (2 * math.sqrt(math.pi)))
+    frac0 = float((wq == 0).mean())
+    se = math.sqrt(p0 * (1 - p0) / wq.size)
+    assert abs(frac0 - p0) < 6 * se, (frac0, p0)
+    fp, fm = float((wq == 1).mean()), float((wq == -1).mean())
+    assert abs(fp - fm) < 12 * se
+
+
+def test_roundclip_ties_and_clip():
+    """RoundClip(z) = max(-1, min(1, floor(z + 0.5))): halves round up ([MF] §2).
+    With gamma = 1 and eps = 0 the divisor is exactly 1, so z = W."""
+    W = np.array([[0.5, -0.5, 1.5, -1.5, 0.49999997, -0.50000006, 7.0, -7.0,
+                   0.0, -0.0, 1.0, -1.0]], dtype=np.float32)
+    got = oracle.ternarize(W, 1.0, 0.0)[0].tolist()
+    assert got == [1, 0, 1, -1, 0, -1, 1, -1, 0, 0, 1, -1]
+
+
+def test_ternarize_is_nearest_level_with_ties_up():
+    """Second formulation: the code is the level in {-1,0,1} nearest to
+    z = fl32(W / fl32(gamma + eps)), ties to the larger level."""
+    W = (RNG.standard_normal(4096) * 0.02).astype(np.float32)
+    gamma, eps = 0.0159, 1e-5
+    wq = oracle.ternarize(W[None, :], gamma, eps)[0]
+    z = W / (np.float32(gamma) + np.float32(eps))            # binary32 as in [MF]
+    levels = np.array([-1.0, 0.0, 1.0])
+    d = np.abs(z.astype(np.float64)[:, None] - levels[None, :])
+    best = np.where(d == d.min(axis=1, keepdims=True), levels[None, :], -np.inf).max(axis=1)
+    np.testing.assert_array_equal(wq, best.astype(np.int8))
+
+
+def test_zero_weights():
+    W = np.zeros((16, 256), dtype=np.float32)
+    g = oracle.absmean_gamma(W)
+    assert g == 0.0
+    assert not oracle.ternarize(W, g).any()
+
+
+# ----------------------------------------------------------------- packing
+
+def test_pack_layout_golden(golden_dir):
+    ex = json.load(open(os.path.join(golden_dir, "packed_layout.json")))
+    n, k = ex["d_out"], ex["d_in"]
+    assert (oracle.pack(np.zeros((n, k), np.int8)) == 0x55555555).all()
+    for c in ex["cases"]:
+        wq = np.zeros((n, k), np.int8)
+        wq[c["o"], c["k"]] = c["w"]
+        p = oracle.pack(wq)
+        expect = np.full(p.shape, 0x55555555, dtype=np.uint32)
+        expect[c["word"]] = int(c["value"], 16)
+        np.testing.assert_array_equal(p, expect, err_msg=str(c))
+
+
+@pytest.mark.parametrize("shape", [(16, 256), (32, 512), (48, 768), (144, 2560)])
+def test_pack_roundtrip(shape):
+    wq = RNG.integers(-1, 2, size=shape).astype(np.int8)
+    p = oracle.pack(wq)
+    assert p.size == shape[0] * shape[1] // 16
+    np.testing.assert_array_equal(oracle.unpack(p, *shape), wq)
+    for o in (0, shape[0] - 1, shape[0] // 3):
+        np.testing.assert_array_equal(oracle.unpack_row(p, *shape, o), wq[o])
+
+
+def test_pack_exhaustive_groups():
+    """All 81 joint values of the four codes that share one byte (same s)
+    and of the four that share one 2-bit slot across bytes (same j)."""
+    import itertools
+    for combo in itertools.product((-1, 0, 1), repeat=4):
+        for pos in (lambda i: i, lambda i: 4 * i):     # same-s group / same-j group
+            wq = np.zeros((16, 256), np.int8)
+            for i, v in enumerate(combo):
+                wq[5, 32 + pos(i)] = v
+            np.testing.assert_array_equal(
+                oracle.unpack(oracle.pack(wq), 16, 256), wq)
+
+
+def test_pack_rejects_bad_input():
+    with pytest.raises(ValueError):
+        oracle.pack(np.full((16, 256), 2, np.int8))
+    with pytest.raises(ValueError):
+        oracle.pack(np.zeros((16, 128), np.int8))
+    p = oracle.pack(np.zeros((16, 256), np.int8))
+    p[7] |= 3  # plant the unused code 3
+    with pytest.raises(ValueError):
+        oracle.unpack(p, 16, 256)
+
+
+# ------------------------------------------------------- activation quant
+
+def test_rms_matches_torch_rms_norm():
+    """rms(x) agrees with torch.nn.functional.rms_norm (float64) to 1e-7."""
+    X = draw(Problem("r", 2560, 16, 8, 0.02, 0.005, 100.0, 11))[1]
+    bits = bf16_bits(X)
+    x64 = X.to(torch.float64)
+    y = torch.nn.functional.rms_norm(x64, (x64.shape[1],), eps=float(np.float32(1e-5)))
+    for t in range(X.shape[0]):
+        k = int(torch.argmax(x64[t].abs()))
+        lib_rms = float(x64[t, k] / y[t, k])
+        assert abs(oracle.rms(bits[t]) - lib_rms) <= 1e-7 * lib_rms
+
+
+def test_quant_act_invariants():
+    X = draw(Problem("a", 2560, 16, 8, 0.02, 0.005, 100.0, 5))[1]
+    bits = bf16_bits(X)
+    xq, beta, rowsum, r = oracle.quant_act(bits)
+    assert xq.min() >= -127 and xq.max() <= 127
+    np.testing.assert_array_equal(rowsum, xq.astype(np.int64).sum(axis=1))
+    xf = X.float().numpy()
+    for t in range(xq.shape[0]):
+        k = int(np.argmax(np.abs(xf[t])))
+        assert abs(int(xq[t, k])) == 127                    # absmax channel -> +-Qb-1
+        assert np.all((xq[t] == 0) | (np.sign(xq[t]) == np.sign(xf[t])))
+        np.testing.assert_allclose(beta[t], np.abs(xf[t]).max() / r[t], rtol=2e-7)
+
+
+def test_quant_act_nearest_integer():
+    """Second formulation: q is the integer nearest to v = fl32(n * s),
+    ties upward, clipped to [-127, 127]."""
+    X = draw(Problem("n", 512, 16, 4, 0.02, 0.01, 50.0, 2))[1]
+    bits = bf16_bits(X)
+    xq, beta, _, r = oracle.quant_act(bits)
+    xf = X.float().numpy()
+    for t in range(4):
+        n = xf[t] / np.float32(r[t])
+        s = np.float32(127.0) / (np.float32(beta[t]) + np.float32(1e-5))
+        v = (n * s).astype(np.float64)
+        cand = np.stack([np.floor(v), np.floor(v) + 1])
+        d = np.abs(v[None] - cand)
+        q = np.where(d[1] <= d[0], cand[1], cand[0])
+        np.testing.assert_array_equal(xq[t], np.clip(q, -127, 127).astype(np.int8))
+
+
+def test_quant_act_scale_invariance():
+    """With eps = 0 the codes of 2^m x equal the codes of x, with and
+    without RMSNorm (norm_eps = 0 too)."""
+    X = draw(Problem("s", 512, 16, 4, 0.02, 0.01, 50.0, 9))[1]
+    for rmsnorm in (False, True):
+        base = oracle.quant_act(bf16_bits(X), rmsnorm=rmsnorm, eps=0.0, norm_eps=0.0)[0]
+        for m in (-3, 1, 5):
+            Xs = (X.float() * 2.0 ** m).to(torch.bfloat16)
+            got = oracle.quant_act(bf16_bits(Xs), rmsnorm=rmsnorm, eps=0.0,
+                                   norm_eps=0.0)[0]
+            np.testing.assert_array_equal(got, base)
+        g = np.full(512, 4.0, np.float32)
+        got = oracle.quant_act(bf16_bits(X), gain=g, rmsnorm=True, eps=0.0,
+                               norm_eps=0.0)[0]
+        np.testing.assert_array_equal(got, oracle.quant_act(
+            bf16_bits(X), rmsnorm=True, eps=0.0, norm_eps=0.0)[0])
+
+
+def test_quant_act_special_tokens():
+    K = 256
+    zero = np.zeros((1, K), np.float32)
+    const = np.full((1, K), -3.0, np.float32)
+    onehot = np.zeros((1, K), np.float32)
+    onehot[0, 77] = 2.5
+    xq, beta, S, r = oracle.quant_act(_bits(np.concatenate([zero, const, onehot])))
+    assert beta[0] == 0 and not xq[0].any() and S[0] == 0
+    assert (xq[1] == -127).all() and S[1] == -127 * K
+    assert xq[2, 77] == 127 and np.count_nonzero(xq[2]) == 1
+    # rms of a one-hot token is |v|/sqrt(K) (+eps): closed form
+    assert abs(r[2] - math.sqrt(2.5 ** 2 / K + float(np.float32(1e-5)))) < 1e-6
+
+
+def test_quant_act_supplied_rms_is_used():
+    X = draw(Problem("u", 512, 16, 3, 0.02, 0.01, 50.0, 4))[1]
+    bits = bf16_bits(X)
+    _, _, _, r = oracle.quant_act(bits)
+    a = oracle.quant_act(bits, rms_in=r)
+    b = oracle.quant_act(bits)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+    c = oracle.quant_act(bits, rms_in=r * 2)
+    np.testing.assert_array_equal(c[3], r * 2)
+
+
+# ------------------------------------------------------------------ product
+
+@pytest.mark.parametrize("T,N,K", [(1, 16, 256), (3, 48, 512), (5, 32, 768)])
+def test_int_matmul_brute_force(T, N, K):
+    wq = RNG.integers(-1, 2, size=(N, K)).astype(np.int8)
+    xq = RNG.integers(-127, 128, size=(T, K)).astype(np.int8)
+    acc = oracle.int_matmul(wq, xq)
+    np.testing.assert_array_equal(acc, xq.astype(np.int64) @ wq.astype(np.int64).T)
+
+
+def test_masked_add_identity_exhaustive():
+    """[MF] §6: accumulator += (x XOR sign) - sign where W != 0.  Over every
+    legal int8 activation and every ternary weight this equals w * x."""
+    for w in (-1, 0, 1):
+        for x in range(-127, 128):
+            got = oracle.dot_masked_add(np.array([w], np.int8), np.array([x], np.int8))
+            assert got == w * x
+
+
+def test_masked_add_matches_int_matmul():
+    wq = RNG.integers(-1, 2, size=(8, 1024)).astype(np.int8)
+    xq = RNG.integers(-127, 128, size=(2, 1024)).astype(np.int8)
+    acc = oracle.int_matmul(wq, xq)
+    for t in range(2):
+        for o in range(8):
+            assert oracle.dot_masked_add(wq[o], xq[t]) == acc[t, o]
+
+
+def test_forward_equals_float_matmul_of_dequantised_operands():
+    """Y = (X~ W~^T) beta gamma / 127 equals the fp64 product of the
+    dequantised operands (gamma W~) and (beta X~ / 127) ([MF] §2)."""
+    p = Problem("f", 512, 48, 4, 0.02, 0.01, 50.0, 6)
+    W, X = draw(p)
+    out = oracle.forward(W.numpy(), bf16_bits(X))
+    Wd = out["gamma"] * out["wq"].astype(np.float64)
+    Xd = out["beta"].astype(np.float64)[:, None] * out["xq"].astype(np.float64) / 127.0
+    np.testing.assert_allclose(out["y"], Xd @ Wd.T, rtol=1e-12, atol=1e-15)
+
+
+def test_forward_special_cases():
+    K, N = 256, 16
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    # zero weights -> y = 0
+    z = oracle.forward(np.zeros((N, K), np.float32), _bits(RNG.standard_normal((2, K))))
+    assert not z["y"].any()
+    # zero activations -> y = 0
+    z = oracle.forward(W, _bits(np.zeros((2, K))))
+    assert not z["y"].any()
+    # one-hot activation v e_j without RMSNorm: y_o = gamma * W~[o][j] * v
+    x = np.zeros((1, K), np.float32)
+    x[0, 9] = -1.5
+    g = oracle.absmean_gamma(W)
+    wq = oracle.ternarize(W, g)
+    xq, beta, _, _ = oracle.quant_act(_bits(x), rmsnorm=False)
+    y = oracle.rescale(oracle.int_matmul(wq, xq), g, beta)[0]
+    np.testing.assert_allclose(y, g * wq[:, 9] * -1.5, rtol=1e-6)
