@@ -1,0 +1,212 @@
+/*
+ * bitlinear.h -- C ABI of the B200 (sm_100a) BitNet b1.58 BitLinear library.
+ *
+ * The operation (cited as [MF]: "BitNet b1.58: Mathematical Foundations of
+ * 1.58-Bit Ternary Quantization, Absmean Scaling, and Multiplication-Free LLM
+ * Architectures", section 2 "Mathematical Formulation of the BitLinear b1.58
+ * Layer", and section 6 "Implementation Considerations and Inference
+ * Engines"):
+ *
+ *   gamma   = mean |W|                                   (absmean, per tensor)
+ *   W~      = RoundClip(W / (gamma + eps), -1, 1)          in {-1, 0, +1}
+ *   n       = RMSNorm(x)                                  (optional, per token)
+ *   beta_t  = max_k |n_tk|                                 (absmax, per token)
+ *   X~      = RoundClip(n * 127 / (beta + eps), -127, 127) int8
+ *   Y       = (X~ W~^T) * beta * gamma / 127               int32 accumulate
+ *   RoundClip(z, a, b) = max(a, min(b, floor(z + 0.5)))
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers on the current CUDA device,
+ *     owned by the caller; the library allocates nothing and keeps no
+ *     pointer after the call returns.
+ *   - All work is enqueued on `stream` (0 = legacy default stream); no entry
+ *     point synchronises except bitlinear_device_error.
+ *   - Shapes: d_out (output features, N) is a positive multiple of 16,
+ *     d_in (input features, K) a positive multiple of 256 and at most 65536,
+ *     T (tokens) is 0 .. 1048576.  T = 0 is a no-op that returns
+ *     BITLINEAR_OK and enqueues nothing.
+ *   - Alignment: W, X, Xq, packed and Y must be 16-byte aligned; gamma, beta,
+ *     rowsum, rms and gain 4-byte aligned.
+ *   - Errors: arguments are validated on the host before anything is
+ *     enqueued; a failed validation returns a status and enqueues nothing.
+ *     A failed launch returns BITLINEAR_ERR_CUDA.  A kernel that gives up a
+ *     bounded wait records BITLINEAR_ERR_TIMEOUT in a device error word read
+ *     by bitlinear_device_error.  No entry point aborts, traps or throws.
+ *   - There is no CPU fallback: without an sm_100 device every compute call
+ *     returns BITLINEAR_ERR_DEVICE.
+ *
+ * Packed ternary weight layout (this library's own format; [MF] section 6
+ * names "packed 2-bit" ternary registers without fixing an order): the
+ * d_out x d_in matrix W~ is cut into tiles of 16 rows x 256 columns stored
+ * tile-row-major (tile (rb, kb) at index rb * (d_in/256) + kb, 1 KiB each);
+ * inside a tile the 16 rows follow one another, each as 16 little-endian
+ * uint32 words; word kw of a row holds columns 16*kw .. 16*kw+15, and the
+ * 2-bit code c = W~ + 1 (0, 1 or 2; 3 never occurs) of column 16*kw + 4*s + j
+ * sits at bits 8*j + 2*s.  Thus (word >> 2s) & 0x03030303 is four int8 codes
+ * of four consecutive columns.  Size: d_out * d_in / 4 bytes.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BITLINEAR_OK = 0,
+    BITLINEAR_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, bad eps */
+    BITLINEAR_ERR_MISALIGNED = 2,        /* pointer alignment rule broken    */
+    BITLINEAR_ERR_UNSUPPORTED_SHAPE = 3, /* shape outside the rules above    */
+    BITLINEAR_ERR_CUDA = 4,              /* a CUDA runtime call failed       */
+    BITLINEAR_ERR_TIMEOUT = 5,           /* a device-side bounded wait expired */
+    BITLINEAR_ERR_DEVICE = 6             /* no usable sm_100 device          */
+} bitlinear_status;
+
+/* Output element types of bitlinear_forward. */
+#define BITLINEAR_OUT_F32 0
+#define BITLINEAR_OUT_BF16 1
+
+/* Flags of bitlinear_quant_act. */
+#define BITLINEAR_RMSNORM 1u
+
+/* Library ABI version (this header: 1). */
+int bitlinear_version(void);
+
+/* Static description of a status code.  Never NULL. */
+const char *bitlinear_status_string(int status);
+
+/* Number of uint32 words of a packed d_out x d_in matrix (d_out*d_in/16),
+ * or 0 when the shape breaks the rules above. */
+size_t bitlinear_packed_words(int64_t d_out, int64_t d_in);
+
+/* Bytes of device scratch bitlinear_pack_weights needs when it computes gamma
+ * itself (gamma_in == NULL); 0 when the shape breaks the rules above. */
+size_t bitlinear_pack_workspace_bytes(int64_t d_out, int64_t d_in);
+
+/*
+ * bitlinear_pack_weights -- absmean ternarisation and 2-bit packing
+ * ([MF] section 2, "Weight Quantization: Absmean Scaling").
+ *
+ *   W          fp32 [d_out][d_in], row-major, latent weights.
+ *   eps        the epsilon of W / (gamma + eps); must be finite and >= 0.
+ *   gamma_in   device fp32 scalar, or NULL.  When given it is used as gamma
+ *              and no reduction runs; when NULL gamma = mean|W| is computed
+ *              (sum of |W| in double over a fixed, deterministic two-stage
+ *              reduction, divided by d_out*d_in and rounded once to fp32).
+ *   workspace  device scratch of bitlinear_pack_workspace_bytes() bytes,
+ *              8-byte aligned; needed only when gamma_in == NULL.
+ *   packed     out: bitlinear_packed_words() uint32 words, layout above.
+ *   gamma_out  out: device fp32 scalar, the gamma used (may equal gamma_in).
+ * W / (gamma + eps) is one binary32 division; floor(z + 0.5) is then taken
+ * exactly and clipped to [-1, 1].  NaN or infinite weights give unspecified
+ * codes (never code 3).
+ */
+int bitlinear_pack_weights(const float *W, int64_t d_out, int64_t d_in, float eps,
+                           const float *gamma_in, void *workspace,
+                           size_t workspace_bytes, uint32_t *packed,
+                           float *gamma_out, cudaStream_t stream);
+
+/*
+ * bitlinear_quant_act -- fused RMSNorm + per-token absmax int8 quantisation
+ * ([MF] section 2, "Activation Quantization: Absmax Scaling"; beta taken per
+ * token; Q_b - 1 = 127 is both multiplier and clip bound).
+ *
+ *   X          bf16 [T][d_in], row-major, as raw uint16 bit patterns.
+ *   norm_gain  fp32 [d_in] RMSNorm gain, or NULL for all ones.
+ *   flags      BITLINEAR_RMSNORM to normalise first, 0 to quantise X as is.
+ *   eps        the epsilon of 127 / (beta + eps); finite, >= 0.
+ *   norm_eps   the epsilon inside the RMS: rms = sqrt(mean(x^2) + norm_eps),
+ *              formed in double and rounded once to fp32; finite, >= 0.
+ *   rms_in     fp32 [T] per-token rms to use instead of computing it, or NULL.
+ *   Xq         out: int8 [T][d_in] activation codes in [-127, 127].
+ *   beta       out: fp32 [T] per-token absmax of the (normalised) row.
+ *   rowsum     out: int32 [T] sum of each row of Xq (consumed by forward).
+ *   rms_out    out: fp32 [T] rms used, or NULL.
+ * n = x / rms is one binary32 division (times the gain, one multiplication);
+ * the scale 127 / (beta + eps) is one binary32 addition and one division,
+ * applied with one multiplication; floor(v + 0.5) is then taken exactly.
+ */
+int bitlinear_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
+                        const float *norm_gain, uint32_t flags, float eps,
+                        float norm_eps, const float *rms_in, int8_t *Xq,
+                        float *beta, int32_t *rowsum, float *rms_out,
+                        cudaStream_t stream);
+
+/*
+ * bitlinear_forward -- the multiplier-free ternary x int8 product with int32
+ * accumulation and the fused rescale ([MF] section 2, "The Linear
+ * Transformation and Rescaling"; section 6, scale-factor fusion):
+ *
+ *   acc[t][o] = sum_k W~[o][k] * Xq[t][k]                 exact int32
+ *   Y[t][o]   = acc[t][o] * (gamma * beta[t] / 127)        one fp32 multiply
+ *
+ * with gamma * beta[t] / 127 formed as one binary32 multiplication and one
+ * division.  The kernels multiply the offset codes c = W~ + 1 and subtract
+ * rowsum[t]; the result is the same exact integer.
+ *
+ *   packed     packed ternary weights (layout above), d_out x d_in.
+ *   gamma      device fp32 scalar.
+ *   Xq, beta, rowsum   as written by bitlinear_quant_act for these T rows.
+ *   Y          out: [T][d_out] row-major, fp32 or bf16 (round to nearest even)
+ *              per out_dtype.
+ *   acc_out    out: int32 [T][d_out] raw accumulators, or NULL.
+ * T <= 16 runs the decode GEMV (register-decoded ternary weights, warp-level
+ * int8 tensor-core MMA); T > 16 runs the prefill GEMM (TMA-staged packed
+ * tiles expanded into tensor memory, tcgen05 int8 MMA, TMEM accumulator).
+ */
+int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
+                      int64_t d_in, const int8_t *Xq, const float *beta,
+                      const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                      int32_t *acc_out, cudaStream_t stream);
+
+/*
+ * bitlinear_linear -- the whole BitLinear forward from bf16 activations:
+ * bitlinear_quant_act (with rms computed, rms_in = NULL) followed by
+ * bitlinear_forward, with the same arguments, meaning and results as those
+ * two calls made back to back ([MF] section 2, all three parts).  Xq, beta
+ * and rowsum are caller-owned intermediates of T*d_in, T and T elements.
+ * The product kernel is launched as a programmatic dependent of the
+ * quantiser so that its weight stream overlaps the quantisation; it reads
+ * the codes only after the quantiser has finished.
+ */
+int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
+                     int64_t d_in, const uint16_t *X, int64_t T,
+                     const float *norm_gain, uint32_t flags, float eps,
+                     float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
+                     void *Y, int out_dtype, cudaStream_t stream);
+
+/*
+ * bitlinear_device_error -- synchronises `stream`, then reads the device
+ * error word that kernels set when a bounded wait gives up.  Returns
+ * BITLINEAR_OK when the word is clear, BITLINEAR_ERR_TIMEOUT when a wait
+ * expired, BITLINEAR_ERR_CUDA when the synchronisation itself failed.  With
+ * clear != 0 the word is reset to zero afterwards.
+ */
+int bitlinear_device_error(cudaStream_t stream, int clear);
+
+/*
+ * bitlinear_set_wait_limit_ns -- the time after which a kernel's bounded wait
+ * on an mbarrier gives up (default 2e9 ns).  Applies to launches made after
+ * the call on the current device.  limit_ns must be in [1e3, 6e10].
+ */
+int bitlinear_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * bitlinear_wait_probe -- launches one CTA that waits, through the same
+ * bounded-wait routine the GEMM uses, on an mbarrier that nothing ever
+ * arrives on.  After limit_ns the wait gives up and the kernel records
+ * BITLINEAR_ERR_TIMEOUT in the device error word and returns.  Exists so the
+ * timeout path can be tested without stalling any real pipeline.
+ */
+int bitlinear_wait_probe(uint64_t limit_ns, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

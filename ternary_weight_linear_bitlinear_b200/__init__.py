@@ -1,0 +1,226 @@
+"""Python binding of the sm_100a BitNet b1.58 BitLinear library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libbitlinear.so`` (C ABI in ``include/bitlinear.h``).  PyTorch
+provides device memory and the current CUDA stream.  There is no CPU
+fallback: if the library is missing, or no sm_100 device is present, every
+call raises.
+
+The operation ("BitNet b1.58: Mathematical Foundations of 1.58-Bit Ternary
+Quantization, Absmean Scaling, and Multiplication-Free LLM Architectures",
+section 2): gamma = mean|W|, W~ = RoundClip(W/(gamma+eps), -1, 1); per-token
+beta = max|RMSNorm(x)|, X~ = RoundClip(x 127/(beta+eps), -127, 127);
+Y = (X~ W~^T) beta gamma / 127 with int32 accumulation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbitlinear.so")
+
+OUT_F32 = 0
+OUT_BF16 = 1
+RMSNORM = 1
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_MISALIGNED = 2
+ERR_UNSUPPORTED_SHAPE = 3
+ERR_CUDA = 4
+ERR_TIMEOUT = 5
+ERR_DEVICE = 6
+
+# Every exported entry point with (restype, argtypes), as in bitlinear.h.
+_vp, _i64, _f32, _u32, _int = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float,
+                               ctypes.c_uint32, ctypes.c_int)
+SIGNATURES = {
+    "bitlinear_version": (_int, []),
+    "bitlinear_status_string": (ctypes.c_char_p, [_int]),
+    "bitlinear_packed_words": (ctypes.c_size_t, [_i64, _i64]),
+    "bitlinear_pack_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "bitlinear_pack_weights": (_int, [_vp, _i64, _i64, _f32, _vp, _vp, ctypes.c_size_t,
+                                      _vp, _vp, _vp]),
+    "bitlinear_quant_act": (_int, [_vp, _i64, _i64, _vp, _u32, _f32, _f32, _vp, _vp, _vp,
+                                   _vp, _vp, _vp]),
+    "bitlinear_forward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int,
+                                 _vp, _vp]),
+    "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
+                                _vp, _vp, _vp, _vp, _int, _vp]),
+    "bitlinear_device_error": (_int, [_vp, _int]),
+    "bitlinear_set_wait_limit_ns": (_int, [ctypes.c_uint64]),
+    "bitlinear_wait_probe": (_int, [ctypes.c_uint64, _vp]),
+}
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libbitlinear.so is not built (run python -m "
+                "ternary_weight_linear_bitlinear_b200.build); there is no fallback")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().bitlinear_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise BitLinearError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+@dataclass
+class PackedTernary:
+    """Packed ternary weights of one BitLinear (layout in bitlinear.h)."""
+    packed: torch.Tensor    # int32 [d_out * d_in / 16] (uint32 bit patterns)
+    gamma: torch.Tensor     # float32 [1]
+    d_out: int
+    d_in: int
+
+
+def packed_words(d_out: int, d_in: int) -> int:
+    return int(lib().bitlinear_packed_words(d_out, d_in))
+
+
+def pack_workspace_bytes(d_out: int, d_in: int) -> int:
+    return int(lib().bitlinear_pack_workspace_bytes(d_out, d_in))
+
+
+def pack_weights(W: torch.Tensor, eps: float = 1e-5, gamma: torch.Tensor = None,
+                 out: PackedTernary = None) -> PackedTernary:
+    """Absmean-ternarise and pack fp32 latent weights [d_out][d_in]."""
+    _need(W, torch.float32, "W")
+    d_out, d_in = W.shape
+    if out is None:
+        n = packed_words(d_out, d_in)
+        if n == 0:
+            _check(ERR_UNSUPPORTED_SHAPE, "pack_weights")
+        out = PackedTernary(torch.empty(n, dtype=torch.int32, device=W.device),
+                            torch.empty(1, dtype=torch.float32, device=W.device), d_out, d_in)
+    ws = None
+    if gamma is None:
+        ws = torch.empty(max(pack_workspace_bytes(d_out, d_in), 8), dtype=torch.uint8,
+                         device=W.device)
+    else:
+        _need(gamma, torch.float32, "gamma")
+    st = lib().bitlinear_pack_weights(_ptr(W), d_out, d_in, eps, _ptr(gamma), _ptr(ws),
+                                      0 if ws is None else ws.numel(), _ptr(out.packed),
+                                      _ptr(out.gamma), _stream())
+    _check(st, "bitlinear_pack_weights")
+    return out
+
+
+def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
+              eps: float = 1e-5, norm_eps: float = 1e-5, rms: torch.Tensor = None):
+    """Fused RMSNorm + per-token absmax int8 codes of bf16 X [T][d_in].
+
+    Returns (Xq int8 [T][d_in], beta f32 [T], rowsum int32 [T], rms f32 [T]).
+    """
+    _need(X, torch.bfloat16, "X")
+    T, d_in = X.shape
+    dev = X.device
+    Xq = torch.empty((T, d_in), dtype=torch.int8, device=dev)
+    beta = torch.empty(T, dtype=torch.float32, device=dev)
+    rowsum = torch.empty(T, dtype=torch.int32, device=dev)
+    rms_out = torch.empty(T, dtype=torch.float32, device=dev)
+    if gain is not None:
+        _need(gain, torch.float32, "gain")
+    if rms is not None:
+        _need(rms, torch.float32, "rms")
+    st = lib().bitlinear_quant_act(_ptr(X), T, d_in, _ptr(gain), RMSNORM if rmsnorm else 0,
+                                   eps, norm_eps, _ptr(rms), _ptr(Xq), _ptr(beta),
+                                   _ptr(rowsum), _ptr(rms_out), _stream())
+    _check(st, "bitlinear_quant_act")
+    return Xq, beta, rowsum, rms_out
+
+
+def forward(w: PackedTernary, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
+            out_dtype=torch.float32, want_acc: bool = False, out: torch.Tensor = None):
+    """Y = (X~ W~^T) gamma beta / 127; returns Y (and the int32 acc if asked)."""
+    _need(Xq, torch.int8, "Xq")
+    T = Xq.shape[0]
+    dev = Xq.device
+    if out is None:
+        out = torch.empty((T, w.d_out), dtype=out_dtype, device=dev)
+    od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
+    acc = torch.empty((T, w.d_out), dtype=torch.int32, device=dev) if want_acc else None
+    st = lib().bitlinear_forward(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq),
+                                 _ptr(beta), _ptr(rowsum), T, _ptr(out), od, _ptr(acc),
+                                 _stream())
+    _check(st, "bitlinear_forward")
+    return (out, acc) if want_acc else out
+
+
+def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
+           eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.float32,
+           out: torch.Tensor = None, scratch=None):
+    """The whole BitLinear forward from bf16 X: quantise, then product."""
+    _need(X, torch.bfloat16, "X")
+    T = X.shape[0]
+    dev = X.device
+    if scratch is None:
+        scratch = (torch.empty((T, w.d_in), dtype=torch.int8, device=dev),
+                   torch.empty(T, dtype=torch.float32, device=dev),
+                   torch.empty(T, dtype=torch.int32, device=dev))
+    Xq, beta, rowsum = scratch
+    if out is None:
+        out = torch.empty((T, w.d_out), dtype=out_dtype, device=dev)
+    od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
+    st = lib().bitlinear_linear(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(X), T,
+                                _ptr(gain), RMSNORM if rmsnorm else 0, eps, norm_eps,
+                                _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
+    _check(st, "bitlinear_linear")
+    return out
+
+
+def device_error(clear: bool = True) -> int:
+    """Synchronise the current stream and return the device error status."""
+    return int(lib().bitlinear_device_error(_stream(), 1 if clear else 0))
+
+
+def set_wait_limit_ns(limit_ns: int):
+    _check(lib().bitlinear_set_wait_limit_ns(int(limit_ns)), "bitlinear_set_wait_limit_ns")
+
+
+def wait_probe(limit_ns: int):
+    _check(lib().bitlinear_wait_probe(int(limit_ns), _stream()), "bitlinear_wait_probe")

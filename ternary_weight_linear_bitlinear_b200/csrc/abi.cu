@@ -1,0 +1,203 @@
+// abi.cu -- the library's C entry points: validation, kernel selection,
+// device error word, bounded-wait configuration.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "bitlinear.h"
+#include "common.cuh"
+
+namespace bl {
+
+bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
+                                  const float *norm_gain, uint32_t flags, float eps,
+                                  float norm_eps, const float *rms_in, int8_t *Xq, float *beta,
+                                  int32_t *rowsum, float *rms_out, cudaStream_t stream);
+bitlinear_status launch_gemv(const uint32_t *packed, const float *gamma, int64_t d_out,
+                             int64_t d_in, const int8_t *Xq, const float *beta,
+                             const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                             int32_t *acc_out, bool pdl, cudaStream_t stream);
+bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                int64_t d_in, const int8_t *Xq, const float *beta,
+                                const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                                int32_t *acc_out, cudaStream_t stream);
+
+// Device error word: set by kernels whose bounded waits expire.
+__device__ uint32_t g_error_word;
+
+__global__ void wait_probe_kernel(DeviceCtx ctx) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        mbar_init_fence();
+        // Nothing ever arrives: the wait must give up after ctx.wait_ns.
+        mbar_wait_bounded(smem_u32(&bar), 0, ctx);
+    }
+}
+
+namespace {
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+std::mutex g_mu;
+uint32_t *g_err_ptr[kMaxDevices];
+uint64_t g_wait_ns[kMaxDevices];
+int g_dev_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 unusable
+}  // namespace
+
+bitlinear_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return BITLINEAR_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_dev_ok[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return BITLINEAR_ERR_DEVICE;
+        g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    return g_dev_ok[dev] == 1 ? BITLINEAR_OK : BITLINEAR_ERR_DEVICE;
+}
+
+bitlinear_status get_ctx(DeviceCtx *ctx) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return BITLINEAR_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+        g_err_ptr[dev] = static_cast<uint32_t *>(p);
+    }
+    ctx->err = g_err_ptr[dev];
+    ctx->wait_ns = g_wait_ns[dev] ? g_wait_ns[dev] : kDefaultWaitNs;
+    return BITLINEAR_OK;
+}
+
+static bitlinear_status validate_forward(const uint32_t *packed, const float *gamma,
+                                         int64_t d_out, int64_t d_in, int64_t T, void *Y,
+                                         int out_dtype, int32_t *acc_out) {
+    if (T < 0 || T > (1 << 20)) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (d_out <= 0 || d_out % 16 || d_out > (1 << 22)) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (d_in <= 0 || d_in % 256 || d_in > 65536) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (out_dtype != BITLINEAR_OUT_F32 && out_dtype != BITLINEAR_OUT_BF16)
+        return BITLINEAR_ERR_INVALID_ARG;
+    if (T == 0) return BITLINEAR_OK;  // empty problem: nothing to check or enqueue
+    if (!packed || !gamma || !Y) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(packed, 16) || !aligned(gamma, 4) || !aligned(Y, 16) ||
+        (acc_out && !aligned(acc_out, 16)))
+        return BITLINEAR_ERR_MISALIGNED;
+    return BITLINEAR_OK;
+}
+
+static bitlinear_status dispatch_forward(const uint32_t *packed, const float *gamma,
+                                         int64_t d_out, int64_t d_in, const int8_t *Xq,
+                                         const float *beta, const int32_t *rowsum, int64_t T,
+                                         void *Y, int out_dtype, int32_t *acc_out, bool pdl,
+                                         cudaStream_t stream) {
+    if (T <= 16)
+        return launch_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
+                           acc_out, pdl, stream);
+    return launch_gemm_tc(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype, acc_out,
+                          stream);
+}
+
+}  // namespace bl
+
+using namespace bl;
+
+extern "C" int bitlinear_version(void) { return 1; }
+
+extern "C" const char *bitlinear_status_string(int status) {
+    switch (status) {
+        case BITLINEAR_OK: return "ok";
+        case BITLINEAR_ERR_INVALID_ARG: return "invalid argument";
+        case BITLINEAR_ERR_MISALIGNED: return "misaligned pointer";
+        case BITLINEAR_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case BITLINEAR_ERR_CUDA: return "CUDA runtime error";
+        case BITLINEAR_ERR_TIMEOUT: return "device-side bounded wait expired";
+        case BITLINEAR_ERR_DEVICE: return "no usable sm_100 device";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                 int64_t d_in, const int8_t *Xq, const float *beta,
+                                 const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                                 int32_t *acc_out, cudaStream_t stream) {
+    bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, acc_out);
+    if (st != BITLINEAR_OK) return st;
+    if (T == 0) return BITLINEAR_OK;
+    if (!Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4))
+        return BITLINEAR_ERR_MISALIGNED;
+    st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
+                            acc_out, false, stream);
+}
+
+extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                int64_t d_in, const uint16_t *X, int64_t T,
+                                const float *norm_gain, uint32_t flags, float eps, float norm_eps,
+                                int8_t *Xq, float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                cudaStream_t stream) {
+    bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, nullptr);
+    if (st != BITLINEAR_OK) return st;
+    if (flags & ~BITLINEAR_RMSNORM) return BITLINEAR_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !std::isfinite(eps) || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps))
+        return BITLINEAR_ERR_INVALID_ARG;
+    if (T == 0) return BITLINEAR_OK;
+    if (!X || !Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4) ||
+        (norm_gain && !aligned(norm_gain, 4)))
+        return BITLINEAR_ERR_MISALIGNED;
+    st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    st = launch_quant_act(X, T, d_in, norm_gain, flags, eps, norm_eps, nullptr, Xq, beta, rowsum,
+                          nullptr, stream);
+    if (st != BITLINEAR_OK) return st;
+    // The product is launched as a programmatic dependent of the quantiser:
+    // it may start streaming weights while the codes are still being written
+    // and waits for them before reading.
+    return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
+                            nullptr, true, stream);
+}
+
+extern "C" int bitlinear_device_error(cudaStream_t stream, int clear) {
+    DeviceCtx ctx;
+    bitlinear_status st = get_ctx(&ctx);
+    if (st != BITLINEAR_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, ctx.err, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return BITLINEAR_ERR_CUDA;
+    if (clear && word) {
+        const uint32_t zero = 0;
+        if (cudaMemcpy(ctx.err, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+            return BITLINEAR_ERR_CUDA;
+    }
+    return (word & kErrTimeout) ? BITLINEAR_ERR_TIMEOUT : BITLINEAR_OK;
+}
+
+extern "C" int bitlinear_set_wait_limit_ns(uint64_t limit_ns) {
+    if (limit_ns < 1000ull || limit_ns > 60000000000ull) return BITLINEAR_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return BITLINEAR_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_wait_ns[dev] = limit_ns;
+    return BITLINEAR_OK;
+}
+
+extern "C" int bitlinear_wait_probe(uint64_t limit_ns, cudaStream_t stream) {
+    if (limit_ns < 1000ull || limit_ns > 60000000000ull) return BITLINEAR_ERR_INVALID_ARG;
+    bitlinear_status st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    DeviceCtx ctx;
+    st = get_ctx(&ctx);
+    if (st != BITLINEAR_OK) return st;
+    ctx.wait_ns = limit_ns;
+    wait_probe_kernel<<<1, 32, 0, stream>>>(ctx);
+    return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}

@@ -1,0 +1,108 @@
+// common.cuh -- device helpers shared by the library's kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "bitlinear.h"
+
+namespace bl {
+
+// Bits of the device error word.
+constexpr uint32_t kErrTimeout = 1u;
+
+// Kernel-side configuration passed by value to every launch.
+struct DeviceCtx {
+    uint32_t *err;        // device error word (see bitlinear_device_error)
+    uint64_t wait_ns;     // bounded-wait limit
+};
+
+// Host side: error-word address and wait limit for the current device.
+bitlinear_status get_ctx(DeviceCtx *ctx);
+// Host side: check the current device is sm_100.
+bitlinear_status check_device();
+
+inline bool aligned(const void *p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+// ------------------------------------------------------------- rounding --
+// RoundClip's floor(z + 0.5), evaluated exactly on a binary32 z: with
+// f = floor(z), z - f is exact whenever it can be near 0.5 (Sterbenz for
+// |z| >= 1; plain representability for |z| < 1), so the comparison decides
+// the same integer as the exact sum.
+__device__ __forceinline__ float round_half_up_exact(float z) {
+    float f = floorf(z);
+    float frac = __fsub_rn(z, f);
+    return (frac >= 0.5f) ? __fadd_rn(f, 1.0f) : f;
+}
+
+// -------------------------------------------------------------- timers ---
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ------------------------------------------------------------ mbarrier ---
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait for the phase of parity `parity` to complete.  Returns false
+// (after recording kErrTimeout) when `limit_ns` elapses first.  Never traps.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  const DeviceCtx &ctx) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > ctx.wait_ns) {
+            atomicOr(ctx.err, kErrTimeout);
+            return false;
+        }
+    }
+}
+
+// ------------------------------------------------- programmatic launch ---
+// Dependent-launch controls (no-ops when the launch was not programmatic).
+__device__ __forceinline__ void pdl_wait_primary() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace bl

@@ -1,0 +1,153 @@
+// pack.cu -- absmean scale and 2-bit ternary packing of latent weights.
+//
+// "BitNet b1.58: Mathematical Foundations of 1.58-Bit Ternary Quantization,
+// Absmean Scaling, and Multiplication-Free LLM Architectures", section 2,
+// "Weight Quantization: Absmean Scaling": gamma = mean |W| over the tensor,
+// W~ = RoundClip(W / (gamma + eps), -1, 1).  Section 6 (Weight Unpacking)
+// names 2-bit packed ternary registers; the tile layout is documented in
+// bitlinear.h.
+//
+// HBM-bound streaming kernels: the reduction reads 4 B per weight, the
+// packer reads 4 B and writes 0.25 B per weight.  Both run offline, once per
+// weight matrix.
+#include <cmath>
+#include <cstdint>
+
+#include "bitlinear.h"
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kRedThreads = 256;
+constexpr int kRedMaxBlocks = 148 * 8;
+
+__device__ __forceinline__ double block_sum_f64(double v, double *sh) {
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) sh[warp] = v;
+    __syncthreads();
+    double r = 0.0;
+    if (threadIdx.x == 0) {
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += sh[w];
+    }
+    __syncthreads();
+    return r;  // valid in thread 0
+}
+
+// Stage 1: each block sums |W| over a fixed grid-stride set of float4s in
+// double and writes one partial.  The order is fixed by (grid, block) sizes,
+// so the result is deterministic for a given shape.
+__global__ void __launch_bounds__(kRedThreads)
+absmean_partial_kernel(const float4 *__restrict__ W4, int64_t n4, double *partial) {
+    __shared__ double sh[kRedThreads / 32];
+    double acc = 0.0;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+        float4 v = __ldg(W4 + i);
+        acc += fabs((double)v.x) + fabs((double)v.y) + fabs((double)v.z) + fabs((double)v.w);
+    }
+    double s = block_sum_f64(acc, sh);
+    if (threadIdx.x == 0) partial[blockIdx.x] = s;
+}
+
+// Stage 2: one block sums the partials in a fixed order; gamma rounded once.
+__global__ void __launch_bounds__(kRedThreads)
+absmean_final_kernel(const double *partial, int nparts, double count, float *gamma) {
+    __shared__ double sh[kRedThreads / 32];
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < nparts; i += blockDim.x) acc += partial[i];
+    double s = block_sum_f64(acc, sh);
+    if (threadIdx.x == 0) *gamma = (float)(s / count);
+}
+
+// One thread per packed word: 16 consecutive weights of one row.
+__global__ void __launch_bounds__(256)
+pack_kernel(const float *__restrict__ W, int64_t d_out, int64_t d_in, float eps,
+            const float *__restrict__ gamma_ptr, uint32_t *__restrict__ packed,
+            float *gamma_out) {
+    const float gamma = *gamma_ptr;
+    const float den = __fadd_rn(gamma, eps);
+    const int64_t tiles_per_row = d_in >> 8;
+    const int64_t nwords = (d_out * d_in) >> 4;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    if (blockIdx.x == 0 && threadIdx.x == 0 && gamma_out != gamma_ptr) *gamma_out = gamma;
+    for (int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < nwords; wi += stride) {
+        const int64_t tile = wi >> 8;
+        const int within = (int)(wi & 255);
+        const int r = within >> 4, kw = within & 15;
+        const int64_t rb = tile / tiles_per_row, kb = tile - rb * tiles_per_row;
+        const int64_t o = rb * 16 + r;
+        const int64_t k0 = kb * 256 + kw * 16;
+        const float4 *src = reinterpret_cast<const float4 *>(W + o * d_in + k0);
+        uint32_t word = 0;
+        #pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            float4 v = __ldg(src + s);
+            float e[4] = {v.x, v.y, v.z, v.w};
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float q = round_half_up_exact(__fdiv_rn(e[j], den));
+                q = fminf(fmaxf(q, -1.0f), 1.0f);
+                const uint32_t c = (uint32_t)((int)q + 1) & 3u;
+                word |= c << (8 * j + 2 * s);
+            }
+        }
+        packed[wi] = word;
+    }
+}
+
+}  // namespace bl
+
+using namespace bl;
+
+extern "C" size_t bitlinear_packed_words(int64_t d_out, int64_t d_in) {
+    if (d_out <= 0 || d_in <= 0 || d_out % 16 || d_in % 256 || d_in > 65536) return 0;
+    return (size_t)(d_out * d_in / 16);
+}
+
+extern "C" size_t bitlinear_pack_workspace_bytes(int64_t d_out, int64_t d_in) {
+    if (bitlinear_packed_words(d_out, d_in) == 0) return 0;
+    return (size_t)kRedMaxBlocks * sizeof(double);
+}
+
+extern "C" int bitlinear_pack_weights(const float *W, int64_t d_out, int64_t d_in, float eps,
+                                      const float *gamma_in, void *workspace,
+                                      size_t workspace_bytes, uint32_t *packed,
+                                      float *gamma_out, cudaStream_t stream) {
+    if (!W || !packed || !gamma_out) return BITLINEAR_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return BITLINEAR_ERR_INVALID_ARG;
+    if (bitlinear_packed_words(d_out, d_in) == 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (!gamma_in) {
+        if (!workspace) return BITLINEAR_ERR_INVALID_ARG;
+        if (workspace_bytes < bitlinear_pack_workspace_bytes(d_out, d_in))
+            return BITLINEAR_ERR_INVALID_ARG;
+        if (!aligned(workspace, 8)) return BITLINEAR_ERR_MISALIGNED;
+    } else if (!aligned(gamma_in, 4)) {
+        return BITLINEAR_ERR_MISALIGNED;
+    }
+    if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(gamma_out, 4))
+        return BITLINEAR_ERR_MISALIGNED;
+    bitlinear_status st = check_device();
+    if (st != BITLINEAR_OK) return st;
+
+    const int64_t n = d_out * d_in;
+    const float *gptr = gamma_in;
+    if (!gamma_in) {
+        const int64_t n4 = n / 4;
+        int blocks = (int)((n4 + kRedThreads * 8 - 1) / (kRedThreads * 8));
+        if (blocks > kRedMaxBlocks) blocks = kRedMaxBlocks;
+        if (blocks < 1) blocks = 1;
+        double *partial = static_cast<double *>(workspace);
+        absmean_partial_kernel<<<blocks, kRedThreads, 0, stream>>>(
+            reinterpret_cast<const float4 *>(W), n4, partial);
+        absmean_final_kernel<<<1, kRedThreads, 0, stream>>>(partial, blocks, (double)n,
+                                                             gamma_out);
+        gptr = gamma_out;
+    }
+    const int64_t nwords = n / 16;
+    int64_t pblocks = (nwords + 255) / 256;
+    if (pblocks > 148 * 16) pblocks = 148 * 16;
+    pack_kernel<<<(int)pblocks, 256, 0, stream>>>(W, d_out, d_in, eps, gptr, packed, gamma_out);
+    return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}

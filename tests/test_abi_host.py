@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI: no GPU needed, no kernel launched.
+
+The library must load, export every entry point the header declares, and
+reject bad arguments on the host before touching a device.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import ternary_weight_linear_bitlinear_b200 as bl
+from ternary_weight_linear_bitlinear_b200 import build as blbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    blbuild.build()
+    return bl.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitlinear_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for must in ("bitlinear_pack_weights", "bitlinear_quant_act", "bitlinear_forward"):
+        assert must in names
+    assert set(names) == set(bl.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", bl.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (bitlinear_\w+)$", out, flags=re.M))
+    missing = set(declared_functions()) - exported
+    assert not missing, missing
+    for name in declared_functions():
+        assert getattr(lib, name) is not None
+
+
+def test_version_and_status_strings(lib):
+    assert lib.bitlinear_version() == 1
+    for code in range(0, 7):
+        s = bl.status_string(code)
+        assert s and s != "unknown status"
+    assert bl.status_string(99) == "unknown status"
+
+
+def test_packed_sizes(lib):
+    assert bl.packed_words(6912, 2560) == 6912 * 2560 // 16
+    assert bl.packed_words(11008, 4096) * 4 == 11272192
+    assert bl.packed_words(4096, 11008) * 4 == 11272192
+    assert bl.packed_words(16, 256) == 256
+    assert bl.packed_words(15, 256) == 0          # d_out not a multiple of 16
+    assert bl.packed_words(16, 128) == 0          # d_in not a multiple of 256
+    assert bl.packed_words(16, 65536 + 256) == 0  # d_in too large
+    assert bl.pack_workspace_bytes(6912, 2560) > 0
+    assert bl.pack_workspace_bytes(16, 100) == 0
+
+
+P = ctypes.c_void_p
+S0 = ctypes.c_void_p(0)
+
+
+def _fwd(lib, packed=0x10000, gamma=0x20000, d_out=64, d_in=256, xq=0x30000, beta=0x40000,
+         rowsum=0x50000, T=4, Y=0x60000, od=0, acc=None):
+    return lib.bitlinear_forward(P(packed), P(gamma), d_out, d_in, P(xq), P(beta), P(rowsum), T,
+                                 P(Y), od, P(acc) if acc else None, S0)
+
+
+def test_forward_validation(lib):
+    assert _fwd(lib, packed=0) == bl.ERR_INVALID_ARG
+    assert _fwd(lib, Y=0) == bl.ERR_INVALID_ARG
+    assert _fwd(lib, d_in=200) == bl.ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, d_out=24) == bl.ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, T=-1) == bl.ERR_UNSUPPORTED_SHAPE
+    assert _fwd(lib, od=7) == bl.ERR_INVALID_ARG
+    assert _fwd(lib, packed=0x10008) == bl.ERR_MISALIGNED
+    assert _fwd(lib, Y=0x60004) == bl.ERR_MISALIGNED
+    assert _fwd(lib, xq=0x30001) == bl.ERR_MISALIGNED
+    assert _fwd(lib, beta=0x40002) == bl.ERR_MISALIGNED
+    # T = 0 is an empty problem: success, nothing enqueued, no device touched.
+    assert _fwd(lib, T=0, xq=0, beta=0, rowsum=0) == bl.OK
+
+
+def test_quant_act_validation(lib):
+    q = lib.bitlinear_quant_act
+    args = dict(X=0x10000, T=2, d_in=512, gain=None, flags=1, eps=1e-5, neps=1e-5, rms=None,
+                xq=0x20000, beta=0x30000, rs=0x40000, rmso=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return q(P(a["X"]), a["T"], a["d_in"], P(a["gain"]) if a["gain"] else None, a["flags"],
+                 a["eps"], a["neps"], P(a["rms"]) if a["rms"] else None, P(a["xq"]),
+                 P(a["beta"]), P(a["rs"]), P(a["rmso"]) if a["rmso"] else None, S0)
+
+    assert call(X=0) == bl.ERR_INVALID_ARG
+    assert call(flags=4) == bl.ERR_INVALID_ARG
+    assert call(eps=float("nan")) == bl.ERR_INVALID_ARG
+    assert call(neps=-1.0) == bl.ERR_INVALID_ARG
+    assert call(d_in=300) == bl.ERR_UNSUPPORTED_SHAPE
+    assert call(X=0x10002) == bl.ERR_MISALIGNED
+    assert call(gain=0x50001) == bl.ERR_MISALIGNED
+    assert call(T=0, X=0, xq=0) == bl.OK
+
+
+def test_pack_validation(lib):
+    p = lib.bitlinear_pack_weights
+    ws = bl.pack_workspace_bytes(64, 256)
+    assert p(None, 64, 256, 1e-5, None, P(0x1000), ws, P(0x2000), P(0x3000), S0) == bl.ERR_INVALID_ARG
+    assert p(P(0x1000), 64, 100, 1e-5, None, P(0x1000), ws, P(0x2000), P(0x3000), S0) == bl.ERR_UNSUPPORTED_SHAPE
+    assert p(P(0x1000), 64, 256, -1.0, None, P(0x1000), ws, P(0x2000), P(0x3000), S0) == bl.ERR_INVALID_ARG
+    # Computing gamma needs a large enough workspace.
+    assert p(P(0x1000), 64, 256, 1e-5, None, None, 0, P(0x2000), P(0x3000), S0) == bl.ERR_INVALID_ARG
+    assert p(P(0x1000), 64, 256, 1e-5, None, P(0x1000), ws - 8, P(0x2000), P(0x3000), S0) == bl.ERR_INVALID_ARG
+    assert p(P(0x1004), 64, 256, 1e-5, None, P(0x1000), ws, P(0x2000), P(0x3000), S0) == bl.ERR_MISALIGNED
+
+
+def test_wait_limit_validation(lib):
+    assert lib.bitlinear_set_wait_limit_ns(10) == bl.ERR_INVALID_ARG
+    assert lib.bitlinear_wait_probe(10, S0) == bl.ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_fails_loudly(lib):
+    """Without an sm_100 GPU a valid compute call reports ERR_DEVICE: there
+    is no CPU fallback behind the C ABI."""
+    assert _fwd(lib) == bl.ERR_DEVICE
+    with pytest.raises((RuntimeError, TypeError)):
+        bl.quant_act(torch.zeros(2, 256, dtype=torch.bfloat16))

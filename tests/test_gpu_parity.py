@@ -1,0 +1,264 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bars: packed codes, activation codes, row sums and int32 accumulators
+bit-exact; gamma and rms within 1e-6 relative; fp32 outputs within
+1e-5 * max(|y|, scale_t) and bf16 outputs within 1e-2 * max(|y|, scale_t),
+where scale_t = gamma beta_t / 127 is one integer step of the output (the
+floor keeps a relative bound meaningful at acc = 0).
+
+Inputs only flow oracle -> GPU: where integer codes are compared, the GPU is
+handed the oracle's gamma / rms (the GPU's own values are checked separately
+against the oracle's to 1e-6), so a last-bit difference in a reduction can
+not flip a code and nothing computed on the GPU enters the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ternary_weight_linear_bitlinear_b200 as bl
+from ternary_weight_linear_bitlinear_b200 import build as blbuild
+from workloads import Problem, bf16_bits, draw
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-5
+NORM_EPS = 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    blbuild.build()
+    bl.lib()
+    torch.cuda.init()
+    yield
+    assert bl.device_error(clear=True) == bl.OK
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+def u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def to_dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.to(dev()) if dtype is None else t.to(dev(), dtype)
+
+
+def oracle_side(W, X, rmsnorm=True, gain=None):
+    """Everything the oracle computes for (W, X), from W and X alone."""
+    Wn = W.numpy()
+    g = oracle.absmean_gamma(Wn)
+    wq = oracle.ternarize(Wn, g, EPS)
+    xb = bf16_bits(X)
+    xq, beta, rowsum, rms = oracle.quant_act(xb, gain=gain, rmsnorm=rmsnorm, eps=EPS,
+                                             norm_eps=NORM_EPS)
+    return dict(gamma=g, wq=wq, xq=xq, beta=beta, rowsum=rowsum, rms=rms, xb=xb)
+
+
+def check_y(y_gpu, acc_ref, gamma, beta, out_bf16, rows=None):
+    """Compare GPU outputs with the oracle's float64 rescale."""
+    y_ref = oracle.rescale(acc_ref, gamma, beta)
+    scale = beta.astype(np.float64)[:, None] * gamma / 127.0
+    yg = y_gpu.float().cpu().numpy().astype(np.float64)
+    if rows is not None:
+        yg = yg[:, rows]
+    tol = (1e-2 if out_bf16 else 1e-5) * np.maximum(np.abs(y_ref), scale)
+    bad = np.abs(yg - y_ref) > tol
+    assert not bad.any(), "y mismatch at %s" % (np.argwhere(bad)[:5],)
+
+
+# ----------------------------------------------------------------- pack ---
+
+PACK_SHAPES = [(16, 256), (48, 512), (272, 768), (512, 512), (6912, 2560)]
+
+
+@pytest.mark.parametrize("d_out,d_in", PACK_SHAPES)
+def test_pack_matches_oracle(d_out, d_in):
+    W = draw(Problem("p", d_in, d_out, 1, 0.02, 0.0, 1.0, 3))[0]
+    Wd = W.to(dev())
+    own = bl.pack_weights(Wd, EPS)
+    g_oracle = oracle.absmean_gamma(W.numpy())
+    g_gpu = float(own.gamma.item())
+    assert abs(g_gpu - g_oracle) <= 1e-6 * g_oracle
+    given = bl.pack_weights(Wd, EPS, gamma=torch.tensor([g_oracle], device=dev()))
+    assert float(given.gamma.item()) == g_oracle
+    expect = oracle.pack(oracle.ternarize(W.numpy(), g_oracle, EPS))
+    np.testing.assert_array_equal(u32(given.packed), expect)
+    if g_gpu == g_oracle:
+        np.testing.assert_array_equal(u32(own.packed), expect)
+
+
+def test_pack_special_weights():
+    # All zero: gamma = 0, every code 0 -> word 0x55555555.
+    z = bl.pack_weights(torch.zeros(32, 512, device=dev()), EPS)
+    assert z.gamma.item() == 0.0
+    assert (u32(z.packed) == 0x55555555).all()
+    # Ties of RoundClip: gamma = 1, eps = 0 -> z = W exactly.
+    vals = torch.tensor([0.5, -0.5, 1.5, -1.5, 0.49999997, -0.50000006, 7.0, -7.0, 0.0, -0.0,
+                         1.0, -1.0, 0.25, -0.75, 0.75, -0.25], dtype=torch.float32)
+    W = vals.repeat(16, 16)
+    p = bl.pack_weights(W.to(dev()), 0.0, gamma=torch.tensor([1.0], device=dev()))
+    expect = oracle.pack(oracle.ternarize(W.numpy(), 1.0, 0.0))
+    np.testing.assert_array_equal(u32(p.packed), expect)
+    codes = oracle.unpack(u32(p.packed), 16, 256)[0, :16].tolist()
+    assert codes == [1, 0, 1, -1, 0, -1, 1, -1, 0, 0, 1, -1, 0, -1, 1, 0]
+
+
+# ------------------------------------------------------------ quant_act ---
+
+QA_CASES = [
+    (4, 512, 0.01, 50.0, True, False),
+    (1, 2560, 0.005, 100.0, True, False),
+    (16, 11008, 0.005, 100.0, True, False),
+    (8, 8192, 0.001, 1000.0, True, False),
+    (3, 768, 0.01, 50.0, False, False),
+    (5, 1024, 0.01, 50.0, True, True),
+    (2048, 4096, 0.0, 1.0, True, False),
+    (1, 65536, 0.001, 100.0, True, False),
+]
+
+
+@pytest.mark.parametrize("T,K,frac,factor,rmsnorm,use_gain", QA_CASES)
+def test_quant_act_matches_oracle(T, K, frac, factor, rmsnorm, use_gain):
+    X = draw(Problem("q", K, 16, T, 0.02, frac, factor, 8))[1]
+    gain = None
+    if use_gain:
+        gen = torch.Generator().manual_seed(1)
+        gain = (torch.rand(K, generator=gen) * 2).numpy().astype(np.float32)
+    xb = bf16_bits(X)
+    q_ref, b_ref, s_ref, r_ref = oracle.quant_act(xb, gain=gain, rmsnorm=rmsnorm, eps=EPS,
+                                                  norm_eps=NORM_EPS)
+    Xd = X.to(dev())
+    gd = None if gain is None else to_dev(gain)
+    # The GPU's own rms agrees with the oracle's.
+    _, _, _, r_gpu = bl.quant_act(Xd, gain=gd, rmsnorm=rmsnorm, eps=EPS, norm_eps=NORM_EPS)
+    np.testing.assert_allclose(r_gpu.cpu().numpy(), r_ref, rtol=1e-6)
+    # With the oracle's rms the codes, beta and row sums are bit-exact.
+    xq, beta, rowsum, r_used = bl.quant_act(Xd, gain=gd, rmsnorm=rmsnorm, eps=EPS,
+                                            norm_eps=NORM_EPS, rms=to_dev(r_ref))
+    np.testing.assert_array_equal(xq.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(beta.cpu().numpy(), b_ref)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), s_ref)
+    assert xq.cpu().numpy().min() >= -127
+
+
+def test_quant_act_special_tokens():
+    K = 512
+    x = torch.zeros(4, K)
+    x[1] = -3.0
+    x[2, 77] = 2.5
+    x[3] = torch.linspace(-1, 1, K)
+    X = x.to(torch.bfloat16)
+    xb = bf16_bits(X)
+    q_ref, b_ref, s_ref, r_ref = oracle.quant_act(xb, eps=EPS, norm_eps=NORM_EPS)
+    xq, beta, rowsum, _ = bl.quant_act(X.to(dev()), rms=to_dev(r_ref))
+    np.testing.assert_array_equal(xq.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), s_ref)
+    assert beta[0].item() == 0 and not xq[0].any()
+    assert (xq[1] == -127).all()
+
+
+# ---------------------------------------------------------------- forward ---
+
+def forward_case(d_out, d_in, T, out_dtype, seed=5, frac=0.01, factor=50.0):
+    W, X = draw(Problem("f", d_in, d_out, T, 0.02, frac, factor, seed))
+    o = oracle_side(W, X)
+    packed = oracle.pack(o["wq"])
+    w = bl.PackedTernary(to_dev(packed.view(np.int32)),
+                         torch.tensor([o["gamma"]], device=dev()), d_out, d_in)
+    y, acc = bl.forward(w, to_dev(o["xq"]), to_dev(o["beta"]), to_dev(o["rowsum"]),
+                        out_dtype=out_dtype, want_acc=True)
+    acc_ref = oracle.int_matmul(o["wq"], o["xq"])
+    np.testing.assert_array_equal(acc.cpu().numpy(), acc_ref)
+    check_y(y, acc_ref, o["gamma"], o["beta"], out_dtype == torch.bfloat16)
+    return o, w, y
+
+
+GEMV_SHAPES = [(16, 256), (48, 512), (272, 768), (512, 512), (6912, 2560), (32, 11008)]
+
+
+@pytest.mark.parametrize("d_out,d_in", GEMV_SHAPES)
+@pytest.mark.parametrize("T", [1, 2, 3, 7, 8, 9, 15, 16])
+def test_gemv_matches_oracle(d_out, d_in, T):
+    forward_case(d_out, d_in, T, torch.float32)
+
+
+@pytest.mark.parametrize("T", [1, 4, 16])
+def test_gemv_bf16_out(T):
+    forward_case(512, 512, T, torch.bfloat16)
+
+
+GEMM_SHAPES = [(128, 256), (144, 512), (272, 768), (512, 512), (384, 2560)]
+
+
+@pytest.mark.parametrize("d_out,d_in", GEMM_SHAPES)
+@pytest.mark.parametrize("T", [17, 100, 256, 300, 600])
+def test_gemm_matches_oracle(d_out, d_in, T):
+    forward_case(d_out, d_in, T, torch.float32)
+
+
+@pytest.mark.parametrize("T", [33, 513])
+def test_gemm_bf16_out(T):
+    forward_case(256, 1024, T, torch.bfloat16)
+
+
+def test_forward_zero_inputs():
+    for T in (1, 40):
+        d_out, d_in = 64, 512
+        w = bl.pack_weights(torch.zeros(d_out, d_in, device=dev()), EPS)
+        X = torch.randn(T, d_in).to(torch.bfloat16).to(dev())
+        y = bl.linear(w, X)
+        assert not y.any()
+        W = torch.randn(d_out, d_in, device=dev()) * 0.02
+        w = bl.pack_weights(W, EPS)
+        y = bl.linear(w, torch.zeros(T, d_in, dtype=torch.bfloat16, device=dev()))
+        assert not y.any()
+
+
+def test_forward_empty_batch():
+    w = bl.pack_weights(torch.randn(64, 512, device=dev()), EPS)
+    Xq = torch.empty(0, 512, dtype=torch.int8, device=dev())
+    e = torch.empty(0, device=dev())
+    y = bl.forward(w, Xq, e, e.to(torch.int32))
+    assert y.shape == (0, 64)
+
+
+def test_forward_max_d_in():
+    forward_case(16, 65536, 1, torch.float32, frac=0.001, factor=100.0)
+    forward_case(16, 65536, 20, torch.float32, frac=0.001, factor=100.0)
+
+
+def test_linear_equals_separate_calls_and_oracle():
+    d_out, d_in = 272, 1024
+    for T in (1, 5, 16, 17, 300):
+        W, X = draw(Problem("l", d_in, d_out, T, 0.02, 0.01, 50.0, 11))
+        Wd, Xd = W.to(dev()), X.to(dev())
+        w = bl.pack_weights(Wd, EPS)
+        y1 = bl.linear(w, Xd)
+        xq, beta, rowsum, _ = bl.quant_act(Xd)
+        y2 = bl.forward(w, xq, beta, rowsum)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2)
+        # End to end against the oracle computed from W and X alone.
+        o = oracle_side(W, X)
+        if float(w.gamma.item()) == o["gamma"]:
+            acc_ref = oracle.int_matmul(o["wq"], o["xq"])
+            check_y(y1, acc_ref, o["gamma"], o["beta"], False)
+
+
+# ------------------------------------------- failure detection (bounded) ---
+
+def test_bounded_wait_reports_timeout():
+    assert bl.device_error(clear=True) == bl.OK
+    bl.wait_probe(2_000_000)           # 2 ms on a barrier nothing arrives on
+    assert bl.device_error(clear=True) == bl.ERR_TIMEOUT
+    assert bl.device_error(clear=True) == bl.OK
+    # The context is still usable afterwards.
+    forward_case(48, 512, 3, torch.float32)
+    forward_case(144, 512, 40, torch.float32)
