@@ -1,0 +1,604 @@
+"""Benchmark of the BitLinear forward hot path on B200.
+
+Prints ONE JSON line on rank 0.
+
+Headline (decode): the single-token 2560 -> 6912 BitLinear forward (fused
+RMSNorm + absmax int8 quantiser, then the ternary GEMV with the fused
+rescale), reported as achieved HBM GB/s of algorithmic bytes.  One step is a
+stack of ``LAYERS`` such forwards over distinct packed weight copies (the
+projections of consecutive layers of one decode step), so each step streams
+more packed weight bytes than the L2 holds and every weight byte comes from
+HBM.  Steps are captured in a CUDA graph and timed with CUDA events.
+
+Also in the line: the prefill forward (2048 tokens, 4096 -> 11008, bf16
+out) as int8 tensor TOPS, the transformer-block and large decode
+workloads, the roofline of the dominant kernel, the CPU oracle baseline,
+an end-to-end number through the public API with host buffers, and SM
+clocks sampled during the timed region.
+
+``--impl reference`` times the CPU oracle instead (the reference arm).
+Multi-GPU (torchrun): independent replicas, one per GPU, no collective on
+the data path; time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import ALL as WORKLOADS, Problem, bf16_bits, draw  # noqa: E402
+
+METRIC = "decode GEMV achieved HBM GB/s (% of peak); prefill int8 TOPS (% of peak)"
+HEADLINE = "decode_gemv_2560x6912_t1"
+LAYERS = 64
+L2_BYTES = 126 * 2 ** 20
+EPS = 1e-5
+
+
+# ----------------------------------------------------------------- peaks ---
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# Dense int8 tensor throughput relative to dense bf16: NVIDIA's B200 figures
+# (4.5 POPS int8 / 2.25 PFLOPS bf16, dense).
+INT8_OVER_BF16 = 2.0
+
+
+# ---------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampler for the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = str(index)
+        try:
+            u = str(torch.cuda.get_device_properties(index).uuid)
+            self.index = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            pass
+        self.proc = None
+        self.lines = []
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, on: bool):
+        self.marks.append((time.time(), on))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
+                    "samples": 0}
+        windows = []
+        for i in range(0, len(self.marks) - 1, 2):
+            windows.append((self.marks[i][0], self.marks[i + 1][0]))
+
+        def inside(t):
+            return any(a - 0.15 <= t <= b + 0.15 for a, b in windows)
+
+        rows = []
+        for t, line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            rows.append((t, f))
+        sel = [f for t, f in rows if inside(t)] or [f for _, f in rows]
+        mhz = [float(f[1]) for f in sel if f[1].replace(".", "").isdigit()]
+        mx = [float(f[2]) for f in sel if f[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for f in sel for i in range(4)
+                          if f[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(sel)}
+
+
+# ------------------------------------------------------- distributed ---
+
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ helpers ---
+
+def decode_bytes(p: Problem, out_bytes: int = 2) -> dict:
+    """Algorithmic bytes of one decode BitLinear forward (quantise + product)."""
+    T, K, N = p.tokens, p.d_in, p.d_out
+    w = N * K // 4                   # packed 2-bit weights
+    x = T * K * 2                    # bf16 activations read by the quantiser
+    xq = 2 * T * K                   # int8 codes written once, read once
+    small = 4 + 2 * 8 * T            # gamma; beta and row sums written and read
+    y = T * N * out_bytes
+    return dict(step=w + x + xq + small + y, gemv=w + T * K + 8 * T + 4 + y, weights=w,
+                weights_and_acts=w + x + y)
+
+
+def time_graph(g: torch.cuda.CUDAGraph, reps: int = 1) -> float:
+    """Milliseconds of `reps` replays of g, CUDA events on the current stream."""
+    s = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(s)
+    for _ in range(reps):
+        g.replay()
+    b.record(s)
+    b.synchronize()
+    return a.elapsed_time(b)
+
+
+def capture(fn):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # one eager call on the side stream before capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def source_sha(name):
+    p = os.path.join(ROOT, "ternary_weight_linear_bitlinear_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def profile_traffic(summary_name: str, source: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    summary was taken on a different version of the kernel source."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_b or m_sha.group(1) != source_sha(source):
+        return None
+    return float(m_b.group(1))
+
+
+# ------------------------------------------------------ decode workload ---
+
+class DecodeRun:
+    """`layers` forwards per step over distinct packed weight copies."""
+
+    def __init__(self, problems, layers, dev, out_dtype=torch.bfloat16):
+        import ternary_weight_linear_bitlinear_b200 as bl
+        self.bl = bl
+        self.problems = problems
+        self.dev = dev
+        self.out_dtype = out_dtype
+        self.layers = []      # (problem, PackedTernary, X, scratch, Y, Xq-state)
+        base = []
+        for p in problems:
+            W, X = draw(p)
+            w = bl.pack_weights(W.to(dev), EPS)
+            base.append((p, w, X.to(dev)))
+            del W
+        reps = max(1, layers // len(problems))
+        for r in range(reps):
+            for p, w0, X in base:
+                if r == 0:
+                    w = w0
+                else:
+                    w = bl.PackedTernary(w0.packed.clone(), w0.gamma.clone(), w0.d_out, w0.d_in)
+                T = p.tokens
+                scratch = (torch.empty((T, p.d_in), dtype=torch.int8, device=dev),
+                           torch.empty(T, dtype=torch.float32, device=dev),
+                           torch.empty(T, dtype=torch.int32, device=dev))
+                Y = torch.empty((T, p.d_out), dtype=out_dtype, device=dev)
+                self.layers.append((p, w, X, scratch, Y))
+        torch.cuda.synchronize()
+        # Pre-quantised activations for the product-only timing.
+        for p, w, X, scratch, Y in self.layers:
+            xq, beta, rowsum, _ = bl.quant_act(X)
+            scratch[0].copy_(xq)
+            scratch[1].copy_(beta)
+            scratch[2].copy_(rowsum)
+        torch.cuda.synchronize()
+
+    def step(self):
+        for p, w, X, scratch, Y in self.layers:
+            self.bl.linear(w, X, out=Y, scratch=scratch)
+
+    def product_only(self):
+        for p, w, X, scratch, Y in self.layers:
+            self.bl.forward(w, scratch[0], scratch[1], scratch[2], out=Y)
+
+    def bytes(self):
+        ob = 2 if self.out_dtype == torch.bfloat16 else 4
+        tot = dict(step=0, gemv=0, weights=0, weights_and_acts=0)
+        for p, *_ in self.layers:
+            for k, v in decode_bytes(p, ob).items():
+                tot[k] += v
+        return tot
+
+    def weight_bytes_resident(self):
+        return sum(w.packed.numel() * 4 for _, w, *_ in self.layers)
+
+
+def run_decode(name, steps, warmup, dev, layers, world):
+    wl = WORKLOADS[name]
+    run = DecodeRun(wl.problems, layers, dev)
+    nb = run.bytes()
+    for _ in range(max(warmup, 3)):
+        run.step()
+    torch.cuda.synchronize()
+
+    def k_steps(k):
+        def f():
+            for _ in range(k):
+                run.step()
+        return f
+
+    g_warm = capture(k_steps(max(warmup, 3)))
+    g_timed = capture(k_steps(steps))
+    time_graph(g_warm)
+    time_graph(g_timed)              # untimed pass: graph upload
+    barrier(world)
+    return run, nb, g_timed
+
+
+def measure_product_only(run, steps):
+    g = capture(lambda: [run.product_only() for _ in range(steps)])
+    time_graph(g)
+    ms = time_graph(g)
+    launches = steps * len(run.layers)
+    return ms / launches, launches
+
+
+# ----------------------------------------------------- prefill workload ---
+
+def measure_prefill(steps, warmup, dev, peaks):
+    import ternary_weight_linear_bitlinear_b200 as bl
+    p = WORKLOADS["prefill_2048x4096x11008"].problems[0]
+    W, X = draw(p)
+    w = bl.pack_weights(W.to(dev), EPS)
+    del W
+    Xd = X.to(dev)
+    T = p.tokens
+    scratch = (torch.empty((T, p.d_in), dtype=torch.int8, device=dev),
+               torch.empty(T, dtype=torch.float32, device=dev),
+               torch.empty(T, dtype=torch.int32, device=dev))
+    Y = torch.empty((T, p.d_out), dtype=torch.bfloat16, device=dev)
+    for _ in range(max(warmup, 3)):
+        bl.linear(w, Xd, out=Y, scratch=scratch)
+    g_step = capture(lambda: [bl.linear(w, Xd, out=Y, scratch=scratch) for _ in range(steps)])
+    time_graph(g_step)
+    ms_step = time_graph(g_step) / steps
+    g_mm = capture(lambda: [bl.forward(w, scratch[0], scratch[1], scratch[2], out=Y)
+                            for _ in range(steps)])
+    time_graph(g_mm)
+    ms_mm = time_graph(g_mm) / steps
+    ops = 2.0 * T * p.d_in * p.d_out
+    tops = ops / (ms_mm * 1e-3) / 1e12
+    peak = peaks["bf16"] * INT8_OVER_BF16
+    return {
+        "workload": WORKLOADS["prefill_2048x4096x11008"].name,
+        "tops_gemm": round(tops, 1), "unit": "TOPS (int8, 2 ops per MAC)",
+        "ms_gemm": round(ms_mm, 4), "ms_step_with_quant": round(ms_step, 4),
+        "tops_step": round(ops / (ms_step * 1e-3) / 1e12, 1),
+        "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(peak, 1),
+                     "unit": "TFLOP/s", "frac": round(tops / peak, 4),
+                     "peak_source": "%s bf16 burst x %.0f (nominal int8/bf16 dense ratio)"
+                                    % (peaks["source"], INT8_OVER_BF16)},
+        "frac_of_datasheet_4500": round(tops / 4500.0, 4),
+        "gpu_launches": 2 * steps,
+    }
+
+
+# ------------------------------------------------------------ e2e ---
+
+def measure_e2e(run, steps):
+    """Through the public API with host buffers: every step copies its
+    activations host -> device from pinned memory and reads each output
+    back device -> host, inside the timed region."""
+    bl = run.bl
+    host_x = [X.cpu().pin_memory() for _, _, X, _, _ in run.layers]
+    host_y = [torch.empty(Y.shape, dtype=Y.dtype).pin_memory() for *_, Y in run.layers]
+    h2d = sum(x.numel() * x.element_size() for x in host_x)
+    d2h = sum(y.numel() * y.element_size() for y in host_y)
+    s = torch.cuda.current_stream()
+
+    def one():
+        for (p, w, X, scratch, Y), hx, hy in zip(run.layers, host_x, host_y):
+            X.copy_(hx, non_blocking=True)
+            bl.linear(w, X, out=Y, scratch=scratch)
+            hy.copy_(Y, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(steps):
+        one()
+    b.record(s)
+    b.synchronize()
+    return a.elapsed_time(b) / steps, h2d, d2h
+
+
+# -------------------------------------------------------- CPU oracle ---
+
+def oracle_layer_step(p, wq, gamma, xb):
+    import oracle
+    xq, beta, rowsum, _ = oracle.quant_act(xb, eps=EPS)
+    acc = oracle.int_matmul(wq, xq)
+    return oracle.rescale(acc, gamma, beta)
+
+
+def cpu_oracle_rate(name, seconds, max_layers=None):
+    """Time the oracle on bounded samples of the workload; returns
+    (GB/s of algorithmic bytes, layers done, seconds, description)."""
+    import oracle
+    oracle.build()
+    wl = WORKLOADS[name]
+    prepared = []
+    for p in wl.problems:
+        W, X = draw(p)
+        Wn = W.numpy()
+        g = oracle.absmean_gamma(Wn)
+        prepared.append((p, oracle.ternarize(Wn, g, EPS), g, bf16_bits(X)))
+        del W, Wn
+    done, nbytes, t0 = 0, 0, time.perf_counter()
+    while True:
+        p, wq, g, xb = prepared[done % len(prepared)]
+        oracle_layer_step(p, wq, g, xb)
+        done += 1
+        nbytes += decode_bytes(p)["step"]
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_layers and done >= max_layers):
+            break
+    return nbytes / el / 1e9, done, el
+
+
+# -------------------------------------------------------------- main ---
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="headline only (no prefill / other decode workloads)")
+    args = ap.parse_args()
+    warmup = max(args.warmup, 3)
+    rank, world, local = dist_init(args.gpus)
+
+    if args.impl == "reference":
+        if rank == 0:
+            reference_arm(args, warmup)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    sampler = ClockSampler(local)
+    sampler.start()
+
+    run, nb, g_timed = run_decode(args.workload, args.steps, warmup, dev, LAYERS, world)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.mark(True)
+    torch.cuda.nvtx.range_push("timed")
+    ms = time_graph(g_timed)
+    torch.cuda.nvtx.range_pop()
+    sampler.mark(False)
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    value = nb["step"] * world / (ms_step * 1e-3) / 1e9
+
+    # Dominant kernel (the GEMV) timed alone, back to back, same weights.
+    sampler.mark(True)
+    gemv_ms, gemv_launches = measure_product_only(run, args.steps)
+    sampler.mark(False)
+    per_gemv_bytes = nb["gemv"] / len(run.layers)
+    gemv_gbs = per_gemv_bytes / (gemv_ms * 1e-3) / 1e9
+    traffic = profile_traffic("gemv_decode_2560x6912_t1.md", "gemv.cu")
+
+    extras = {}
+    if not args.no_extras:
+        sampler.mark(True)
+        extras["prefill"] = measure_prefill(max(10, min(args.steps, 50)), warmup, dev, peaks)
+        sampler.mark(False)
+        other = {}
+        for name in ("decode_block_4096_t1", "decode_block_4096_t16", "large_gemv_8192x28672_t1",
+                     "large_gemv_8192x28672_t8"):
+            wl = WORKLOADS[name]
+            per = sum(decode_bytes(p)["weights"] for p in wl.problems)
+            layers = max(len(wl.problems), int(np.ceil(4 * L2_BYTES / per)) * len(wl.problems))
+            r2 = DecodeRun(wl.problems, layers, dev)
+            g2 = capture(lambda: [r2.step() for _ in range(5)])
+            time_graph(g2)
+            sampler.mark(True)
+            t2 = time_graph(g2) / 5
+            sampler.mark(False)
+            b2 = r2.bytes()
+            other[name] = {"gbs_step": round(b2["step"] / (t2 * 1e-3) / 1e9, 1),
+                           "ms_per_pass": round(t2, 4), "forwards_per_pass": len(r2.layers),
+                           "frac_of_hbm": round(b2["step"] / (t2 * 1e-3) / 1e9 / peaks["hbm"], 4)}
+            del r2, g2
+            torch.cuda.empty_cache()
+        extras["decode_other"] = other
+
+    e2e_ms, h2d, d2h = measure_e2e(run, max(3, min(args.steps, 20)))
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    sampler.stop()
+    status = run.bl.device_error(clear=True)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        rate, done, el = cpu_oracle_rate(args.workload, args.cpu_seconds)
+        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": "%d single-token %s BitLinear forwards (quantise + int32 product + "
+                         "rescale) by the plain C oracle, single thread, %.1f s"
+                         % (done, "x".join(args.workload.split("_")[2:3]), el)}
+
+    if rank == 0:
+        clocks = sampler.summary()
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8", "data": "synthetic",
+            "config": {
+                "workload": args.workload, "forwards_per_step": len(run.layers),
+                "tokens": run.problems[0].tokens, "d_in": run.problems[0].d_in,
+                "d_out": run.problems[0].d_out, "out_dtype": "bf16",
+                "bytes_per_step": nb["step"],
+                "l2": "inputs larger than L2: each step streams %d distinct packed weight "
+                      "copies (%.0f MB > %d MB L2)" % (len(run.layers),
+                                                       run.weight_bytes_resident() / 1e6,
+                                                       L2_BYTES // 2 ** 20),
+                "parallelism": "replicas" if world > 1 else "single GPU",
+                "timing": "CUDA graph of all timed steps, CUDA events, max over ranks"},
+            "frac_of_hbm": round(value / world / peaks["hbm"], 4),
+            "frac_of_datasheet_8000": round(value / world / 8000.0, 4),
+            "gbs_weights_and_activations": round(nb["weights_and_acts"] * world /
+                                                 (ms_step * 1e-3) / 1e9, 2),
+            "roofline": {"bound": "hbm", "kernel": "gemv_kernel (decode GEMV)",
+                         "achieved": round(gemv_gbs, 1), "peak": peaks["hbm"],
+                         "unit": "GB/s", "frac": round(gemv_gbs / peaks["hbm"], 4),
+                         "traffic": traffic, "algorithmic_bytes_per_launch": per_gemv_bytes,
+                         "avg_launch_us": round(gemv_ms * 1e3, 3),
+                         "launches_timed": gemv_launches,
+                         "peak_source": peaks["source"] + " HBM copy bandwidth"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(nb["step"] * world / (e2e_ms * 1e-3) / 1e9, 3),
+                    "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 4),
+                    "how": "public Python API, pinned host X copied in and Y copied out "
+                           "every forward, eager launches"},
+            "gpu_launches": 2 * len(run.layers) * args.steps,
+            "clocks": clocks,
+            "device_error": run.bl.status_string(status),
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+
+
+def reference_arm(args, warmup):
+    """The CPU oracle timed on this host: each step is a bounded sample
+    (one BitLinear forward of the workload's shape), same metric and unit."""
+    import oracle
+    oracle.build()
+    wl = WORKLOADS[args.workload]
+    prepared = []
+    for p in wl.problems:
+        W, X = draw(p)
+        Wn = W.numpy()
+        g = oracle.absmean_gamma(Wn)
+        prepared.append((p, oracle.ternarize(Wn, g, EPS), g, bf16_bits(X)))
+    for i in range(warmup):
+        p, wq, g, xb = prepared[i % len(prepared)]
+        oracle_layer_step(p, wq, g, xb)
+    nbytes = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        p, wq, g, xb = prepared[i % len(prepared)]
+        oracle_layer_step(p, wq, g, xb)
+        nbytes += decode_bytes(p)["step"]
+    el = time.perf_counter() - t0
+    value = nbytes / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": warmup,
+        "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": args.workload, "forwards_per_step": 1,
+                   "tokens": wl.problems[0].tokens, "d_in": wl.problems[0].d_in,
+                   "d_out": wl.problems[0].d_out},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "each step one BitLinear forward of the workload by the "
+                                   "plain C oracle, single thread"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
