@@ -112,6 +112,36 @@ int bitlinear_pack_weights(const float *W, int64_t d_out, int64_t d_in, float ep
                            float *gamma_out, cudaStream_t stream);
 
 /*
+ * bitlinear_pack_weights_noalloc -- bitlinear_pack_weights with gamma
+ * computed, for callers that cannot allocate device memory.  The pages have
+ * no counterpart: this entry exists for callers such as code that packs
+ * weights while a stream is being captured into a CUDA graph (where
+ * cudaMalloc is not allowed), runtimes whose device memory is entirely
+ * reserved up front by their own pool, or hosts with no device allocator
+ * they may call -- none of which can supply the workspace that
+ * bitlinear_pack_weights needs for its partial sums of |W|.
+ *
+ * Same arguments and results as bitlinear_pack_weights(W, d_out, d_in, eps,
+ * NULL, workspace, ..., packed, gamma_out, stream); gamma is bit-identical.
+ * The partial sums live instead in one fixed array inside the library of
+ * 1184 doubles (9,472 bytes), held in the memory of every GPU that loads
+ * the library until the process exits.  Shapes whose reduction would need
+ * more partials than that are rejected with BITLINEAR_ERR_UNSUPPORTED_SHAPE
+ * (the reduction grid is capped at 1184 blocks, so every shape the other
+ * rules accept fits).  Calls no allocator (no cudaMalloc, cudaFree or
+ * allocating library routine).  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  All calls share the one
+ * array, which keeps the last call's contents (every partial read is first
+ * written by the same call, so nothing needs clearing): calls that overlap
+ * on the GPU -- on different streams, or on different host threads -- race
+ * and must be serialised by the caller.
+ */
+int bitlinear_pack_weights_noalloc(const float *W, int64_t d_out, int64_t d_in,
+                                   float eps, uint32_t *packed, float *gamma_out,
+                                   cudaStream_t stream);
+
+/*
  * bitlinear_quant_act -- fused RMSNorm + per-token absmax int8 quantisation
  * ([MF] section 2, "Activation Quantization: Absmax Scaling"; beta taken per
  * token; Q_b - 1 = 127 is both multiplier and clip bound).

@@ -45,6 +45,7 @@ SIGNATURES = {
     "bitlinear_pack_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bitlinear_pack_weights": (_int, [_vp, _i64, _i64, _f32, _vp, _vp, ctypes.c_size_t,
                                       _vp, _vp, _vp]),
+    "bitlinear_pack_weights_noalloc": (_int, [_vp, _i64, _i64, _f32, _vp, _vp, _vp]),
     "bitlinear_quant_act": (_int, [_vp, _i64, _i64, _vp, _u32, _f32, _f32, _vp, _vp, _vp,
                                    _vp, _vp, _vp]),
     "bitlinear_forward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int,

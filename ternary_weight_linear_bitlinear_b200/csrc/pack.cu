@@ -12,6 +12,7 @@
 // weight matrix.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "bitlinear.h"
 #include "common.cuh"
@@ -149,5 +150,81 @@ extern "C" int bitlinear_pack_weights(const float *W, int64_t d_out, int64_t d_i
     int64_t pblocks = (nwords + 255) / 256;
     if (pblocks > 148 * 16) pblocks = 148 * 16;
     pack_kernel<<<(int)pblocks, 256, 0, stream>>>(W, d_out, d_in, eps, gptr, packed, gamma_out);
+    return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of bitlinear_pack_weights.
+//
+// Some callers cannot allocate device memory at the point where they pack
+// weights: code running while a stream is being captured into a CUDA graph
+// (cudaMalloc is not permitted during capture), runtimes whose device memory
+// is fully reserved up front by their own pool, and hosts without a device
+// allocator they may call.  bitlinear_pack_weights needs such callers to hand
+// it a device workspace for the partial sums of mean|W|.  This variant keeps
+// those partial sums in a fixed array inside the library instead.
+//
+// The array below lives in every GPU's memory that loads the library, until
+// the process exits.  Host code cannot use its name as a device address, so
+// the address is looked up once per device with cudaGetSymbolAddress (on the
+// first call made with that device current) and passed to the kernels.
+// ---------------------------------------------------------------------------
+namespace bl {
+
+constexpr int kNoallocPartials = kRedMaxBlocks;   // 1184 doubles = 9,472 bytes
+
+static __device__ __align__(256) double g_pack_partials[kNoallocPartials];
+
+namespace {
+std::mutex g_noalloc_mu;
+double *g_noalloc_ptr[64];
+}  // namespace
+
+static bitlinear_status noalloc_scratch(double **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BITLINEAR_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_pack_partials) != cudaSuccess || !p)
+            return BITLINEAR_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<double *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return BITLINEAR_OK;
+}
+
+}  // namespace bl
+
+extern "C" int bitlinear_pack_weights_noalloc(const float *W, int64_t d_out, int64_t d_in,
+                                              float eps, uint32_t *packed, float *gamma_out,
+                                              cudaStream_t stream) {
+    if (!W || !packed || !gamma_out) return BITLINEAR_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return BITLINEAR_ERR_INVALID_ARG;
+    if (bitlinear_packed_words(d_out, d_in) == 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(gamma_out, 4))
+        return BITLINEAR_ERR_MISALIGNED;
+    // Same reduction grid as bitlinear_pack_weights, so gamma is bit-identical.
+    const int64_t n = d_out * d_in;
+    const int64_t n4 = n / 4;
+    int64_t blocks = (n4 + kRedThreads * 8 - 1) / (kRedThreads * 8);
+    if (blocks > kRedMaxBlocks) blocks = kRedMaxBlocks;
+    if (blocks < 1) blocks = 1;
+    if (blocks > kNoallocPartials) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    bitlinear_status st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    double *partial = nullptr;
+    st = noalloc_scratch(&partial);
+    if (st != BITLINEAR_OK) return st;
+    // Every partial the final kernel reads is written by this call first, so
+    // nothing in the shared array has to start at zero.
+    absmean_partial_kernel<<<(int)blocks, kRedThreads, 0, stream>>>(
+        reinterpret_cast<const float4 *>(W), n4, partial);
+    absmean_final_kernel<<<1, kRedThreads, 0, stream>>>(partial, (int)blocks, (double)n,
+                                                         gamma_out);
+    int64_t pblocks = (n / 16 + 255) / 256;
+    if (pblocks > 148 * 16) pblocks = 148 * 16;
+    pack_kernel<<<(int)pblocks, 256, 0, stream>>>(W, d_out, d_in, eps, gamma_out, packed,
+                                                  gamma_out);
     return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
