@@ -72,8 +72,8 @@ def _load():
         lib.oracle_unpack.restype = i32
         lib.oracle_unpack_row.argtypes = [vp, i64, i64, i64, vp]
         lib.oracle_unpack_row.restype = i32
-        lib.oracle_rms.argtypes = [vp, i64, f32]
-        lib.oracle_rms.restype = f32
+        lib.oracle_inv_rms.argtypes = [vp, i64, f32]
+        lib.oracle_inv_rms.restype = f32
         lib.oracle_quant_act.argtypes = [vp, i64, i64, vp, i32, f32, f32, vp,
                                          vp, vp, vp, vp]
         lib.oracle_quant_act.restype = None
@@ -167,21 +167,22 @@ def unpack_row(packed, d_out: int, d_in: int, o: int) -> np.ndarray:
 
 # ------------------------------------------------ activation quantisation ---
 
-def rms(x_bf16_bits, norm_eps: float = 1e-5) -> float:
+def inv_rms(x_bf16_bits, norm_eps: float = 1e-5) -> float:
+    """1 / sqrt(mean(x^2) + norm_eps) of one token, in double, rounded to f32."""
     x = _c(x_bf16_bits, np.uint16)
-    return float(_load().oracle_rms(_ptr(x), x.size, norm_eps))
+    return float(_load().oracle_inv_rms(_ptr(x), x.size, norm_eps))
 
 
 def quant_act(X_bf16_bits, gain=None, rmsnorm: bool = True, eps: float = 1e-5,
-              norm_eps: float = 1e-5, rms_in=None):
+              norm_eps: float = 1e-5, inv_rms_in=None):
     """Per-token absmax int8 quantisation, optional RMSNorm first ([MF] §2).
 
-    Returns (xq int8 [T][K], beta f32 [T], rowsum int32 [T], rms f32 [T]).
+    Returns (xq int8 [T][K], beta f32 [T], rowsum int32 [T], inv_rms f32 [T]).
     """
     X = _c(X_bf16_bits, np.uint16)
     T, K = X.shape
     g = None if gain is None else _c(gain, np.float32)
-    r_in = None if rms_in is None else _c(rms_in, np.float32)
+    r_in = None if inv_rms_in is None else _c(inv_rms_in, np.float32)
     xq = np.empty((T, K), dtype=np.int8)
     beta = np.empty(T, dtype=np.float32)
     rowsum = np.empty(T, dtype=np.int32)
@@ -223,13 +224,13 @@ def rescale(acc, gamma: float, beta) -> np.ndarray:
 
 
 def forward(W, X_bf16_bits, eps: float = 1e-5, norm_eps: float = 1e-5, gain=None,
-            rmsnorm: bool = True, gamma=None, rms_in=None):
+            rmsnorm: bool = True, gamma=None, inv_rms_in=None):
     """The whole BitLinear forward on the CPU: returns a dict of every stage."""
     g = absmean_gamma(W) if gamma is None else float(gamma)
     wq = ternarize(W, g, eps)
     xq, beta, rowsum, r = quant_act(X_bf16_bits, gain, rmsnorm, eps, norm_eps,
-                                    rms_in)
+                                    inv_rms_in)
     acc = int_matmul(wq, xq)
     y = rescale(acc, g, beta)
-    return dict(gamma=g, wq=wq, xq=xq, beta=beta, rowsum=rowsum, rms=r, acc=acc,
+    return dict(gamma=g, wq=wq, xq=xq, beta=beta, rowsum=rowsum, inv_rms=r, acc=acc,
                 y=y)

@@ -19,7 +19,7 @@
  *
  * Precision: reductions (the absmean sum, the RMS sum of squares) and the
  * final rescale are carried in double.  The quantities that feed an integer
- * code (z = W / (gamma + eps), n = x / rms, v = n * 127 / (beta + eps)) are
+ * code (z = W / (gamma + eps), n = x * r, v = n * 127 / (beta + eps)) are
  * formed in IEEE binary32, one correctly rounded operation at a time, because
  * that is the precision in which the GPU kernels form them; the rounding
  * floor(z + 0.5) itself is then evaluated exactly.  This file is compiled
@@ -29,8 +29,9 @@
  *   - Q_b - 1 = 127 is both the activation multiplier and the clip bound; the
  *     code range is the symmetric [-127, 127].
  *   - The activation absmax beta is taken per token (one row of X).
- *   - RMSNorm is x / sqrt(mean(x^2) + norm_eps) * g, with g = 1 unless a gain
- *     vector is given; the page names RMSNorm but prints no formula.
+ *   - RMSNorm is x * r * g with r = 1 / sqrt(mean(x^2) + norm_eps) (the
+ *     reciprocal formed once per token) and g = 1 unless a gain vector is
+ *     given; the page names RMSNorm but prints no formula.
  *   - The rescale is the literal beta*gamma/(Q_b-1), without the epsilons used
  *     inside the two quantisers.
  *   - RoundClip rounds with floor(z + 0.5), i.e. halves go toward +infinity,
@@ -186,46 +187,49 @@ int oracle_unpack_row(const uint32_t *packed, int64_t n_out, int64_t n_in,
 
 /* ---------------------------------------- activation quantisation ([MF] §2) */
 
-/* RMS of one token: sqrt(mean(x^2) + norm_eps), carried in double and
+/* Reciprocal RMS of one token: 1 / sqrt(mean(x^2) + norm_eps), carried in
+ * double (sum, mean, square root and reciprocal each correctly rounded) and
  * rounded once to binary32. */
-float oracle_rms(const uint16_t *x, int64_t K, float norm_eps)
+float oracle_inv_rms(const uint16_t *x, int64_t K, float norm_eps)
 {
     double ss = 0.0;
     for (int64_t k = 0; k < K; ++k) {
         double v = (double)oracle_bf16_to_f32(x[k]);
         ss += v * v;
     }
-    return (float)sqrt(ss / (double)K + (double)norm_eps);
+    return (float)(1.0 / sqrt(ss / (double)K + (double)norm_eps));
 }
 
 /*
  * Per-token absmax int8 quantisation with optional RMSNorm in front.
- *   n_k   = x_k / rms (binary32 division), times g_k if a gain is given
- *           (binary32 multiplication); n_k = x_k when rmsnorm == 0
+ *   n_k   = x_k * r (binary32 multiplication) with r the token's reciprocal
+ *           RMS, times g_k if a gain is given (binary32 multiplication);
+ *           n_k = x_k when rmsnorm == 0
  *   beta  = max_k |n_k|
  *   q_k   = RoundClip(n_k * 127 / (beta + eps), -127, 127) with the scale
  *           127 / (beta + eps) formed first (binary32 add, then divide) and
  *           applied with one binary32 multiplication
  *   S     = sum_k q_k (the correction term of the offset-code product)
- * rms_in, when not NULL, supplies the per-token rms instead of computing it
- * (used to compare integer codes against a GPU that computed its own rms).
+ * inv_rms_in, when not NULL, supplies the per-token reciprocal RMS instead of
+ * computing it (used to compare integer codes against a GPU that computed
+ * its own).
  */
 void oracle_quant_act(const uint16_t *X, int64_t T, int64_t K, const float *gain,
-                      int rmsnorm, float eps, float norm_eps, const float *rms_in,
-                      int8_t *xq, float *beta, int32_t *rowsum, float *rms_out)
+                      int rmsnorm, float eps, float norm_eps, const float *inv_rms_in,
+                      int8_t *xq, float *beta, int32_t *rowsum, float *inv_rms_out)
 {
     for (int64_t t = 0; t < T; ++t) {
         const uint16_t *x = X + t * K;
-        float rms = 1.0f;
+        float r = 1.0f;
         if (rmsnorm)
-            rms = rms_in ? rms_in[t] : oracle_rms(x, K, norm_eps);
-        if (rms_out) rms_out[t] = rms;
+            r = inv_rms_in ? inv_rms_in[t] : oracle_inv_rms(x, K, norm_eps);
+        if (inv_rms_out) inv_rms_out[t] = r;
 
         float b = 0.0f;
         for (int64_t k = 0; k < K; ++k) {
             float n = oracle_bf16_to_f32(x[k]);
             if (rmsnorm) {
-                n = n / rms;
+                n = n * r;
                 if (gain) n = n * gain[k];
             }
             float a = fabsf(n);
@@ -238,7 +242,7 @@ void oracle_quant_act(const uint16_t *X, int64_t T, int64_t K, const float *gain
         for (int64_t k = 0; k < K; ++k) {
             float n = oracle_bf16_to_f32(x[k]);
             if (rmsnorm) {
-                n = n / rms;
+                n = n * r;
                 if (gain) n = n * gain[k];
             }
             float v = n * scale;

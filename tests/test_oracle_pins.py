@@ -35,7 +35,7 @@ def test_worked_example(golden_dir):
     out = oracle.forward(W, X, eps=ex["eps"], norm_eps=ex["norm_eps"])
     assert out["gamma"] == ex["gamma"]
     np.testing.assert_array_equal(out["wq"], np.array(ex["W_ternary"]))
-    assert abs(out["rms"][0] - ex["rms"]) < 2e-6
+    assert abs(out["inv_rms"][0] - ex["inv_rms"]) < 2e-6
     assert abs(out["beta"][0] - ex["beta"]) < 2e-6
     np.testing.assert_array_equal(out["xq"], np.array(ex["X_int8"]))
     np.testing.assert_array_equal(out["rowsum"], np.array(ex["rowsum"]))
@@ -189,16 +189,17 @@ def test_pack_rejects_bad_input():
 
 # ------------------------------------------------------- activation quant
 
-def test_rms_matches_torch_rms_norm():
-    """rms(x) agrees with torch.nn.functional.rms_norm (float64) to 1e-7."""
+def test_inv_rms_matches_torch_rms_norm():
+    """The reciprocal RMS agrees with torch.nn.functional.rms_norm (float64),
+    whose output is x * r, to 1e-7."""
     X = draw(Problem("r", 2560, 16, 8, 0.02, 0.005, 100.0, 11))[1]
     bits = bf16_bits(X)
     x64 = X.to(torch.float64)
     y = torch.nn.functional.rms_norm(x64, (x64.shape[1],), eps=float(np.float32(1e-5)))
     for t in range(X.shape[0]):
         k = int(torch.argmax(x64[t].abs()))
-        lib_rms = float(x64[t, k] / y[t, k])
-        assert abs(oracle.rms(bits[t]) - lib_rms) <= 1e-7 * lib_rms
+        lib_r = float(y[t, k] / x64[t, k])
+        assert abs(oracle.inv_rms(bits[t]) - lib_r) <= 1e-7 * lib_r
 
 
 def test_quant_act_invariants():
@@ -212,7 +213,7 @@ def test_quant_act_invariants():
         k = int(np.argmax(np.abs(xf[t])))
         assert abs(int(xq[t, k])) == 127                    # absmax channel -> +-Qb-1
         assert np.all((xq[t] == 0) | (np.sign(xq[t]) == np.sign(xf[t])))
-        np.testing.assert_allclose(beta[t], np.abs(xf[t]).max() / r[t], rtol=2e-7)
+        np.testing.assert_allclose(beta[t], np.abs(xf[t]).max() * r[t], rtol=2e-7)
 
 
 def test_quant_act_nearest_integer():
@@ -223,7 +224,7 @@ def test_quant_act_nearest_integer():
     xq, beta, _, r = oracle.quant_act(bits)
     xf = X.float().numpy()
     for t in range(4):
-        n = xf[t] / np.float32(r[t])
+        n = xf[t] * np.float32(r[t])
         s = np.float32(127.0) / (np.float32(beta[t]) + np.float32(1e-5))
         v = (n * s).astype(np.float64)
         cand = np.stack([np.floor(v), np.floor(v) + 1])
@@ -260,19 +261,19 @@ def test_quant_act_special_tokens():
     assert beta[0] == 0 and not xq[0].any() and S[0] == 0
     assert (xq[1] == -127).all() and S[1] == -127 * K
     assert xq[2, 77] == 127 and np.count_nonzero(xq[2]) == 1
-    # rms of a one-hot token is |v|/sqrt(K) (+eps): closed form
-    assert abs(r[2] - math.sqrt(2.5 ** 2 / K + float(np.float32(1e-5)))) < 1e-6
+    # reciprocal rms of a one-hot token is 1/sqrt(v^2/K + eps): closed form
+    assert abs(r[2] - 1 / math.sqrt(2.5 ** 2 / K + float(np.float32(1e-5)))) < 1e-6
 
 
-def test_quant_act_supplied_rms_is_used():
+def test_quant_act_supplied_inv_rms_is_used():
     X = draw(Problem("u", 512, 16, 3, 0.02, 0.01, 50.0, 4))[1]
     bits = bf16_bits(X)
     _, _, _, r = oracle.quant_act(bits)
-    a = oracle.quant_act(bits, rms_in=r)
+    a = oracle.quant_act(bits, inv_rms_in=r)
     b = oracle.quant_act(bits)
     for u, v in zip(a, b):
         np.testing.assert_array_equal(u, v)
-    c = oracle.quant_act(bits, rms_in=r * 2)
+    c = oracle.quant_act(bits, inv_rms_in=r * 2)
     np.testing.assert_array_equal(c[3], r * 2)
 
 
