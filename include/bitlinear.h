@@ -9,7 +9,7 @@
  *
  *   gamma   = mean |W|                                   (absmean, per tensor)
  *   W~      = RoundClip(W / (gamma + eps), -1, 1)          in {-1, 0, +1}
- *   n       = RMSNorm(x)                                  (optional, per token)
+ *   n       = RMSNorm(x) = x * r,  r = 1/sqrt(mean(x^2)+e) (optional, per token)
  *   beta_t  = max_k |n_tk|                                 (absmax, per token)
  *   X~      = RoundClip(n * 127 / (beta + eps), -127, 127) int8
  *   Y       = (X~ W~^T) * beta * gamma / 127               int32 accumulate
@@ -71,8 +71,13 @@ typedef enum {
 #define BITLINEAR_OUT_F32 0
 #define BITLINEAR_OUT_BF16 1
 
-/* Flags of bitlinear_quant_act. */
+/* Flags of bitlinear_quant_act and bitlinear_linear. */
 #define BITLINEAR_RMSNORM 1u
+/* bitlinear_linear only: the caller guarantees that no work still in flight
+ * on the stream writes `packed` or `gamma`, so the product kernel may start
+ * reading them before earlier work completes (decode layers with fixed
+ * weights: the next layer's weight stream overlaps the current layer). */
+#define BITLINEAR_STATIC_WEIGHTS 2u
 
 /* Library ABI version (this header: 1). */
 int bitlinear_version(void);
@@ -150,21 +155,22 @@ int bitlinear_pack_weights_noalloc(const float *W, int64_t d_out, int64_t d_in,
  *   norm_gain  fp32 [d_in] RMSNorm gain, or NULL for all ones.
  *   flags      BITLINEAR_RMSNORM to normalise first, 0 to quantise X as is.
  *   eps        the epsilon of 127 / (beta + eps); finite, >= 0.
- *   norm_eps   the epsilon inside the RMS: rms = sqrt(mean(x^2) + norm_eps),
- *              formed in double and rounded once to fp32; finite, >= 0.
- *   rms_in     fp32 [T] per-token rms to use instead of computing it, or NULL.
+ *   norm_eps   the epsilon inside the RMS; finite, >= 0.  The reciprocal RMS
+ *              r = 1 / sqrt(mean(x^2) + norm_eps) is formed in double (sum of
+ *              squares in a fixed order) and rounded once to fp32.
+ *   inv_rms_in fp32 [T] per-token r to use instead of computing it, or NULL.
  *   Xq         out: int8 [T][d_in] activation codes in [-127, 127].
  *   beta       out: fp32 [T] per-token absmax of the (normalised) row.
  *   rowsum     out: int32 [T] sum of each row of Xq (consumed by forward).
- *   rms_out    out: fp32 [T] rms used, or NULL.
- * n = x / rms is one binary32 division (times the gain, one multiplication);
- * the scale 127 / (beta + eps) is one binary32 addition and one division,
+ *   inv_rms_out out: fp32 [T] r used, or NULL.
+ * n = x * r is one binary32 multiplication (times the gain, one more); the
+ * scale 127 / (beta + eps) is one binary32 addition and one division,
  * applied with one multiplication; floor(v + 0.5) is then taken exactly.
  */
 int bitlinear_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                         const float *norm_gain, uint32_t flags, float eps,
-                        float norm_eps, const float *rms_in, int8_t *Xq,
-                        float *beta, int32_t *rowsum, float *rms_out,
+                        float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                        float *beta, int32_t *rowsum, float *inv_rms_out,
                         cudaStream_t stream);
 
 /*
@@ -196,13 +202,17 @@ int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
 
 /*
  * bitlinear_linear -- the whole BitLinear forward from bf16 activations:
- * bitlinear_quant_act (with rms computed, rms_in = NULL) followed by
- * bitlinear_forward, with the same arguments, meaning and results as those
- * two calls made back to back ([MF] section 2, all three parts).  Xq, beta
- * and rowsum are caller-owned intermediates of T*d_in, T and T elements.
- * The product kernel is launched as a programmatic dependent of the
- * quantiser so that its weight stream overlaps the quantisation; it reads
- * the codes only after the quantiser has finished.
+ * bitlinear_quant_act (with r computed, inv_rms_in = NULL) followed by
+ * bitlinear_forward, with the same arguments, meaning and results (bit for
+ * bit) as those two calls made back to back ([MF] section 2, all three
+ * parts).  flags: BITLINEAR_RMSNORM, BITLINEAR_STATIC_WEIGHTS.  Xq, beta and
+ * rowsum are caller-owned intermediates of T*d_in, T and T elements, written
+ * with the codes, absmax and row sums.  For T <= 8 with T*d_in <= 32768 one
+ * kernel quantises (in shared memory, per CTA) and multiplies; otherwise the
+ * quantiser runs first and the product kernel is its programmatic dependent.
+ * Kernels are launched as programmatic dependents of the work before them
+ * and read nothing earlier work produces before their dependency wait,
+ * except the weights under BITLINEAR_STATIC_WEIGHTS.
  */
 int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
                      int64_t d_in, const uint16_t *X, int64_t T,

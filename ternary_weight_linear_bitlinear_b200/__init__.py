@@ -26,6 +26,7 @@ LIB_PATH = os.path.join(_PKG, "libbitlinear.so")
 OUT_F32 = 0
 OUT_BF16 = 1
 RMSNORM = 1
+STATIC_WEIGHTS = 2
 
 OK = 0
 ERR_INVALID_ARG = 1
@@ -152,10 +153,11 @@ def pack_weights(W: torch.Tensor, eps: float = 1e-5, gamma: torch.Tensor = None,
 
 
 def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
-              eps: float = 1e-5, norm_eps: float = 1e-5, rms: torch.Tensor = None):
+              eps: float = 1e-5, norm_eps: float = 1e-5, inv_rms: torch.Tensor = None):
     """Fused RMSNorm + per-token absmax int8 codes of bf16 X [T][d_in].
 
-    Returns (Xq int8 [T][d_in], beta f32 [T], rowsum int32 [T], rms f32 [T]).
+    Returns (Xq int8 [T][d_in], beta f32 [T], rowsum int32 [T], inv_rms f32 [T]),
+    inv_rms being the per-token reciprocal RMS used (or given).
     """
     _need(X, torch.bfloat16, "X")
     T, d_in = X.shape
@@ -166,10 +168,10 @@ def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
     rms_out = torch.empty(T, dtype=torch.float32, device=dev)
     if gain is not None:
         _need(gain, torch.float32, "gain")
-    if rms is not None:
-        _need(rms, torch.float32, "rms")
+    if inv_rms is not None:
+        _need(inv_rms, torch.float32, "inv_rms")
     st = lib().bitlinear_quant_act(_ptr(X), T, d_in, _ptr(gain), RMSNORM if rmsnorm else 0,
-                                   eps, norm_eps, _ptr(rms), _ptr(Xq), _ptr(beta),
+                                   eps, norm_eps, _ptr(inv_rms), _ptr(Xq), _ptr(beta),
                                    _ptr(rowsum), _ptr(rms_out), _stream())
     _check(st, "bitlinear_quant_act")
     return Xq, beta, rowsum, rms_out
@@ -194,8 +196,14 @@ def forward(w: PackedTernary, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torc
 
 def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
            eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.float32,
-           out: torch.Tensor = None, scratch=None):
-    """The whole BitLinear forward from bf16 X: quantise, then product."""
+           out: torch.Tensor = None, scratch=None, static_weights: bool = False):
+    """The whole BitLinear forward from bf16 X: quantise, then product.
+
+    static_weights: promise that no work still in flight on the stream
+    writes w.packed or w.gamma (the product may then stream the weights
+    before earlier work has finished).  ``scratch`` = (Xq, beta, rowsum)
+    receives the intermediates.
+    """
     _need(X, torch.bfloat16, "X")
     T = X.shape[0]
     dev = X.device
@@ -207,8 +215,11 @@ def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm
     if out is None:
         out = torch.empty((T, w.d_out), dtype=out_dtype, device=dev)
     od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
+    if gain is not None:
+        _need(gain, torch.float32, "gain")
+    flags = (RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
     st = lib().bitlinear_linear(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(X), T,
-                                _ptr(gain), RMSNORM if rmsnorm else 0, eps, norm_eps,
+                                _ptr(gain), flags, eps, norm_eps,
                                 _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
     _check(st, "bitlinear_linear")
     return out

@@ -11,12 +11,19 @@ namespace bl {
 
 bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                                   const float *norm_gain, uint32_t flags, float eps,
-                                  float norm_eps, const float *rms_in, int8_t *Xq, float *beta,
-                                  int32_t *rowsum, float *rms_out, cudaStream_t stream);
+                                  float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                  float *beta, int32_t *rowsum, float *inv_rms_out, bool pdl,
+                                  cudaStream_t stream);
 bitlinear_status launch_gemv(const uint32_t *packed, const float *gamma, int64_t d_out,
                              int64_t d_in, const int8_t *Xq, const float *beta,
                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                             int32_t *acc_out, bool pdl, cudaStream_t stream);
+                             int32_t *acc_out, bool static_weights, cudaStream_t stream);
+bool decode_can_fuse(int64_t T, int64_t d_in);
+bitlinear_status launch_linear_fused(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                     int64_t d_in, const uint16_t *X, int64_t T,
+                                     const float *gain, bool rmsnorm, float eps, float norm_eps,
+                                     int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
+                                     int out_dtype, bool static_weights, cudaStream_t stream);
 bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int64_t d_out,
                                 int64_t d_in, const int8_t *Xq, const float *beta,
                                 const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
@@ -74,6 +81,29 @@ bitlinear_status get_ctx(DeviceCtx *ctx) {
     return BITLINEAR_OK;
 }
 
+cudaError_t ensure_dynamic_smem(const void *kernel, size_t bytes) {
+    struct Entry { const void *kernel; int dev; size_t bytes; };
+    static Entry entries[256];
+    static int n_entries = 0;
+    if (bytes <= 16 * 1024) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < n_entries; ++i)
+        if (entries[i].kernel == kernel && entries[i].dev == dev && entries[i].bytes >= bytes)
+            return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < n_entries; ++i)
+        if (entries[i].kernel == kernel && entries[i].dev == dev) {
+            entries[i].bytes = bytes;
+            return cudaSuccess;
+        }
+    if (n_entries < 256) entries[n_entries++] = {kernel, dev, bytes};
+    return cudaSuccess;
+}
+
 static bitlinear_status validate_forward(const uint32_t *packed, const float *gamma,
                                          int64_t d_out, int64_t d_in, int64_t T, void *Y,
                                          int out_dtype, int32_t *acc_out) {
@@ -93,11 +123,11 @@ static bitlinear_status validate_forward(const uint32_t *packed, const float *ga
 static bitlinear_status dispatch_forward(const uint32_t *packed, const float *gamma,
                                          int64_t d_out, int64_t d_in, const int8_t *Xq,
                                          const float *beta, const int32_t *rowsum, int64_t T,
-                                         void *Y, int out_dtype, int32_t *acc_out, bool pdl,
-                                         cudaStream_t stream) {
+                                         void *Y, int out_dtype, int32_t *acc_out,
+                                         bool static_weights, cudaStream_t stream) {
     if (T <= 16)
         return launch_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                           acc_out, pdl, stream);
+                           acc_out, static_weights, stream);
     return launch_gemm_tc(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype, acc_out,
                           stream);
 }
@@ -144,7 +174,7 @@ extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int6
                                 cudaStream_t stream) {
     bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, nullptr);
     if (st != BITLINEAR_OK) return st;
-    if (flags & ~BITLINEAR_RMSNORM) return BITLINEAR_ERR_INVALID_ARG;
+    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_STATIC_WEIGHTS)) return BITLINEAR_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !std::isfinite(eps) || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps))
         return BITLINEAR_ERR_INVALID_ARG;
     if (T == 0) return BITLINEAR_OK;
@@ -154,14 +184,19 @@ extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int6
         return BITLINEAR_ERR_MISALIGNED;
     st = check_device();
     if (st != BITLINEAR_OK) return st;
-    st = launch_quant_act(X, T, d_in, norm_gain, flags, eps, norm_eps, nullptr, Xq, beta, rowsum,
-                          nullptr, stream);
+    const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
+    const bool rmsnorm = (flags & BITLINEAR_RMSNORM) != 0;
+    if (decode_can_fuse(T, d_in))
+        return launch_linear_fused(packed, gamma, d_out, d_in, X, T, norm_gain, rmsnorm, eps,
+                                   norm_eps, Xq, beta, rowsum, Y, out_dtype, static_weights,
+                                   stream);
+    // Quantiser, then the product as its programmatic dependent: with static
+    // weights the product streams them while the codes are still being made.
+    st = launch_quant_act(X, T, d_in, norm_gain, flags & BITLINEAR_RMSNORM, eps, norm_eps,
+                          nullptr, Xq, beta, rowsum, nullptr, true, stream);
     if (st != BITLINEAR_OK) return st;
-    // The product is launched as a programmatic dependent of the quantiser:
-    // it may start streaming weights while the codes are still being written
-    // and waits for them before reading.
     return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                            nullptr, true, stream);
+                            nullptr, static_weights, stream);
 }
 
 extern "C" int bitlinear_device_error(cudaStream_t stream, int clear) {

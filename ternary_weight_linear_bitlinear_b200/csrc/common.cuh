@@ -19,6 +19,9 @@ struct DeviceCtx {
 
 // Host side: error-word address and wait limit for the current device.
 bitlinear_status get_ctx(DeviceCtx *ctx);
+// Host side: opt `kernel` in to `bytes` of dynamic shared memory on the
+// current device (once per kernel, device and size increase).
+cudaError_t ensure_dynamic_smem(const void *kernel, size_t bytes);
 // Host side: check the current device is sm_100.
 bitlinear_status check_device();
 

@@ -9,39 +9,91 @@
 // here the unpacking feeds the int8 tensor-core MMA instead, which does the
 // same additions with far fewer issued instructions.
 //
-// Work decomposition: one CTA per 16-row tile of W~, its 8 warps splitting
-// the 256-column tiles of that row band.  A warp streams one 1 KiB packed
-// tile per step with two fully coalesced 16-byte loads per lane (lane l
-// reads bytes 16l.. of rows 0..7 and of rows 8..15) and keeps `D` tiles in
-// flight.  Lane (g = l/4, q = l%4) then holds words 4q..4q+3 of rows g and
-// g+8, i.e. the A fragments of m16n8k32 MMAs under a permutation of the
-// reduction index that the activation fragments follow too:
+// Work decomposition.  Row tiles (16 rows of W~) are taken R at a time
+// ("groups"); a persistent CTA owns a contiguous run of groups, so it streams
+// its packed weights in address order.  The CTA is warp-specialised: one
+// producer warp issues bulk asynchronous copies (the TMA engine) of whole
+// K-slabs -- for each row tile of a group, `ks` consecutive 1 KiB packed
+// tiles, one contiguous copy -- into a ring of shared-memory stages, plus the
+// matching activation codes unless they were quantised in shared memory; four
+// consumer warps take the k-blocks of a stage in turn (warp w: blocks w,
+// w+4, ...) and release the stage through an "empty" barrier.
+//
+// MMA fragments straight from the packed layout.  In a 1 KiB tile lane l
+// reads bytes 16l.. of rows 0..7 and of rows 8..15 (conflict-free), so lane
+// (g = l/4, q = l%4) holds words 4q..4q+3 of rows g and g+8, i.e. the A
+// fragments of m16n8k32 MMAs under a permutation of the reduction index that
+// the activation fragments follow too:
 //   MMA (p, s), p in {0,1}, s in {0..3}:
 //     a0/a2 = word 4q+2p / 4q+2p+1 of row g  masked to slot s,
 //     a1/a3 = the same words of row g+8,
 //     b0/b1 = activation bytes 64q+32p+4s.. and 64q+32p+16+4s.. of token g.
 // Masking slot s without shifting leaves the codes scaled by 4^s (at most
-// 2*64 = 128, a valid u8), so each slot has its own accumulator and the
-// four are combined exactly as acc0 + acc1/4 + acc2/16 + acc3/64 at the end.
-// Codes are c = W~ + 1; the epilogue subtracts the activation row sum.
+// 2*64 = 128, a valid u8), so each slot has its own accumulator and the four
+// are combined exactly as acc0 + acc1/4 + acc2/16 + acc3/64.  Codes are
+// c = W~ + 1; the epilogue subtracts the activation row sum.
+//
+// FUSED variant: the consumer warps first quantise the bf16 activations
+// themselves (the routine of quant_common.cuh, same order as the stand-alone
+// quantiser) into shared memory, so a whole decode BitLinear forward is one
+// kernel.
+//
+// Dependent launch: every variant is launched as a programmatic dependent of
+// the previous kernel in the stream.  Nothing produced earlier is read before
+// griddepcontrol.wait, except the packed weights and gamma when the caller
+// declared them static (not written by work still in flight): then the
+// weight stream of this layer overlaps the tail of the previous one.
+//
+// Every mbarrier wait is bounded; on expiry the CTA stops consuming, the
+// producer waits (bounded) for the copies it issued, and the error word is
+// set.
 #include <cstdint>
 
 #include <cuda_bf16.h>
 
 #include "bitlinear.h"
 #include "common.cuh"
+#include "quant_common.cuh"
 
 namespace bl {
 
-constexpr int kGemvWarps = 8;
+constexpr int kDecWarps = 4;                          // consumer warps
+constexpr int kDecThreads = (kDecWarps + 1) * 32;      // + one producer warp
+constexpr int kDecMaxStages = 4;
+static_assert(kDecWarps * 32 == kQuantThreads, "fused quantiser runs on the consumer warps");
 
-__device__ __forceinline__ uint4 ld_stream_v4(const uint4 *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
+struct DecodeArgs {
+    const uint4 *packed;
+    const float *gamma;
+    int d_out;
+    int kb_total;            // d_in / 256
+    int T;
+    // product-only inputs (written by the stand-alone quantiser)
+    const int8_t *Xq;
+    const float *beta;
+    const int32_t *rowsum;
+    // fused inputs and the intermediates CTA 0 writes back
+    const uint16_t *X;
+    const float *gain;
+    int rmsnorm;
+    float eps;
+    float norm_eps;
+    int8_t *Xq_out;
+    float *beta_out;
+    int32_t *rowsum_out;
+    // outputs
+    void *Y;
+    int32_t *acc_out;
+    int static_weights;
+};
+
+struct DecodePlan {
+    int ks;            // k-blocks per slab
+    int nslab;         // slabs per row tile
+    int stages;        // ring depth
+    int stage_bytes;   // R * ks KiB of weights + T * ks * 256 B of codes (unfused)
+    int xs_bytes;      // fused: T * K codes, rounded up to 128
+};
 
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -52,170 +104,426 @@ __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int NT, int D, bool OUT_BF16>
-__global__ void __launch_bounds__(kGemvWarps * 32)
-gemv_kernel(const uint4 *__restrict__ packed, const float *__restrict__ gamma_ptr, int d_out,
-            int kb_total, const int8_t *__restrict__ Xq, const float *__restrict__ beta,
-            const int32_t *__restrict__ rowsum, int T, void *__restrict__ Y,
-            int32_t *__restrict__ acc_out) {
-    __shared__ int4 red[kGemvWarps][NT][32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, q = lane & 3;
-    const int rt = blockIdx.x;
-    const int kb_begin = (kb_total * warp) / kGemvWarps;
-    const int nblk = (kb_total * (warp + 1)) / kGemvWarps - kb_begin;
-    const int d_in = kb_total * 256;
+// Bulk (TMA-engine) copy of `bytes` contiguous bytes global -> shared,
+// completing on an mbarrier.  Both addresses 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
 
-    // Tile (rt, kb) starts at uint4 index (rt * kb_total + kb) * 64.
-    const uint4 *wsrc = packed + ((size_t)rt * kb_total + kb_begin) * 64 + lane;
+__device__ __forceinline__ void consumer_barrier() {
+    asm volatile("bar.sync 2, %0;" ::"n"(kDecWarps * 32) : "memory");
+}
 
-    // The weights are not written by the kernel this one may overlap with,
-    // so they stream in before the dependency wait.
-    uint4 wa[D], wb[D];
-    #pragma unroll
-    for (int d = 0; d < D; ++d) {
-        if (d < nblk) {
-            wa[d] = ld_stream_v4(wsrc + d * 64);
-            wb[d] = ld_stream_v4(wsrc + d * 64 + 32);
+// Bounded wait that also gives up once another role has aborted.
+__device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, const DeviceCtx &ctx,
+                                         volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > ctx.wait_ns) {
+            atomicOr(ctx.err, kErrTimeout);
+            *abort_flag = 1;
+            return false;
         }
     }
+}
 
-    pdl_wait_primary();
+template <int NT, int R, bool FUSED, bool OUT_BF16>
+__global__ void __launch_bounds__(kDecThreads)
+decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx ctx) {
+    constexpr int TMAX = NT * 8;
+    extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ __align__(8) uint64_t full_bar[kDecMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kDecMaxStages];
+    __shared__ QuantShared<FUSED ? TMAX : 1> qs;
+    __shared__ int4 red[kDecWarps][R][NT][32];
+    __shared__ float s_yscale[TMAX];
+    __shared__ int s_rowsum[TMAX];
+    __shared__ int s_abort;
 
-    int acc[NT][4][4];
-    #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-        #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            #pragma unroll
-            for (int r = 0; r < 4; ++r) acc[nt][s][r] = 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB = a.kb_total, K = KB * 256, T = a.T;
+    const int n_rt = a.d_out >> 4;
+    const int n_groups = (n_rt + R - 1) / R;
+    const int grp0 = (int)(((long long)n_groups * blockIdx.x) / gridDim.x);
+    const int ngrp = (int)(((long long)n_groups * (blockIdx.x + 1)) / gridDim.x) - grp0;
+    const int ks = plan.ks, nslab = plan.nslab, stages = plan.stages;
+    const int stage_bytes = plan.stage_bytes;
+    const int units = ngrp * nslab;
+    int8_t *xs = reinterpret_cast<int8_t *>(dsm);
+    uint8_t *ring = dsm + plan.xs_bytes;
+    const uint32_t ring_s = smem_u32(ring);
+    volatile int *abort_flag = &s_abort;
 
-    const uint4 *xsrc[NT];
-    bool xvalid[NT];
-    #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int t = nt * 8 + g;
-        xvalid[nt] = t < T;
-        xsrc[nt] = reinterpret_cast<const uint4 *>(Xq + (size_t)(xvalid[nt] ? t : 0) * d_in +
-                                                   (size_t)kb_begin * 256 + 64 * q);
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < stages; ++st) {
+            mbar_init(smem_u32(&full_bar[st]), 1);
+            mbar_init(smem_u32(&empty_bar[st]), kDecWarps);
+        }
+        s_abort = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    if (warp == kDecWarps) {
+        // ------------------------------------------------------ producer ---
+        if (lane == 0) {
+            // Unit (gi, sl): group grp0 + gi, slab sl; units run gi-major.
+            auto slab_kb = [&](int sl) { return KB - sl * ks < ks ? KB - sl * ks : ks; };
+            auto issue_w = [&](int gi, int sl, int st) {
+                const uint32_t bar = smem_u32(&full_bar[st]);
+                const int rt = (grp0 + gi) * R;
+                const int nkb = slab_kb(sl);
+                int nrow = 0;
+                #pragma unroll
+                for (int r = 0; r < R; ++r) nrow += rt + r < n_rt ? 1 : 0;
+                const uint32_t xbytes = FUSED ? 0u : (uint32_t)(T * nkb * 256);
+                mbar_arrive_expect_tx(bar, (uint32_t)(nrow * nkb * 1024) + xbytes);
+                for (int r = 0; r < nrow; ++r)
+                    bulk_g2s(ring_s + st * stage_bytes + r * ks * 1024,
+                             a.packed + ((size_t)(rt + r) * KB + (size_t)sl * ks) * 64,
+                             (uint32_t)(nkb * 1024), bar);
+            };
+            auto issue_x = [&](int sl, int st) {
+                if (FUSED) return;
+                const uint32_t bar = smem_u32(&full_bar[st]);
+                const int nkb = slab_kb(sl);
+                for (int t = 0; t < T; ++t)
+                    bulk_g2s(ring_s + st * stage_bytes + R * ks * 1024 + t * ks * 256,
+                             a.Xq + (size_t)t * K + (size_t)sl * ks * 256, (uint32_t)(nkb * 256),
+                             bar);
+            };
+            const int first = units < stages ? units : stages;
+            if (a.static_weights) {
+                int gi = 0, sl = 0;
+                for (int u = 0; u < first; ++u) {
+                    issue_w(gi, sl, u);
+                    if (++sl == nslab) { sl = 0; ++gi; }
+                }
+            }
+            pdl_wait_primary();
+            pdl_launch_dependents();
+            int gi = 0, sl = 0, st = 0, round = 0, issued = 0;
+            for (int u = 0; u < units; ++u) {
+                if (round > 0) {
+                    // Stage st was last used by unit u - stages: wait for its
+                    // release (completion number round - 1 of its barrier).
+                    if (!dec_wait(smem_u32(&empty_bar[st]), (uint32_t)(round - 1) & 1u, ctx,
+                                  abort_flag))
+                        break;
+                    issue_w(gi, sl, st);
+                } else if (!a.static_weights) {
+                    issue_w(gi, sl, st);
+                }
+                issue_x(sl, st);
+                ++issued;
+                if (++sl == nslab) { sl = 0; ++gi; }
+                if (++st == stages) { st = 0; ++round; }
+            }
+            // Every copy issued must land before the CTA may exit.
+            for (int u = issued > stages ? issued - stages : 0; u < issued; ++u)
+                mbar_wait_bounded(smem_u32(&full_bar[u % stages]), (uint32_t)(u / stages) & 1u,
+                                  ctx);
+        } else {
+            pdl_wait_primary();
+            pdl_launch_dependents();
+        }
+        return;
     }
 
-    for (int i0 = 0; i0 < nblk; i0 += D) {
+    // ------------------------------------------------------- consumers ---
+    pdl_wait_primary();
+    pdl_launch_dependents();
+    const int g = lane >> 2, q = lane & 3;
+    const float gamma = *a.gamma;
+    if constexpr (FUSED) {
+        token_stats<TMAX>(a.X, T, K, a.gain, a.rmsnorm != 0, a.eps, a.norm_eps, nullptr, qs);
+        token_codes<TMAX>(a.X, T, K, a.gain, a.rmsnorm != 0, xs, qs);
+        if (threadIdx.x < T) {
+            const int t = threadIdx.x;
+            s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, qs.beta[t]), 127.0f);
+            s_rowsum[t] = qs.rowsum[t];
+            if (blockIdx.x == 0) {
+                if (a.beta_out) a.beta_out[t] = qs.beta[t];
+                if (a.rowsum_out) a.rowsum_out[t] = qs.rowsum[t];
+            }
+        }
+        if (blockIdx.x == 0 && a.Xq_out) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(xs);
+            uint4 *dst = reinterpret_cast<uint4 *>(a.Xq_out);
+            for (int v = threadIdx.x; v < (T * K) >> 4; v += kDecWarps * 32) dst[v] = src[v];
+        }
+    } else {
+        if (threadIdx.x < T) {
+            const int t = threadIdx.x;
+            s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, a.beta[t]), 127.0f);
+            s_rowsum[t] = a.rowsum[t];
+        }
+    }
+    consumer_barrier();
+
+    bool ok = true;
+    int st = 0;
+    uint32_t fph = 0;
+    for (int gi = 0; gi < ngrp; ++gi) {
+        int acc[R][NT][4][4];
         #pragma unroll
-        for (int d = 0; d < D; ++d) {
-            const int i = i0 + d;
-            if (i < nblk) {
+        for (int r = 0; r < R; ++r)
+            #pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                #pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[r][nt][s][e] = 0;
+
+        for (int sl = 0; sl < nslab && ok; ++sl) {
+            ok = dec_wait(smem_u32(&full_bar[st]), fph, ctx, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            const uint8_t *stage = ring + st * stage_bytes;
+            const int nkb = KB - sl * ks < ks ? KB - sl * ks : ks;
+            for (int kk = warp; kk < nkb; kk += kDecWarps) {
+                uint32_t w0[R][4], w1[R][4];
+                #pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const uint8_t *tile = stage + (r * ks + kk) * 1024;
+                    const uint4 lo = *reinterpret_cast<const uint4 *>(tile + lane * 16);
+                    const uint4 hi = *reinterpret_cast<const uint4 *>(tile + 512 + lane * 16);
+                    w0[r][0] = lo.x; w0[r][1] = lo.y; w0[r][2] = lo.z; w0[r][3] = lo.w;
+                    w1[r][0] = hi.x; w1[r][1] = hi.y; w1[r][2] = hi.z; w1[r][3] = hi.w;
+                }
                 uint32_t xr[NT][16];
                 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
+                    const int t = nt * 8 + g;
+                    const uint8_t *xsrc =
+                        FUSED ? reinterpret_cast<const uint8_t *>(xs) + (size_t)t * K +
+                                    (size_t)(sl * ks + kk) * 256 + 64 * q
+                              : stage + R * ks * 1024 + (t * ks + kk) * 256 + 64 * q;
                     #pragma unroll
                     for (int v = 0; v < 4; ++v) {
-                        uint4 x = xvalid[nt] ? __ldg(xsrc[nt] + i * 16 + v) : make_uint4(0, 0, 0, 0);
+                        uint4 x = make_uint4(0, 0, 0, 0);
+                        if (t < T) x = *reinterpret_cast<const uint4 *>(xsrc + 16 * v);
                         xr[nt][4 * v + 0] = x.x;
                         xr[nt][4 * v + 1] = x.y;
                         xr[nt][4 * v + 2] = x.z;
                         xr[nt][4 * v + 3] = x.w;
                     }
                 }
-                const uint32_t w0[4] = {wa[d].x, wa[d].y, wa[d].z, wa[d].w};
-                const uint32_t w1[4] = {wb[d].x, wb[d].y, wb[d].z, wb[d].w};
-                if (i + D < nblk) {
-                    wa[d] = ld_stream_v4(wsrc + (i + D) * 64);
-                    wb[d] = ld_stream_v4(wsrc + (i + D) * 64 + 32);
-                }
                 #pragma unroll
-                for (int p = 0; p < 2; ++p) {
+                for (int r = 0; r < R; ++r) {
                     #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        const uint32_t m = 0x03030303u << (2 * s);
-                        const uint32_t a0 = w0[2 * p] & m, a2 = w0[2 * p + 1] & m;
-                        const uint32_t a1 = w1[2 * p] & m, a3 = w1[2 * p + 1] & m;
+                    for (int p = 0; p < 2; ++p) {
                         #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-                            mma_u8s8(acc[nt][s], a0, a1, a2, a3, xr[nt][8 * p + s],
-                                     xr[nt][8 * p + 4 + s]);
+                        for (int s = 0; s < 4; ++s) {
+                            const uint32_t m = 0x03030303u << (2 * s);
+                            const uint32_t a0 = w0[r][2 * p] & m, a2 = w0[r][2 * p + 1] & m;
+                            const uint32_t a1 = w1[r][2 * p] & m, a3 = w1[r][2 * p + 1] & m;
+                            #pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                mma_u8s8(acc[r][nt][s], a0, a1, a2, a3, xr[nt][8 * p + s],
+                                         xr[nt][8 * p + 4 + s]);
+                        }
                     }
                 }
             }
+            // This warp is done with the stage.
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+            if (++st == stages) { st = 0; fph ^= 1u; }
         }
-    }
 
-    #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        int c[4];
         #pragma unroll
-        for (int r = 0; r < 4; ++r)
-            c[r] = acc[nt][0][r] + (acc[nt][1][r] >> 2) + (acc[nt][2][r] >> 4) +
-                   (acc[nt][3][r] >> 6);
-        red[warp][nt][lane] = make_int4(c[0], c[1], c[2], c[3]);
-    }
-    __syncthreads();
+        for (int r = 0; r < R; ++r)
+            #pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                int c[4];
+                #pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    c[e] = acc[r][nt][0][e] + (acc[r][nt][1][e] >> 2) +
+                           (acc[r][nt][2][e] >> 4) + (acc[r][nt][3][e] >> 6);
+                red[warp][r][nt][lane] = make_int4(c[0], c[1], c[2], c[3]);
+            }
+        consumer_barrier();
 
-    // Epilogue: thread i -> (token t = i / 16, row r = i % 16), so a warp
-    // stores two tokens' 16 consecutive outputs.
-    const int i = threadIdx.x;
-    const int t = i >> 4, r = i & 15;
-    if (t < T) {
-        const int gg = r & 7, half = r >> 3;
-        const int nt = t >> 3, tt = t & 7;
-        const int src_lane = gg * 4 + (tt >> 1);
-        const int reg = (tt & 1) + 2 * half;
-        int v = 0;
-        #pragma unroll
-        for (int w = 0; w < kGemvWarps; ++w) {
-            const int *e = reinterpret_cast<const int *>(&red[w][nt][src_lane]);
-            v += e[reg];
+        // Epilogue of this group: output i -> (token t, row tile r, row), rows
+        // fastest, so consecutive threads store consecutive outputs.
+        const int rt0 = (grp0 + gi) * R;
+        const int per_t = 16 * R;
+        for (int idx = threadIdx.x; idx < T * per_t; idx += kDecWarps * 32) {
+            const int t = idx / per_t, rem = idx - t * per_t;
+            const int r = rem >> 4, row = rem & 15;
+            if (rt0 + r >= n_rt) continue;
+            const int gg = row & 7, half = row >> 3;
+            const int nt = t >> 3, tt = t & 7;
+            const int src_lane = gg * 4 + (tt >> 1);
+            const int reg = (tt & 1) + 2 * half;
+            int v = 0;
+            #pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) {
+                const int *e = reinterpret_cast<const int *>(&red[w][r][nt][src_lane]);
+                v += e[reg];
+            }
+            const int accv = v - s_rowsum[t];
+            const int o = (rt0 + r) * 16 + row;
+            const size_t yi = (size_t)t * a.d_out + o;
+            if (a.acc_out) a.acc_out[yi] = accv;
+            const float y = __fmul_rn((float)accv, s_yscale[t]);
+            if (OUT_BF16)
+                reinterpret_cast<__nv_bfloat16 *>(a.Y)[yi] = __float2bfloat16_rn(y);
+            else
+                reinterpret_cast<float *>(a.Y)[yi] = y;
         }
-        const int a = v - rowsum[t];
-        const int o = rt * 16 + r;
-        const size_t idx = (size_t)t * d_out + o;
-        if (acc_out) acc_out[idx] = a;
-        const float scale = __fdiv_rn(__fmul_rn(*gamma_ptr, beta[t]), 127.0f);
-        const float y = __fmul_rn((float)a, scale);
-        if (OUT_BF16)
-            reinterpret_cast<__nv_bfloat16 *>(Y)[idx] = __float2bfloat16_rn(y);
-        else
-            reinterpret_cast<float *>(Y)[idx] = y;
+        consumer_barrier();
     }
 }
 
-template <int NT, bool OUT_BF16>
-static cudaError_t launch_gemv_t(const uint32_t *packed, const float *gamma, int d_out, int d_in,
-                                 const int8_t *Xq, const float *beta, const int32_t *rowsum,
-                                 int T, void *Y, int32_t *acc_out, bool pdl,
-                                 cudaStream_t stream) {
-    constexpr int D = 4;
+// Compile-time tuning knobs (defaults are the measured choices).
+#ifndef BL_FUSED_MAX_CODE_BYTES
+#define BL_FUSED_MAX_CODE_BYTES 32768   // largest T * d_in quantised inside the GEMV CTA
+#endif
+#ifndef BL_DEC_WIDE_ROW_TILES
+#define BL_DEC_WIDE_ROW_TILES (148 * 8) // from this many 16-row tiles on, 2 tiles per group
+#endif
+#ifndef BL_DEC_STAGE_BYTES
+#define BL_DEC_STAGE_BYTES 32768        // target bytes per pipeline stage
+#endif
+#ifndef BL_DEC_RING_BYTES
+#define BL_DEC_RING_BYTES 98304         // bytes of all stages of a CTA
+#endif
+#ifndef BL_DEC_CTA_FRACTION
+#define BL_DEC_CTA_FRACTION 1           // persistent grid = resident CTAs / this
+#endif
+constexpr int kFusedMaxCodeBytes = BL_FUSED_MAX_CODE_BYTES;
+
+template <int NT, int R, bool FUSED, bool OUT_BF16>
+static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
+                                   cudaStream_t stream) {
+    const int n_rt = args.d_out / 16;
+    const int n_groups = (n_rt + R - 1) / R;
+    const int KB = args.kb_total, K = KB * 256;
+    DecodePlan plan;
+    plan.xs_bytes = FUSED ? ((args.T * K + 127) & ~127) : 0;
+    const int per_kb = R * 1024 + (FUSED ? 0 : args.T * 256);   // bytes per k-block column
+    plan.ks = BL_DEC_STAGE_BYTES / per_kb;
+    if (plan.ks < 1) plan.ks = 1;
+    if (plan.ks > KB) plan.ks = KB;
+    plan.nslab = (KB + plan.ks - 1) / plan.ks;
+    plan.stage_bytes = plan.ks * per_kb;
+    plan.stages = BL_DEC_RING_BYTES / plan.stage_bytes;
+    if (plan.stages > kDecMaxStages) plan.stages = kDecMaxStages;
+    // No deeper than the units a CTA can get when up to 8 CTAs fit per SM.
+    const int min_units = ((n_groups + 148 * 8 - 1) / (148 * 8)) * plan.nslab;
+    if (plan.stages > min_units) plan.stages = min_units;
+    if (plan.stages < 2) plan.stages = 2;
+    const size_t smem = (size_t)plan.xs_bytes + (size_t)plan.stages * plan.stage_bytes;
+    auto kern = decode_kernel<NT, R, FUSED, OUT_BF16>;
+    cudaError_t e = ensure_dynamic_smem((const void *)kern, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem) !=
+            cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    int max_ctas = sms * per_sm / BL_DEC_CTA_FRACTION;
+    if (max_ctas < sms) max_ctas = sms;
+    const int grid = n_groups < max_ctas ? n_groups : max_ctas;
+
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(d_out / 16));
-    cfg.blockDim = dim3(kGemvWarps * 32);
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, D, OUT_BF16>,
-                              reinterpret_cast<const uint4 *>(packed), gamma, d_out, d_in / 256,
-                              Xq, beta, rowsum, T, Y, acc_out);
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args, plan, ctx);
+}
+
+template <bool FUSED, bool OUT_BF16>
+static cudaError_t launch_decode_r(const DecodeArgs &args, const DeviceCtx &ctx,
+                                   cudaStream_t stream) {
+    // One row tile per group while that still leaves a few CTAs per SM;
+    // larger matrices share each activation fragment over two row tiles.
+    const int n_rt = args.d_out / 16;
+    const bool wide = n_rt >= BL_DEC_WIDE_ROW_TILES;
+    if (args.T <= 8)
+        return wide ? launch_decode_t<1, 2, FUSED, OUT_BF16>(args, ctx, stream)
+                    : launch_decode_t<1, 1, FUSED, OUT_BF16>(args, ctx, stream);
+    if constexpr (FUSED) return cudaErrorInvalidValue;   // fused path is T <= 8 only
+    return wide ? launch_decode_t<2, 2, false, OUT_BF16>(args, ctx, stream)
+                : launch_decode_t<2, 1, false, OUT_BF16>(args, ctx, stream);
+}
+
+bool decode_can_fuse(int64_t T, int64_t d_in) {
+    return T >= 1 && T <= 8 && T * d_in <= kFusedMaxCodeBytes;
+}
+
+bitlinear_status launch_decode(const DecodeArgs &args, bool fused, int out_dtype,
+                               cudaStream_t stream) {
+    DeviceCtx ctx;
+    bitlinear_status st = get_ctx(&ctx);
+    if (st != BITLINEAR_OK) return st;
+    cudaError_t e;
+    const bool bf = out_dtype == BITLINEAR_OUT_BF16;
+    if (fused)
+        e = bf ? launch_decode_r<true, true>(args, ctx, stream)
+               : launch_decode_r<true, false>(args, ctx, stream);
+    else
+        e = bf ? launch_decode_r<false, true>(args, ctx, stream)
+               : launch_decode_r<false, false>(args, ctx, stream);
+    return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
 bitlinear_status launch_gemv(const uint32_t *packed, const float *gamma, int64_t d_out,
                              int64_t d_in, const int8_t *Xq, const float *beta,
                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                             int32_t *acc_out, bool pdl, cudaStream_t stream) {
-    cudaError_t e;
-    const bool bf = out_dtype == BITLINEAR_OUT_BF16;
-    if (T <= 8)
-        e = bf ? launch_gemv_t<1, true>(packed, gamma, (int)d_out, (int)d_in, Xq, beta, rowsum,
-                                        (int)T, Y, acc_out, pdl, stream)
-               : launch_gemv_t<1, false>(packed, gamma, (int)d_out, (int)d_in, Xq, beta, rowsum,
-                                         (int)T, Y, acc_out, pdl, stream);
-    else
-        e = bf ? launch_gemv_t<2, true>(packed, gamma, (int)d_out, (int)d_in, Xq, beta, rowsum,
-                                        (int)T, Y, acc_out, pdl, stream)
-               : launch_gemv_t<2, false>(packed, gamma, (int)d_out, (int)d_in, Xq, beta, rowsum,
-                                         (int)T, Y, acc_out, pdl, stream);
-    return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+                             int32_t *acc_out, bool static_weights, cudaStream_t stream) {
+    DecodeArgs a = {};
+    a.packed = reinterpret_cast<const uint4 *>(packed);
+    a.gamma = gamma;
+    a.d_out = (int)d_out;
+    a.kb_total = (int)(d_in / 256);
+    a.T = (int)T;
+    a.Xq = Xq;
+    a.beta = beta;
+    a.rowsum = rowsum;
+    a.Y = Y;
+    a.acc_out = acc_out;
+    a.static_weights = static_weights ? 1 : 0;
+    return launch_decode(a, false, out_dtype, stream);
+}
+
+bitlinear_status launch_linear_fused(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                     int64_t d_in, const uint16_t *X, int64_t T,
+                                     const float *gain, bool rmsnorm, float eps, float norm_eps,
+                                     int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
+                                     int out_dtype, bool static_weights, cudaStream_t stream) {
+    DecodeArgs a = {};
+    a.packed = reinterpret_cast<const uint4 *>(packed);
+    a.gamma = gamma;
+    a.d_out = (int)d_out;
+    a.kb_total = (int)(d_in / 256);
+    a.T = (int)T;
+    a.X = X;
+    a.gain = gain;
+    a.rmsnorm = rmsnorm ? 1 : 0;
+    a.eps = eps;
+    a.norm_eps = norm_eps;
+    a.Xq_out = Xq;
+    a.beta_out = beta;
+    a.rowsum_out = rowsum;
+    a.Y = Y;
+    a.static_weights = static_weights ? 1 : 0;
+    return launch_decode(a, true, out_dtype, stream);
 }
 
 }  // namespace bl

@@ -1,0 +1,213 @@
+// quant_common.cuh -- per-token RMSNorm / absmax statistics and int8 codes,
+// shared by the stand-alone quantiser and the fused decode kernel so that both
+// reduce in one canonical order and produce bit-identical results.
+//
+// "BitNet b1.58: Mathematical Foundations of 1.58-Bit Ternary Quantization,
+// Absmean Scaling, and Multiplication-Free LLM Architectures", section 2,
+// "Activation Quantization: Absmax Scaling".
+//
+// RMSNorm is n = x * r (* g) with the reciprocal RMS r = 1 / sqrt(mean(x^2) +
+// norm_eps) formed once per token in double and rounded once to binary32.
+// Canonical order (a CTA of kQuantThreads threads): thread i owns the 16-byte
+// vectors i, i + kQuantThreads, ... of a token row and accumulates x^2 in
+// double over them in that order; a warp xor-butterfly combines the 32 lanes;
+// the kQuantWarps warp sums are added in warp order.  Without a gain vector
+// beta = fl(max|x| * r): correctly rounded multiplication by r > 0 is
+// monotone, so this is exactly max_k fl(|x_k| * r).  With a gain it is the
+// max of the normalised values themselves.
+//
+// Tokens are processed in a loop that is not unrolled, keeping the code small
+// (a fully unrolled multi-token version spent most of its time on
+// instruction-cache misses).
+#pragma once
+
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kQuantThreads = 128;
+constexpr int kQuantWarps = kQuantThreads / 32;
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&x)[8]) {
+    x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x);
+    x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
+    x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z);
+    x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
+}
+
+// Shared scratch for the statistics of up to TMAX tokens.
+template <int TMAX>
+struct QuantShared {
+    double ss[kQuantWarps][TMAX];
+    float amax[kQuantWarps][TMAX];
+    int sum[kQuantWarps][TMAX];
+    float inv_rms[TMAX];
+    float beta[TMAX];
+    float scale[TMAX];   // 127 / (beta + eps)
+    int rowsum[TMAX];
+};
+
+// Barrier over the kQuantThreads threads (warps 0..kQuantWarps-1) that run
+// the quantiser; a CTA may hold further warps that do not take part.
+__device__ __forceinline__ void quant_barrier() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kQuantThreads) : "memory");
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max_f32(float v) {
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ int warp_sum_i32(int v) {
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Statistics of tokens 0..T-1 (T <= TMAX) of X [T][K] (bf16 bits).  Threads
+// 0..kQuantThreads-1 of the CTA must all call it.  inv_rms_in, when
+// given, supplies the per-token reciprocal RMS.  Results: qs.inv_rms, beta,
+// scale.
+template <int TMAX>
+__device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int T, int K,
+                                         const float *__restrict__ gain, bool rmsnorm,
+                                         float eps, float norm_eps,
+                                         const float *__restrict__ inv_rms_in,
+                                         QuantShared<TMAX> &qs) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nvec = K >> 3;
+    const bool need_ss = rmsnorm && !inv_rms_in;
+    #pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)t * K);
+        double ss = 0.0;
+        float am = 0.0f;
+        for (int v = tid; v < nvec; v += kQuantThreads) {
+            float x[8];
+            unpack8(__ldg(row + v), x);
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (need_ss) ss += (double)x[j] * (double)x[j];
+                am = fmaxf(am, fabsf(x[j]));
+            }
+        }
+        ss = warp_sum_f64(ss);
+        am = warp_max_f32(am);
+        if (lane == 0) {
+            qs.ss[warp][t] = ss;
+            qs.amax[warp][t] = am;
+        }
+    }
+    quant_barrier();
+    if (tid < T) {
+        const int t = tid;
+        float r = 1.0f;
+        if (rmsnorm) {
+            if (inv_rms_in) {
+                r = inv_rms_in[t];
+            } else {
+                double s = qs.ss[0][t];
+                #pragma unroll
+                for (int w = 1; w < kQuantWarps; ++w) s += qs.ss[w][t];
+                r = (float)__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(s / (double)K, (double)norm_eps)));
+            }
+        }
+        float m = qs.amax[0][t];
+        #pragma unroll
+        for (int w = 1; w < kQuantWarps; ++w) m = fmaxf(m, qs.amax[w][t]);
+        qs.inv_rms[t] = r;
+        qs.beta[t] = rmsnorm ? __fmul_rn(m, r) : m;   // replaced below when a gain is set
+    }
+    quant_barrier();
+    if (rmsnorm && gain) {
+        // With a gain the absmax is that of fl(fl(x * r) * g).
+        #pragma unroll 1
+        for (int t = 0; t < T; ++t) {
+            const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)t * K);
+            const float r = qs.inv_rms[t];
+            float a = 0.0f;
+            for (int v = tid; v < nvec; v += kQuantThreads) {
+                float x[8];
+                unpack8(__ldg(row + v), x);
+                #pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    a = fmaxf(a, fabsf(__fmul_rn(__fmul_rn(x[j], r), __ldg(gain + 8 * v + j))));
+            }
+            a = warp_max_f32(a);
+            if (lane == 0) qs.amax[warp][t] = a;
+        }
+        quant_barrier();
+        if (tid < T) {
+            float m = qs.amax[0][tid];
+            #pragma unroll
+            for (int w = 1; w < kQuantWarps; ++w) m = fmaxf(m, qs.amax[w][tid]);
+            qs.beta[tid] = m;
+        }
+        quant_barrier();
+    }
+    if (tid < T) qs.scale[tid] = __fdiv_rn(127.0f, __fadd_rn(qs.beta[tid], eps));
+    quant_barrier();
+}
+
+// Codes of tokens 0..T-1 written to dst (row stride K bytes; global or shared
+// memory) and their row sums to qs.rowsum.  Call after token_stats.
+template <int TMAX>
+__device__ __forceinline__ void token_codes(const uint16_t *__restrict__ X, int T, int K,
+                                         const float *__restrict__ gain, bool rmsnorm,
+                                         int8_t *dst, QuantShared<TMAX> &qs) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nvec = K >> 3;
+    const bool use_gain = rmsnorm && gain;
+    #pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)t * K);
+        uint2 *out = reinterpret_cast<uint2 *>(dst + (size_t)t * K);
+        const float r = rmsnorm ? qs.inv_rms[t] : 1.0f, scale = qs.scale[t];
+        int sum = 0;
+        for (int v = tid; v < nvec; v += kQuantThreads) {
+            float x[8];
+            unpack8(__ldg(row + v), x);
+            float g[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+            if (use_gain) {
+                #pragma unroll
+                for (int j = 0; j < 8; ++j) g[j] = __ldg(gain + 8 * v + j);
+            }
+            uint32_t lo = 0, hi = 0;
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float n = x[j];
+                if (rmsnorm) n = __fmul_rn(n, r);
+                if (use_gain) n = __fmul_rn(n, g[j]);
+                float q = round_half_up_exact(__fmul_rn(n, scale));
+                q = fminf(fmaxf(q, -127.0f), 127.0f);
+                const int qi = (int)q;
+                sum += qi;
+                const uint32_t b = (uint32_t)(qi & 0xff);
+                if (j < 4) lo |= b << (8 * j); else hi |= b << (8 * (j - 4));
+            }
+            out[v] = make_uint2(lo, hi);
+        }
+        sum = warp_sum_i32(sum);
+        if (lane == 0) qs.sum[warp][t] = sum;
+    }
+    quant_barrier();
+    if (tid < T) {
+        int s = 0;
+        #pragma unroll
+        for (int w = 0; w < kQuantWarps; ++w) s += qs.sum[w][tid];
+        qs.rowsum[tid] = s;
+    }
+    quant_barrier();
+}
+
+}  // namespace bl

@@ -1,13 +1,13 @@
 """Parity of the CUDA path (through the C ABI) with the CPU oracle.
 
 Bars: packed codes, activation codes, row sums and int32 accumulators
-bit-exact; gamma and rms within 1e-6 relative; fp32 outputs within
+bit-exact; gamma and the reciprocal RMS within 1e-6 relative; fp32 outputs within
 1e-5 * max(|y|, scale_t) and bf16 outputs within 1e-2 * max(|y|, scale_t),
 where scale_t = gamma beta_t / 127 is one integer step of the output (the
 floor keeps a relative bound meaningful at acc = 0).
 
 Inputs only flow oracle -> GPU: where integer codes are compared, the GPU is
-handed the oracle's gamma / rms (the GPU's own values are checked separately
+handed the oracle's gamma / reciprocal RMS (the GPU's own values are checked separately
 against the oracle's to 1e-6), so a last-bit difference in a reduction can
 not flip a code and nothing computed on the GPU enters the oracle.
 """
@@ -58,7 +58,7 @@ def oracle_side(W, X, rmsnorm=True, gain=None):
     xb = bf16_bits(X)
     xq, beta, rowsum, rms = oracle.quant_act(xb, gain=gain, rmsnorm=rmsnorm, eps=EPS,
                                              norm_eps=NORM_EPS)
-    return dict(gamma=g, wq=wq, xq=xq, beta=beta, rowsum=rowsum, rms=rms, xb=xb)
+    return dict(gamma=g, wq=wq, xq=xq, beta=beta, rowsum=rowsum, inv_rms=rms, xb=xb)
 
 
 def check_y(y_gpu, acc_ref, gamma, beta, out_bf16, rows=None):
@@ -136,12 +136,12 @@ def test_quant_act_matches_oracle(T, K, frac, factor, rmsnorm, use_gain):
                                                   norm_eps=NORM_EPS)
     Xd = X.to(dev())
     gd = None if gain is None else to_dev(gain)
-    # The GPU's own rms agrees with the oracle's.
+    # The GPU's own reciprocal RMS agrees with the oracle's.
     _, _, _, r_gpu = bl.quant_act(Xd, gain=gd, rmsnorm=rmsnorm, eps=EPS, norm_eps=NORM_EPS)
     np.testing.assert_allclose(r_gpu.cpu().numpy(), r_ref, rtol=1e-6)
-    # With the oracle's rms the codes, beta and row sums are bit-exact.
+    # With the oracle's reciprocal RMS the codes, beta and row sums are bit-exact.
     xq, beta, rowsum, r_used = bl.quant_act(Xd, gain=gd, rmsnorm=rmsnorm, eps=EPS,
-                                            norm_eps=NORM_EPS, rms=to_dev(r_ref))
+                                            norm_eps=NORM_EPS, inv_rms=to_dev(r_ref))
     np.testing.assert_array_equal(xq.cpu().numpy(), q_ref)
     np.testing.assert_array_equal(beta.cpu().numpy(), b_ref)
     np.testing.assert_array_equal(rowsum.cpu().numpy(), s_ref)
@@ -157,7 +157,7 @@ def test_quant_act_special_tokens():
     X = x.to(torch.bfloat16)
     xb = bf16_bits(X)
     q_ref, b_ref, s_ref, r_ref = oracle.quant_act(xb, eps=EPS, norm_eps=NORM_EPS)
-    xq, beta, rowsum, _ = bl.quant_act(X.to(dev()), rms=to_dev(r_ref))
+    xq, beta, rowsum, _ = bl.quant_act(X.to(dev()), inv_rms=to_dev(r_ref))
     np.testing.assert_array_equal(xq.cpu().numpy(), q_ref)
     np.testing.assert_array_equal(rowsum.cpu().numpy(), s_ref)
     assert beta[0].item() == 0 and not xq[0].any()
@@ -250,6 +250,58 @@ def test_linear_equals_separate_calls_and_oracle():
         if float(w.gamma.item()) == o["gamma"]:
             acc_ref = oracle.int_matmul(o["wq"], o["xq"])
             check_y(y1, acc_ref, o["gamma"], o["beta"], False)
+
+
+FUSED_CASES = [
+    # (d_out, d_in, T, rmsnorm, gain, static, out_dtype)
+    (272, 1024, 1, True, False, False, torch.float32),
+    (272, 1024, 8, True, False, True, torch.float32),
+    (6912, 2560, 1, True, False, True, torch.bfloat16),
+    (144, 32768, 1, True, False, False, torch.float32),     # largest fused T * d_in
+    (512, 4096, 8, True, True, False, torch.float32),       # gain
+    (512, 4096, 3, False, False, True, torch.float32),      # no RMSNorm
+    (512, 4096, 9, True, False, False, torch.float32),      # T > 8: two kernels
+    (18960, 256, 1, True, False, True, torch.float32),      # 1185 row tiles: 2 per CTA, ragged
+    (18960, 256, 12, True, False, False, torch.float32),
+    (18960, 512, 5, True, True, True, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("d_out,d_in,T,rmsnorm,use_gain,static,out_dtype", FUSED_CASES)
+def test_linear_paths_match_oracle(d_out, d_in, T, rmsnorm, use_gain, static, out_dtype):
+    """bitlinear_linear (fused one-kernel path for small T*d_in, otherwise
+    quantiser + product) against the oracle; its intermediates against the
+    stand-alone quantiser; its output bit-equal to the two separate calls."""
+    W, X = draw(Problem("fz", d_in, d_out, T, 0.02, 0.01, 50.0, 17))
+    gain = None
+    if use_gain:
+        gen = torch.Generator().manual_seed(2)
+        gain = (torch.rand(d_in, generator=gen) * 2).numpy().astype(np.float32)
+    Wn = W.numpy()
+    g = oracle.absmean_gamma(Wn)
+    wq = oracle.ternarize(Wn, g, EPS)
+    xq_ref, beta_ref, rs_ref, rms_ref = oracle.quant_act(bf16_bits(X), gain=gain, rmsnorm=rmsnorm,
+                                                         eps=EPS, norm_eps=NORM_EPS)
+    w = bl.PackedTernary(to_dev(oracle.pack(wq).view(np.int32)), torch.tensor([g], device=dev()),
+                         d_out, d_in)
+    Xd = X.to(dev())
+    gd = None if gain is None else to_dev(gain)
+    scratch = (torch.empty((T, d_in), dtype=torch.int8, device=dev()),
+               torch.empty(T, dtype=torch.float32, device=dev()),
+               torch.empty(T, dtype=torch.int32, device=dev()))
+    y = bl.linear(w, Xd, gain=gd, rmsnorm=rmsnorm, out_dtype=out_dtype, scratch=scratch,
+                  static_weights=static)
+    xq2, b2, s2, r2 = bl.quant_act(Xd, gain=gd, rmsnorm=rmsnorm)
+    torch.cuda.synchronize()
+    assert torch.equal(scratch[0], xq2) and torch.equal(scratch[1], b2)
+    assert torch.equal(scratch[2], s2)
+    y2 = bl.forward(w, xq2, b2, s2, out_dtype=out_dtype)
+    assert torch.equal(y, y2)
+    np.testing.assert_allclose(r2.cpu().numpy(), rms_ref, rtol=1e-6)
+    if np.array_equal(r2.cpu().numpy(), rms_ref):
+        np.testing.assert_array_equal(xq2.cpu().numpy(), xq_ref)
+        acc_ref = oracle.int_matmul(wq, xq_ref)
+        check_y(y, acc_ref, g, beta_ref, out_dtype == torch.bfloat16)
 
 
 # ------------------------------------------- failure detection (bounded) ---
