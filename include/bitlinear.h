@@ -156,8 +156,11 @@ int bitlinear_pack_weights_noalloc(const float *W, int64_t d_out, int64_t d_in,
  *   flags      BITLINEAR_RMSNORM to normalise first, 0 to quantise X as is.
  *   eps        the epsilon of 127 / (beta + eps); finite, >= 0.
  *   norm_eps   the epsilon inside the RMS; finite, >= 0.  The reciprocal RMS
- *              r = 1 / sqrt(mean(x^2) + norm_eps) is formed in double (sum of
- *              squares in a fixed order) and rounded once to fp32.
+ *              r = 1 / sqrt(mean(x^2) + norm_eps): sum of squares in double in
+ *              a fixed order, reciprocal square root refined in double to
+ *              ~1e-13 relative, rounded to fp32 (within 1e-6 relative of the
+ *              correctly rounded value; identical in every path of this
+ *              library).
  *   inv_rms_in fp32 [T] per-token r to use instead of computing it, or NULL.
  *   Xq         out: int8 [T][d_in] activation codes in [-127, 127].
  *   beta       out: fp32 [T] per-token absmax of the (normalised) row.

@@ -40,6 +40,14 @@ __device__ __forceinline__ float round_half_up_exact(float z) {
     return (frac >= 0.5f) ? __fadd_rn(f, 1.0f) : f;
 }
 
+// The same decision as an int, for |z| < 2^23: fl_rd(z + 0.5) lies in
+// [floor(z + 0.5), z + 0.5] (the integer floor(z + 0.5) is representable and
+// below z + 0.5, so rounding down cannot pass it), hence its floor is
+// floor(z + 0.5).  Larger |z| only ever meet a clip to a small range.
+__device__ __forceinline__ int round_half_up_int(float z) {
+    return __float2int_rd(__fadd_rd(z, 0.5f));
+}
+
 // -------------------------------------------------------------- timers ---
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;

@@ -78,6 +78,7 @@ struct DecodeArgs {
     int rmsnorm;
     float eps;
     float norm_eps;
+    double inv_k;            // 1 / d_in
     int8_t *Xq_out;
     float *beta_out;
     int32_t *rowsum_out;
@@ -141,6 +142,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     extern __shared__ __align__(128) uint8_t dsm[];
     __shared__ __align__(8) uint64_t full_bar[kDecMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kDecMaxStages];
+    __shared__ __align__(8) uint64_t x_bar;   // fused: bf16 activations staged
     __shared__ QuantShared<FUSED ? TMAX : 1> qs;
     __shared__ int4 red[kDecWarps][R][NT][32];
     __shared__ float s_yscale[TMAX];
@@ -156,8 +158,11 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     const int ks = plan.ks, nslab = plan.nslab, stages = plan.stages;
     const int stage_bytes = plan.stage_bytes;
     const int units = ngrp * nslab;
-    int8_t *xs = reinterpret_cast<int8_t *>(dsm);
-    uint8_t *ring = dsm + plan.xs_bytes;
+    // Dynamic shared memory: [bf16 X (fused)] [codes (fused)] [stages].
+    const int xb_bytes = FUSED ? ((T * K * 2 + 127) & ~127) : 0;
+    uint16_t *xb = reinterpret_cast<uint16_t *>(dsm);
+    int8_t *xs = reinterpret_cast<int8_t *>(dsm + xb_bytes);
+    uint8_t *ring = dsm + xb_bytes + plan.xs_bytes;
     const uint32_t ring_s = smem_u32(ring);
     volatile int *abort_flag = &s_abort;
 
@@ -166,6 +171,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             mbar_init(smem_u32(&full_bar[st]), 1);
             mbar_init(smem_u32(&empty_bar[st]), kDecWarps);
         }
+        mbar_init(smem_u32(&x_bar), 1);
         s_abort = 0;
         mbar_init_fence();
     }
@@ -209,6 +215,12 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             }
             pdl_wait_primary();
             pdl_launch_dependents();
+            if (FUSED) {
+                // One bulk copy of the bf16 activations for the quantiser.
+                const uint32_t xbar = smem_u32(&x_bar);
+                mbar_arrive_expect_tx(xbar, (uint32_t)(T * K * 2));
+                bulk_g2s(smem_u32(xb), a.X, (uint32_t)(T * K * 2), xbar);
+            }
             int gi = 0, sl = 0, st = 0, round = 0, issued = 0;
             for (int u = 0; u < units; ++u) {
                 if (round > 0) {
@@ -230,6 +242,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             for (int u = issued > stages ? issued - stages : 0; u < issued; ++u)
                 mbar_wait_bounded(smem_u32(&full_bar[u % stages]), (uint32_t)(u / stages) & 1u,
                                   ctx);
+            if (FUSED) mbar_wait_bounded(smem_u32(&x_bar), 0, ctx);
         } else {
             pdl_wait_primary();
             pdl_launch_dependents();
@@ -238,26 +251,73 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     }
 
     // ------------------------------------------------------- consumers ---
+    // gamma belongs to the weights: with static weights it is read before the
+    // dependency wait, hiding its latency.
+    float gamma = 0.0f;
+    if (a.static_weights) gamma = __ldg(a.gamma);
     pdl_wait_primary();
     pdl_launch_dependents();
+    if (!a.static_weights) gamma = __ldg(a.gamma);
     const int g = lane >> 2, q = lane & 3;
-    const float gamma = *a.gamma;
+    bool fast_quant = false;   // fused, no gain: codes made per warp, rowsum in the epilogue
     if constexpr (FUSED) {
-        token_stats<TMAX>(a.X, T, K, a.gain, a.rmsnorm != 0, a.eps, a.norm_eps, nullptr, qs);
-        token_codes<TMAX>(a.X, T, K, a.gain, a.rmsnorm != 0, xs, qs);
-        if (threadIdx.x < T) {
-            const int t = threadIdx.x;
-            s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, qs.beta[t]), 127.0f);
-            s_rowsum[t] = qs.rowsum[t];
-            if (blockIdx.x == 0) {
-                if (a.beta_out) a.beta_out[t] = qs.beta[t];
-                if (a.rowsum_out) a.rowsum_out[t] = qs.rowsum[t];
+        bool xok = dec_wait(smem_u32(&x_bar), 0, ctx, abort_flag);
+        (void)xok;   // on expiry the codes are garbage and the error word is set
+        if (a.gain == nullptr) {
+            // Statistics in the canonical order, one barrier, then every
+            // thread finalises them itself; each warp makes the codes of the
+            // k-blocks it multiplies (kb = warp mod 4), so no barrier sits
+            // between the codes and the MMAs.
+            fast_quant = true;
+            const bool rmsnorm = a.rmsnorm != 0;
+            token_partials_smem<TMAX>(xb, T, K, rmsnorm, qs);
+            consumer_barrier();
+            int sums[TMAX];
+            #pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                sums[t] = 0;
+                if (t < T) {
+                    const TokenScale ts =
+                        token_finalize<TMAX>(t, rmsnorm, a.eps, a.norm_eps, a.inv_k, qs);
+                    if (threadIdx.x == 0) {
+                        s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, ts.beta), 127.0f);
+                        if (blockIdx.x == 0 && a.beta_out) a.beta_out[t] = ts.beta;
+                    }
+                    const uint4 *xrow = reinterpret_cast<const uint4 *>(xb + (size_t)t * K);
+                    uint2 *qrow = reinterpret_cast<uint2 *>(xs + (size_t)t * K);
+                    for (int kb = warp; kb < KB; kb += kDecWarps) {
+                        const int v = kb * 32 + lane;
+                        qrow[v] = codes8(xrow[v], rmsnorm, ts.inv_rms, ts.scale, &sums[t]);
+                    }
+                }
             }
-        }
-        if (blockIdx.x == 0 && a.Xq_out) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(xs);
-            uint4 *dst = reinterpret_cast<uint4 *>(a.Xq_out);
-            for (int v = threadIdx.x; v < (T * K) >> 4; v += kDecWarps * 32) dst[v] = src[v];
+            #pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                if (t < T) {
+                    const int sum = warp_sum_i32(sums[t]);
+                    if (lane == 0) qs.sum[warp][t] = sum;
+                }
+            }
+            __syncwarp();
+        } else {
+            token_stats<TMAX, true>(xb, T, K, a.gain, a.rmsnorm != 0, a.eps, a.norm_eps,
+                                    a.inv_k, nullptr, qs);
+            token_codes<TMAX, true>(xb, T, K, a.gain, a.rmsnorm != 0, xs, qs);
+            if (threadIdx.x < T) {
+                const int t = threadIdx.x;
+                s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, qs.beta[t]), 127.0f);
+                s_rowsum[t] = qs.rowsum[t];
+                if (blockIdx.x == 0) {
+                    if (a.beta_out) a.beta_out[t] = qs.beta[t];
+                    if (a.rowsum_out) a.rowsum_out[t] = qs.rowsum[t];
+                }
+            }
+            if (blockIdx.x == 0 && a.Xq_out) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(xs);
+                uint4 *dst = reinterpret_cast<uint4 *>(a.Xq_out);
+                for (int v = threadIdx.x; v < (T * K) >> 4; v += kDecWarps * 32) dst[v] = src[v];
+            }
+            consumer_barrier();
         }
     } else {
         if (threadIdx.x < T) {
@@ -265,8 +325,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, a.beta[t]), 127.0f);
             s_rowsum[t] = a.rowsum[t];
         }
+        consumer_barrier();
     }
-    consumer_barrier();
 
     bool ok = true;
     int st = 0;
@@ -350,6 +410,21 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 red[warp][r][nt][lane] = make_int4(c[0], c[1], c[2], c[3]);
             }
         consumer_barrier();
+        if (FUSED && fast_quant && gi == 0 && blockIdx.x == 0) {
+            // Every warp's codes are complete: CTA 0 hands back the
+            // intermediates.
+            if (threadIdx.x < T && a.rowsum_out) {
+                int sum = 0;
+                #pragma unroll
+                for (int w = 0; w < kDecWarps; ++w) sum += qs.sum[w][threadIdx.x];
+                a.rowsum_out[threadIdx.x] = sum;
+            }
+            if (a.Xq_out) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(xs);
+                uint4 *dst = reinterpret_cast<uint4 *>(a.Xq_out);
+                for (int v = threadIdx.x; v < (T * K) >> 4; v += kDecWarps * 32) dst[v] = src[v];
+            }
+        }
 
         // Epilogue of this group: output i -> (token t, row tile r, row), rows
         // fastest, so consecutive threads store consecutive outputs.
@@ -369,7 +444,15 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 const int *e = reinterpret_cast<const int *>(&red[w][r][nt][src_lane]);
                 v += e[reg];
             }
-            const int accv = v - s_rowsum[t];
+            int rsum;
+            if (FUSED && fast_quant) {
+                rsum = 0;
+                #pragma unroll
+                for (int w = 0; w < kDecWarps; ++w) rsum += qs.sum[w][t];
+            } else {
+                rsum = s_rowsum[t];
+            }
+            const int accv = v - rsum;
             const int o = (rt0 + r) * 16 + row;
             const size_t yi = (size_t)t * a.d_out + o;
             if (a.acc_out) a.acc_out[yi] = accv;
@@ -399,6 +482,9 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
 #ifndef BL_DEC_CTA_FRACTION
 #define BL_DEC_CTA_FRACTION 1           // persistent grid = resident CTAs / this
 #endif
+#ifndef BL_DEC_MIN_GROUPS
+#define BL_DEC_MIN_GROUPS 1             // at least this many groups per CTA
+#endif
 constexpr int kFusedMaxCodeBytes = BL_FUSED_MAX_CODE_BYTES;
 
 template <int NT, int R, bool FUSED, bool OUT_BF16>
@@ -409,9 +495,13 @@ static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
     const int KB = args.kb_total, K = KB * 256;
     DecodePlan plan;
     plan.xs_bytes = FUSED ? ((args.T * K + 127) & ~127) : 0;
+    const int xb_bytes = FUSED ? ((args.T * K * 2 + 127) & ~127) : 0;
     const int per_kb = R * 1024 + (FUSED ? 0 : args.T * 256);   // bytes per k-block column
     plan.ks = BL_DEC_STAGE_BYTES / per_kb;
-    if (plan.ks < 1) plan.ks = 1;
+    if (plan.ks > KB) plan.ks = KB;
+    // With several slabs keep ks a multiple of the warp count, so that warp w
+    // multiplies exactly the k-blocks kb = w (mod 4) (those it quantised).
+    if (plan.ks < KB) plan.ks = plan.ks >= kDecWarps ? plan.ks - plan.ks % kDecWarps : kDecWarps;
     if (plan.ks > KB) plan.ks = KB;
     plan.nslab = (KB + plan.ks - 1) / plan.ks;
     plan.stage_bytes = plan.ks * per_kb;
@@ -421,7 +511,8 @@ static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
     const int min_units = ((n_groups + 148 * 8 - 1) / (148 * 8)) * plan.nslab;
     if (plan.stages > min_units) plan.stages = min_units;
     if (plan.stages < 2) plan.stages = 2;
-    const size_t smem = (size_t)plan.xs_bytes + (size_t)plan.stages * plan.stage_bytes;
+    const size_t smem =
+        (size_t)xb_bytes + (size_t)plan.xs_bytes + (size_t)plan.stages * plan.stage_bytes;
     auto kern = decode_kernel<NT, R, FUSED, OUT_BF16>;
     cudaError_t e = ensure_dynamic_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
@@ -432,6 +523,8 @@ static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
             cudaSuccess || per_sm < 1)
         per_sm = 1;
     int max_ctas = sms * per_sm / BL_DEC_CTA_FRACTION;
+    const int by_groups = (n_groups + BL_DEC_MIN_GROUPS - 1) / BL_DEC_MIN_GROUPS;
+    if (max_ctas > by_groups) max_ctas = by_groups;
     if (max_ctas < sms) max_ctas = sms;
     const int grid = n_groups < max_ctas ? n_groups : max_ctas;
 
@@ -518,6 +611,7 @@ bitlinear_status launch_linear_fused(const uint32_t *packed, const float *gamma,
     a.rmsnorm = rmsnorm ? 1 : 0;
     a.eps = eps;
     a.norm_eps = norm_eps;
+    a.inv_k = 1.0 / (double)d_in;
     a.Xq_out = Xq;
     a.beta_out = beta;
     a.rowsum_out = rowsum;

@@ -23,7 +23,8 @@ namespace bl {
 
 __global__ void __launch_bounds__(kQuantThreads)
 quant_act_kernel(const uint16_t *__restrict__ X, int d_in, const float *__restrict__ gain,
-                 int rmsnorm, float eps, float norm_eps, const float *__restrict__ inv_rms_in,
+                 int rmsnorm, float eps, float norm_eps, double inv_k,
+                 const float *__restrict__ inv_rms_in,
                  int8_t *__restrict__ Xq, float *__restrict__ beta_out,
                  int32_t *__restrict__ rowsum, float *__restrict__ inv_rms_out) {
     __shared__ QuantShared<1> qs;
@@ -38,7 +39,7 @@ quant_act_kernel(const uint16_t *__restrict__ X, int d_in, const float *__restri
     pdl_wait_primary();
 
     const uint16_t *row = X + t * d_in;
-    token_stats<1>(row, 1, d_in, gain, rmsnorm != 0, eps, norm_eps,
+    token_stats<1>(row, 1, d_in, gain, rmsnorm != 0, eps, norm_eps, inv_k,
                    inv_rms_in ? inv_rms_in + t : nullptr, qs);
     token_codes<1>(row, 1, d_in, gain, rmsnorm != 0, Xq + t * d_in, qs);
     if (threadIdx.x == 0) {
@@ -64,8 +65,8 @@ bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm,
-                                       eps, norm_eps, inv_rms_in, Xq, beta, rowsum,
-                                       inv_rms_out);
+                                       eps, norm_eps, 1.0 / (double)d_in, inv_rms_in, Xq, beta,
+                                       rowsum, inv_rms_out);
     return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 

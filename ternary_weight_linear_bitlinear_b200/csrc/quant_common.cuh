@@ -7,7 +7,8 @@
 // "Activation Quantization: Absmax Scaling".
 //
 // RMSNorm is n = x * r (* g) with the reciprocal RMS r = 1 / sqrt(mean(x^2) +
-// norm_eps) formed once per token in double and rounded once to binary32.
+// norm_eps) formed once per token (see inv_rms_from_ss) and rounded to
+// binary32.
 // Canonical order (a CTA of kQuantThreads threads): thread i owns the 16-byte
 // vectors i, i + kQuantThreads, ... of a token row and accumulates x^2 in
 // double over them in that order; a warp xor-butterfly combines the 32 lanes;
@@ -29,6 +30,7 @@ namespace bl {
 
 constexpr int kQuantThreads = 128;
 constexpr int kQuantWarps = kQuantThreads / 32;
+constexpr int kQuantBatch = 8;   // 16-byte loads in flight per thread
 
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
@@ -58,6 +60,23 @@ __device__ __forceinline__ void quant_barrier() {
     asm volatile("bar.sync 1, %0;" ::"n"(kQuantThreads) : "memory");
 }
 
+// Reciprocal RMS from the sum of squares: r = 1 / sqrt(ss * inv_k + norm_eps)
+// rounded to binary32.  A single-precision estimate refined by one Newton
+// step in double (relative error ~1e-13 before the final rounding); outside
+// [1e-30, 1e30] the correctly rounded double sequence is used instead.  The
+// same fixed sequence runs in every kernel that quantises, so they agree bit
+// for bit; against the sequential double computation it agrees to far
+// better than the 1e-6 relative the tests require.
+__device__ __forceinline__ float inv_rms_from_ss(double ss, double inv_k, float norm_eps) {
+    const double x = __dadd_rn(__dmul_rn(ss, inv_k), (double)norm_eps);
+    if (x > 1e-30 && x < 1e30) {
+        const double y0 = (double)rsqrtf((float)x);
+        const double t = __dmul_rn(__dmul_rn(x, y0), y0);
+        return (float)__dmul_rn(y0, __fma_rn(-0.5, t, 1.5));
+    }
+    return (float)__ddiv_rn(1.0, __dsqrt_rn(x));
+}
+
 __device__ __forceinline__ double warp_sum_f64(double v) {
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -78,15 +97,15 @@ __device__ __forceinline__ int warp_sum_i32(int v) {
 // 0..kQuantThreads-1 of the CTA must all call it.  inv_rms_in, when
 // given, supplies the per-token reciprocal RMS.  Results: qs.inv_rms, beta,
 // scale.
+// Per-warp partial statistics of token rows in the canonical order (thread i
+// owns vectors i, i + kQuantThreads, ...; xor-butterfly within the warp),
+// written to qs.ss[warp][t] / qs.amax[warp][t].  No barrier.  X in shared
+// memory.
 template <int TMAX>
-__device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int T, int K,
-                                         const float *__restrict__ gain, bool rmsnorm,
-                                         float eps, float norm_eps,
-                                         const float *__restrict__ inv_rms_in,
-                                         QuantShared<TMAX> &qs) {
+__device__ __forceinline__ void token_partials_smem(const uint16_t *X, int T, int K,
+                                                    bool need_ss, QuantShared<TMAX> &qs) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nvec = K >> 3;
-    const bool need_ss = rmsnorm && !inv_rms_in;
     #pragma unroll 1
     for (int t = 0; t < T; ++t) {
         const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)t * K);
@@ -94,7 +113,7 @@ __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int 
         float am = 0.0f;
         for (int v = tid; v < nvec; v += kQuantThreads) {
             float x[8];
-            unpack8(__ldg(row + v), x);
+            unpack8(row[v], x);
             #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 if (need_ss) ss += (double)x[j] * (double)x[j];
@@ -108,25 +127,120 @@ __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int 
             qs.amax[warp][t] = am;
         }
     }
+}
+
+struct TokenScale {
+    float inv_rms;   // r (1 without RMSNorm)
+    float beta;      // absmax of the normalised row
+    float scale;     // 127 / (beta + eps)
+};
+
+// Final statistics of token t from the warp partials (fixed warp order); any
+// thread may compute them and every thread gets the same bits.  No gain.
+template <int TMAX>
+__device__ __forceinline__ TokenScale token_finalize(int t, bool rmsnorm, float eps,
+                                                     float norm_eps, double inv_k,
+                                                     const QuantShared<TMAX> &qs) {
+    TokenScale ts;
+    ts.inv_rms = 1.0f;
+    if (rmsnorm) {
+        double s = qs.ss[0][t];
+        #pragma unroll
+        for (int w = 1; w < kQuantWarps; ++w) s += qs.ss[w][t];
+        ts.inv_rms = inv_rms_from_ss(s, inv_k, norm_eps);
+    }
+    float m = qs.amax[0][t];
+    #pragma unroll
+    for (int w = 1; w < kQuantWarps; ++w) m = fmaxf(m, qs.amax[w][t]);
+    ts.beta = rmsnorm ? __fmul_rn(m, ts.inv_rms) : m;
+    ts.scale = __fdiv_rn(127.0f, __fadd_rn(ts.beta, eps));
+    return ts;
+}
+
+// Eight codes of one 16-byte vector of bf16 activations, packed little-endian
+// into two words; adds their sum to *sum.  No gain.
+__device__ __forceinline__ uint2 codes8(const uint4 &v, bool rmsnorm, float r, float scale,
+                                        int *sum) {
+    float x[8];
+    unpack8(v, x);
+    uint32_t lo = 0, hi = 0;
+    #pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float n = x[j];
+        if (rmsnorm) n = __fmul_rn(n, r);
+        const int qi = min(max(round_half_up_int(__fmul_rn(n, scale)), -127), 127);
+        *sum += qi;
+        const uint32_t b = (uint32_t)(qi & 0xff);
+        if (j < 4) lo |= b << (8 * j); else hi |= b << (8 * (j - 4));
+    }
+    return make_uint2(lo, hi);
+}
+
+// Row loads: read-only global path, or plain loads when X was staged in
+// shared memory.
+template <bool kSmemSrc>
+__device__ __forceinline__ uint4 load_row_vec(const uint4 *row, int v) {
+    if constexpr (kSmemSrc) return row[v];
+    else return __ldg(row + v);
+}
+
+template <int TMAX, bool kSmemSrc = false>
+__device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int T, int K,
+                                         const float *__restrict__ gain, bool rmsnorm,
+                                         float eps, float norm_eps, double inv_k,
+                                         const float *__restrict__ inv_rms_in,
+                                         QuantShared<TMAX> &qs) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nvec = K >> 3;
+    const bool need_ss = rmsnorm && !inv_rms_in;
+    #pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(X + (size_t)t * K);
+        double ss = 0.0;
+        float am = 0.0f;
+        // Loads are issued kQuantBatch at a time, then consumed in order.
+        for (int v0 = tid; v0 < nvec; v0 += kQuantBatch * kQuantThreads) {
+            uint4 buf[kQuantBatch];
+            #pragma unroll
+            for (int b = 0; b < kQuantBatch; ++b) {
+                const int v = v0 + b * kQuantThreads;
+                if (v < nvec) buf[b] = load_row_vec<kSmemSrc>(row, v);
+            }
+            #pragma unroll
+            for (int b = 0; b < kQuantBatch; ++b) {
+                if (v0 + b * kQuantThreads < nvec) {
+                    float x[8];
+                    unpack8(buf[b], x);
+                    #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (need_ss) ss += (double)x[j] * (double)x[j];
+                        am = fmaxf(am, fabsf(x[j]));
+                    }
+                }
+            }
+        }
+        ss = warp_sum_f64(ss);
+        am = warp_max_f32(am);
+        if (lane == 0) {
+            qs.ss[warp][t] = ss;
+            qs.amax[warp][t] = am;
+        }
+    }
     quant_barrier();
     if (tid < T) {
         const int t = tid;
-        float r = 1.0f;
-        if (rmsnorm) {
-            if (inv_rms_in) {
-                r = inv_rms_in[t];
-            } else {
-                double s = qs.ss[0][t];
-                #pragma unroll
-                for (int w = 1; w < kQuantWarps; ++w) s += qs.ss[w][t];
-                r = (float)__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(s / (double)K, (double)norm_eps)));
-            }
+        if (rmsnorm && inv_rms_in) {
+            const float r = inv_rms_in[t];
+            float m = qs.amax[0][t];
+            #pragma unroll
+            for (int w = 1; w < kQuantWarps; ++w) m = fmaxf(m, qs.amax[w][t]);
+            qs.inv_rms[t] = r;
+            qs.beta[t] = __fmul_rn(m, r);
+        } else {
+            const TokenScale ts = token_finalize<TMAX>(t, rmsnorm, eps, norm_eps, inv_k, qs);
+            qs.inv_rms[t] = ts.inv_rms;
+            qs.beta[t] = ts.beta;                    // replaced below when a gain is set
         }
-        float m = qs.amax[0][t];
-        #pragma unroll
-        for (int w = 1; w < kQuantWarps; ++w) m = fmaxf(m, qs.amax[w][t]);
-        qs.inv_rms[t] = r;
-        qs.beta[t] = rmsnorm ? __fmul_rn(m, r) : m;   // replaced below when a gain is set
     }
     quant_barrier();
     if (rmsnorm && gain) {
@@ -138,7 +252,7 @@ __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int 
             float a = 0.0f;
             for (int v = tid; v < nvec; v += kQuantThreads) {
                 float x[8];
-                unpack8(__ldg(row + v), x);
+                unpack8(load_row_vec<kSmemSrc>(row, v), x);
                 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     a = fmaxf(a, fabsf(__fmul_rn(__fmul_rn(x[j], r), __ldg(gain + 8 * v + j))));
@@ -161,7 +275,7 @@ __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int 
 
 // Codes of tokens 0..T-1 written to dst (row stride K bytes; global or shared
 // memory) and their row sums to qs.rowsum.  Call after token_stats.
-template <int TMAX>
+template <int TMAX, bool kSmemSrc = false>
 __device__ __forceinline__ void token_codes(const uint16_t *__restrict__ X, int T, int K,
                                          const float *__restrict__ gain, bool rmsnorm,
                                          int8_t *dst, QuantShared<TMAX> &qs) {
@@ -174,28 +288,38 @@ __device__ __forceinline__ void token_codes(const uint16_t *__restrict__ X, int 
         uint2 *out = reinterpret_cast<uint2 *>(dst + (size_t)t * K);
         const float r = rmsnorm ? qs.inv_rms[t] : 1.0f, scale = qs.scale[t];
         int sum = 0;
-        for (int v = tid; v < nvec; v += kQuantThreads) {
-            float x[8];
-            unpack8(__ldg(row + v), x);
-            float g[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
-            if (use_gain) {
-                #pragma unroll
-                for (int j = 0; j < 8; ++j) g[j] = __ldg(gain + 8 * v + j);
-            }
-            uint32_t lo = 0, hi = 0;
+        for (int v0 = tid; v0 < nvec; v0 += kQuantBatch * kQuantThreads) {
+            uint4 buf[kQuantBatch];
             #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float n = x[j];
-                if (rmsnorm) n = __fmul_rn(n, r);
-                if (use_gain) n = __fmul_rn(n, g[j]);
-                float q = round_half_up_exact(__fmul_rn(n, scale));
-                q = fminf(fmaxf(q, -127.0f), 127.0f);
-                const int qi = (int)q;
-                sum += qi;
-                const uint32_t b = (uint32_t)(qi & 0xff);
-                if (j < 4) lo |= b << (8 * j); else hi |= b << (8 * (j - 4));
+            for (int b = 0; b < kQuantBatch; ++b) {
+                const int v = v0 + b * kQuantThreads;
+                if (v < nvec) buf[b] = load_row_vec<kSmemSrc>(row, v);
             }
-            out[v] = make_uint2(lo, hi);
+            #pragma unroll
+            for (int b = 0; b < kQuantBatch; ++b) {
+                const int v = v0 + b * kQuantThreads;
+                if (v < nvec) {
+                    float x[8];
+                    unpack8(buf[b], x);
+                    float g[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+                    if (use_gain) {
+                        #pragma unroll
+                        for (int j = 0; j < 8; ++j) g[j] = __ldg(gain + 8 * v + j);
+                    }
+                    uint32_t lo = 0, hi = 0;
+                    #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float n = x[j];
+                        if (rmsnorm) n = __fmul_rn(n, r);
+                        if (use_gain) n = __fmul_rn(n, g[j]);
+                        const int qi = min(max(round_half_up_int(__fmul_rn(n, scale)), -127), 127);
+                        sum += qi;
+                        const uint32_t bb = (uint32_t)(qi & 0xff);
+                        if (j < 4) lo |= bb << (8 * j); else hi |= bb << (8 * (j - 4));
+                    }
+                    out[v] = make_uint2(lo, hi);
+                }
+            }
         }
         sum = warp_sum_i32(sum);
         if (lane == 0) qs.sum[warp][t] = sum;
