@@ -89,6 +89,10 @@ const char *bitlinear_status_string(int status);
  * or 0 when the shape breaks the rules above. */
 size_t bitlinear_packed_words(int64_t d_out, int64_t d_in);
 
+/* The same size in bytes (4 x bitlinear_packed_words: 0.25 byte per weight,
+ * [MF] section 6's 2-bit code); 0 when the shape breaks the rules above. */
+size_t bitlinear_packed_bytes(int64_t d_out, int64_t d_in);
+
 /* Bytes of device scratch bitlinear_pack_weights needs when it computes gamma
  * itself (gamma_in == NULL); 0 when the shape breaks the rules above. */
 size_t bitlinear_pack_workspace_bytes(int64_t d_out, int64_t d_in);
@@ -231,6 +235,10 @@ int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
  * clear != 0 the word is reset to zero afterwards.
  */
 int bitlinear_device_error(cudaStream_t stream, int clear);
+
+/* bitlinear_device_error(stream, 1): synchronise, report, then clear the
+ * device error word. */
+int bitlinear_get_last_device_error(cudaStream_t stream);
 
 /*
  * bitlinear_set_wait_limit_ns -- the time after which a kernel's bounded wait

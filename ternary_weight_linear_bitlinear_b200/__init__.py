@@ -43,6 +43,7 @@ SIGNATURES = {
     "bitlinear_version": (_int, []),
     "bitlinear_status_string": (ctypes.c_char_p, [_int]),
     "bitlinear_packed_words": (ctypes.c_size_t, [_i64, _i64]),
+    "bitlinear_packed_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bitlinear_pack_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bitlinear_pack_weights": (_int, [_vp, _i64, _i64, _f32, _vp, _vp, ctypes.c_size_t,
                                       _vp, _vp, _vp]),
@@ -54,6 +55,7 @@ SIGNATURES = {
     "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
                                 _vp, _vp, _vp, _vp, _int, _vp]),
     "bitlinear_device_error": (_int, [_vp, _int]),
+    "bitlinear_get_last_device_error": (_int, [_vp]),
     "bitlinear_set_wait_limit_ns": (_int, [ctypes.c_uint64]),
     "bitlinear_wait_probe": (_int, [ctypes.c_uint64, _vp]),
 }
@@ -122,6 +124,10 @@ class PackedTernary:
 
 def packed_words(d_out: int, d_in: int) -> int:
     return int(lib().bitlinear_packed_words(d_out, d_in))
+
+
+def packed_bytes(d_out: int, d_in: int) -> int:
+    return int(lib().bitlinear_packed_bytes(d_out, d_in))
 
 
 def pack_workspace_bytes(d_out: int, d_in: int) -> int:
@@ -228,6 +234,11 @@ def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm
 def device_error(clear: bool = True) -> int:
     """Synchronise the current stream and return the device error status."""
     return int(lib().bitlinear_device_error(_stream(), 1 if clear else 0))
+
+
+def get_last_device_error() -> int:
+    """Synchronise the current stream, return the device error status, clear it."""
+    return int(lib().bitlinear_get_last_device_error(_stream()))
 
 
 def set_wait_limit_ns(limit_ns: int):

@@ -215,6 +215,10 @@ extern "C" int bitlinear_device_error(cudaStream_t stream, int clear) {
     return (word & kErrTimeout) ? BITLINEAR_ERR_TIMEOUT : BITLINEAR_OK;
 }
 
+extern "C" int bitlinear_get_last_device_error(cudaStream_t stream) {
+    return bitlinear_device_error(stream, 1);
+}
+
 extern "C" int bitlinear_set_wait_limit_ns(uint64_t limit_ns) {
     if (limit_ns < 1000ull || limit_ns > 60000000000ull) return BITLINEAR_ERR_INVALID_ARG;
     int dev = 0;

@@ -107,6 +107,10 @@ extern "C" size_t bitlinear_packed_words(int64_t d_out, int64_t d_in) {
     return (size_t)(d_out * d_in / 16);
 }
 
+extern "C" size_t bitlinear_packed_bytes(int64_t d_out, int64_t d_in) {
+    return 4 * bitlinear_packed_words(d_out, d_in);
+}
+
 extern "C" size_t bitlinear_pack_workspace_bytes(int64_t d_out, int64_t d_in) {
     if (bitlinear_packed_words(d_out, d_in) == 0) return 0;
     return (size_t)kRedMaxBlocks * sizeof(double);

@@ -63,6 +63,10 @@ def test_packed_sizes(lib):
     assert bl.packed_words(15, 256) == 0          # d_out not a multiple of 16
     assert bl.packed_words(16, 128) == 0          # d_in not a multiple of 256
     assert bl.packed_words(16, 65536 + 256) == 0  # d_in too large
+    # byte count of the scope table's boundary: 0.25 byte per weight
+    assert bl.packed_bytes(6912, 2560) == 4423680
+    assert bl.packed_bytes(8192, 28672) == 58720256
+    assert bl.packed_bytes(15, 256) == 0
     assert bl.pack_workspace_bytes(6912, 2560) > 0
     assert bl.pack_workspace_bytes(16, 100) == 0
 

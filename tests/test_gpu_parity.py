@@ -311,6 +311,10 @@ def test_bounded_wait_reports_timeout():
     bl.wait_probe(2_000_000)           # 2 ms on a barrier nothing arrives on
     assert bl.device_error(clear=True) == bl.ERR_TIMEOUT
     assert bl.device_error(clear=True) == bl.OK
+    # The same report through the scope table's name, which also clears.
+    bl.wait_probe(2_000_000)
+    assert bl.get_last_device_error() == bl.ERR_TIMEOUT
+    assert bl.get_last_device_error() == bl.OK
     # The context is still usable afterwards.
     forward_case(48, 512, 3, torch.float32)
     forward_case(144, 512, 40, torch.float32)
