@@ -410,10 +410,12 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 red[warp][r][nt][lane] = make_int4(c[0], c[1], c[2], c[3]);
             }
         consumer_barrier();
-        if (FUSED && fast_quant && gi == 0 && blockIdx.x == 0) {
-            // Every warp's codes are complete: CTA 0 hands back the
-            // intermediates.
-            if (threadIdx.x < T && a.rowsum_out) {
+        if (FUSED && fast_quant && gi == 0) {
+            // Every warp's codes are complete: the CTAs hand back the
+            // intermediates.  Every CTA holds the same codes, so they are
+            // written in slices spread over the grid, and no single CTA
+            // lengthens it.
+            if (blockIdx.x == 0 && threadIdx.x < T && a.rowsum_out) {
                 int sum = 0;
                 #pragma unroll
                 for (int w = 0; w < kDecWarps; ++w) sum += qs.sum[w][threadIdx.x];
@@ -422,7 +424,10 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             if (a.Xq_out) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(xs);
                 uint4 *dst = reinterpret_cast<uint4 *>(a.Xq_out);
-                for (int v = threadIdx.x; v < (T * K) >> 4; v += kDecWarps * 32) dst[v] = src[v];
+                const int nv = (T * K) >> 4;
+                for (int v = blockIdx.x * kDecWarps * 32 + threadIdx.x; v < nv;
+                     v += gridDim.x * kDecWarps * 32)
+                    dst[v] = src[v];
             }
         }
 

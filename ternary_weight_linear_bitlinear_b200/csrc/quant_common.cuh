@@ -10,9 +10,10 @@
 // norm_eps) formed once per token (see inv_rms_from_ss) and rounded to
 // binary32.
 // Canonical order (a CTA of kQuantThreads threads): thread i owns the 16-byte
-// vectors i, i + kQuantThreads, ... of a token row and accumulates x^2 in
-// double over them in that order; a warp xor-butterfly combines the 32 lanes;
-// the kQuantWarps warp sums are added in warp order.  Without a gain vector
+// vectors i, i + kQuantThreads, ... of a token row and accumulates, in double
+// and in that order, each vector's sum of squares (sq_sum8); a warp
+// xor-butterfly combines the 32 lanes; the kQuantWarps warp sums are added in
+// warp order.  Without a gain vector
 // beta = fl(max|x| * r): correctly rounded multiplication by r > 0 is
 // monotone, so this is exactly max_k fl(|x_k| * r).  With a gain it is the
 // max of the normalised values themselves.
@@ -77,6 +78,25 @@ __device__ __forceinline__ float inv_rms_from_ss(double ss, double inv_k, float 
     return (float)__ddiv_rn(1.0, __dsqrt_rn(x));
 }
 
+// Sum of the squares of eight bf16 values, returned in double.  A bf16 value
+// has an 8-bit significand, so its square is exact in binary32 whenever it
+// neither overflows nor leaves the normal range; the eight squares are then
+// added as a fixed pairwise tree in binary32 (relative error at most 3 x
+// 2^-24).  When that sum is not finite or below 2^-100 (huge or tiny inputs)
+// the squares are formed and added sequentially in double instead.
+__device__ __forceinline__ double sq_sum8(const float (&x)[8]) {
+    float p[8];
+    #pragma unroll
+    for (int j = 0; j < 8; ++j) p[j] = __fmul_rn(x[j], x[j]);
+    const float s = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3])),
+                              __fadd_rn(__fadd_rn(p[4], p[5]), __fadd_rn(p[6], p[7])));
+    if (s >= 0x1p-100f && s <= 3.40282347e38f) return (double)s;
+    double d = 0.0;
+    #pragma unroll
+    for (int j = 0; j < 8; ++j) d = __dadd_rn(d, __dmul_rn((double)x[j], (double)x[j]));
+    return d;
+}
+
 __device__ __forceinline__ double warp_sum_f64(double v) {
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -114,11 +134,9 @@ __device__ __forceinline__ void token_partials_smem(const uint16_t *X, int T, in
         for (int v = tid; v < nvec; v += kQuantThreads) {
             float x[8];
             unpack8(row[v], x);
+            if (need_ss) ss = __dadd_rn(ss, sq_sum8(x));
             #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (need_ss) ss += (double)x[j] * (double)x[j];
-                am = fmaxf(am, fabsf(x[j]));
-            }
+            for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(x[j]));
         }
         ss = warp_sum_f64(ss);
         am = warp_max_f32(am);
@@ -211,11 +229,9 @@ __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int 
                 if (v0 + b * kQuantThreads < nvec) {
                     float x[8];
                     unpack8(buf[b], x);
+                    if (need_ss) ss = __dadd_rn(ss, sq_sum8(x));
                     #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        if (need_ss) ss += (double)x[j] * (double)x[j];
-                        am = fmaxf(am, fabsf(x[j]));
-                    }
+                    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(x[j]));
                 }
             }
         }

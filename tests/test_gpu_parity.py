@@ -264,6 +264,11 @@ FUSED_CASES = [
     (18960, 256, 1, True, False, True, torch.float32),      # 1185 row tiles: 2 per CTA, ragged
     (18960, 256, 12, True, False, False, torch.float32),
     (18960, 512, 5, True, True, True, torch.bfloat16),
+    (4096, 4096, 1, True, False, True, torch.bfloat16),     # attention projection, one token
+    (6928, 2560, 2, True, False, False, torch.float32),     # 433 row tiles
+    (8000, 4096, 4, True, True, True, torch.bfloat16),      # gain, bf16 out
+    (4752, 8192, 1, False, False, False, torch.float32),    # no RMSNorm, several slabs
+    (4096, 11008, 1, True, False, True, torch.bfloat16),    # down projection, 43 k-blocks
 ]
 
 
