@@ -20,7 +20,8 @@
  *     owned by the caller; the library allocates nothing and keeps no
  *     pointer after the call returns.
  *   - All work is enqueued on `stream` (0 = legacy default stream); no entry
- *     point synchronises except bitlinear_device_error.
+ *     point synchronises except bitlinear_device_error and
+ *     bitlinear_get_last_device_error.
  *   - Shapes: d_out (output features, N) is a positive multiple of 16,
  *     d_in (input features, K) a positive multiple of 256 and at most 65536,
  *     T (tokens) is 0 .. 1048576.  T = 0 is a no-op that returns
