@@ -416,6 +416,59 @@ def measure_prefill(steps, warmup, dev, peaks):
     }
 
 
+# ------------------------------------------------------- bf16 context ---
+
+def measure_context_bf16(dev, peaks, decode_us: dict, prefill_ms: float):
+    """The dense bf16 layer of the same shapes (bitlinear_dense_bf16_forward,
+    hand-written kernels), timed the same way: decode forwards over distinct
+    weight copies (more bytes than L2) in a CUDA graph; the prefill GEMM one
+    call at a time after an L2 flush."""
+    import ternary_weight_linear_bitlinear_b200 as bl
+    out = {"kernel": "bitlinear_dense_bf16_forward (streaming GEMV for T <= 16, "
+                     "tcgen05 kind::f16 GEMM above)"}
+    g = torch.Generator().manual_seed(0)
+    for name in ("decode_gemv_2560x6912_t1", "large_gemv_8192x28672_t1"):
+        p = WORKLOADS[name].problems[0]
+        wbytes = 2 * p.d_out * p.d_in
+        copies = max(2, int(np.ceil(2 * L2_BYTES / wbytes)))
+        Ws = [(torch.randn(p.d_out, p.d_in, generator=g) * p.sigma).to(torch.bfloat16).to(dev)
+              for _ in range(copies)]
+        X = torch.randn(p.tokens, p.d_in, generator=g).to(torch.bfloat16).to(dev)
+        Y = torch.empty((p.tokens, p.d_out), dtype=torch.bfloat16, device=dev)
+        reps = 8
+        for W in Ws:
+            bl.dense_bf16_forward(W, X, out=Y)
+        gr = capture(lambda: [bl.dense_bf16_forward(W, X, out=Y) for _ in range(reps)
+                              for W in Ws])
+        time_graph(gr)
+        us = time_graph(gr) * 1e3 / (reps * copies)
+        nbytes = wbytes + 2 * p.tokens * p.d_in + 2 * p.tokens * p.d_out
+        out[name] = {"us_per_forward": round(us, 3),
+                     "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+                     "frac_of_hbm": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm"], 4),
+                     "weight_bytes": wbytes}
+        if name in decode_us:
+            out[name]["ternary_speedup"] = round(us / decode_us[name], 2)
+        del Ws, gr
+        torch.cuda.empty_cache()
+    p = WORKLOADS["prefill_2048x4096x11008"].problems[0]
+    W = (torch.randn(p.d_out, p.d_in, generator=g) * p.sigma).to(torch.bfloat16).to(dev)
+    X = torch.randn(p.tokens, p.d_in, generator=g).to(torch.bfloat16).to(dev)
+    Y = torch.empty((p.tokens, p.d_out), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        bl.dense_bf16_forward(W, X, out=Y)
+    ms = time_each(lambda: bl.dense_bf16_forward(W, X, out=Y), 10, flush)
+    tflops = 2.0 * p.tokens * p.d_in * p.d_out / (ms * 1e-3) / 1e12
+    out["prefill_2048x4096x11008"] = {
+        "ms": round(ms, 4), "tflops": round(tflops, 1),
+        "frac_of_bf16_peak": round(tflops / peaks["bf16"], 4),
+        "ternary_speedup": round(ms / prefill_ms, 2) if prefill_ms else None}
+    del W, X, Y, flush
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------ e2e ---
 
 def measure_e2e(run, steps):
@@ -575,6 +628,14 @@ def main():
             del r2, g2
             torch.cuda.empty_cache()
         extras["decode_other"] = other
+        sampler.mark(True)
+        extras["context_bf16"] = measure_context_bf16(
+            dev, peaks,
+            {args.workload: ms_step * 1e3 / len(run.layers),
+             "large_gemv_8192x28672_t1": other["large_gemv_8192x28672_t1"]["ms_per_pass"] * 1e3
+             / other["large_gemv_8192x28672_t1"]["forwards_per_pass"]},
+            extras["prefill"]["ms_gemm"])
+        sampler.mark(False)
 
     e2e_ms, h2d, d2h = measure_e2e(run, max(3, min(args.steps, 20)))
     e2e_ms = max_over_ranks(e2e_ms, world)

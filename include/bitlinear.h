@@ -229,6 +229,25 @@ int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
                      void *Y, int out_dtype, cudaStream_t stream);
 
 /*
+ * bitlinear_dense_bf16_forward -- the dense bf16 linear layer Y = X W^T that
+ * BitLinear replaces, kept as the context the measurements compare against
+ * ([MF] section 2, "The Linear Transformation and Rescaling", without the
+ * quantisers; section 4, "Memory Bandwidth and Latency Bounds": 2 bytes per
+ * weight instead of 0.25).  Not a step of the method.
+ *
+ *   W          bf16 [d_out][d_in], row-major, 16-byte aligned.
+ *   X          bf16 [T][d_in], row-major, 16-byte aligned.
+ *   Y          out: [T][d_out] row-major, fp32 or bf16 (out_dtype), 16-byte
+ *              aligned.
+ *   Products and sums in fp32 (fused multiply-add, order unspecified), the
+ *   result rounded to nearest even for bf16.  T <= 16 runs a streaming
+ *   GEMV, larger T a tcgen05 GEMM.  Shape and error rules as above.
+ */
+int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, int64_t d_in,
+                                 const uint16_t *X, int64_t T, void *Y, int out_dtype,
+                                 cudaStream_t stream);
+
+/*
  * bitlinear_device_error -- synchronises `stream`, then reads the device
  * error word that kernels set when a bounded wait gives up.  Returns
  * BITLINEAR_OK when the word is clear, BITLINEAR_ERR_TIMEOUT when a wait

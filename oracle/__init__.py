@@ -83,6 +83,10 @@ def _load():
         lib.oracle_dot_masked_add.restype = ctypes.c_int32
         lib.oracle_rescale.argtypes = [vp, i64, i64, f32, vp, vp]
         lib.oracle_rescale.restype = None
+        lib.oracle_dense_bf16_dot.argtypes = [vp, vp, i64]
+        lib.oracle_dense_bf16_dot.restype = ctypes.c_double
+        lib.oracle_dense_bf16.argtypes = [vp, vp, i64, i64, i64, vp]
+        lib.oracle_dense_bf16.restype = None
         _lib = lib
     return _lib
 
@@ -221,6 +225,26 @@ def rescale(acc, gamma: float, beta) -> np.ndarray:
     y = np.empty((T, N), dtype=np.float64)
     _load().oracle_rescale(_ptr(acc), T, N, gamma, _ptr(beta), _ptr(y))
     return y
+
+
+# ------------------------------------------------ dense bf16 (context) ---
+
+def dense_bf16(W_bits, X_bits) -> np.ndarray:
+    """Y = X W^T of bf16 bit patterns, in double (the layer BitLinear replaces)."""
+    W = _c(W_bits, np.uint16)
+    X = _c(X_bits, np.uint16)
+    N, K = W.shape
+    T = X.shape[0]
+    y = np.empty((T, N), dtype=np.float64)
+    _load().oracle_dense_bf16(_ptr(W), _ptr(X), T, N, K, _ptr(y))
+    return y
+
+
+def dense_bf16_dot(w_bits, x_bits) -> float:
+    """One output of dense_bf16: sum_k w_k x_k in double, index order."""
+    w = _c(w_bits, np.uint16)
+    x = _c(x_bits, np.uint16)
+    return float(_load().oracle_dense_bf16_dot(_ptr(w), _ptr(x), w.size))
 
 
 def forward(W, X_bf16_bits, eps: float = 1e-5, norm_eps: float = 1e-5, gain=None,

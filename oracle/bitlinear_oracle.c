@@ -296,3 +296,26 @@ void oracle_rescale(const int32_t *acc, int64_t T, int64_t N, float gamma,
             y[t * N + o] = (double)acc[t * N + o] * scale;
     }
 }
+
+/*
+ * The dense bf16 layer that BitLinear replaces, Y = X W^T ([MF] §2, "The
+ * Linear Transformation and Rescaling", without the quantisers): the context
+ * the measurements compare against.  Each product of two bf16 values is
+ * exact in double (8 + 8 significant bits); the K products of one output are
+ * summed in double in index order.
+ */
+double oracle_dense_bf16_dot(const uint16_t *w, const uint16_t *x, int64_t K)
+{
+    double s = 0.0;
+    for (int64_t k = 0; k < K; ++k)
+        s += (double)oracle_bf16_to_f32(w[k]) * (double)oracle_bf16_to_f32(x[k]);
+    return s;
+}
+
+void oracle_dense_bf16(const uint16_t *W, const uint16_t *X, int64_t T, int64_t N, int64_t K,
+                       double *y)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t o = 0; o < N; ++o)
+            y[t * N + o] = oracle_dense_bf16_dot(W + o * K, X + t * K, K);
+}

@@ -54,6 +54,7 @@ SIGNATURES = {
                                  _vp, _vp]),
     "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
                                 _vp, _vp, _vp, _vp, _int, _vp]),
+    "bitlinear_dense_bf16_forward": (_int, [_vp, _i64, _i64, _vp, _i64, _vp, _int, _vp]),
     "bitlinear_device_error": (_int, [_vp, _int]),
     "bitlinear_get_last_device_error": (_int, [_vp]),
     "bitlinear_set_wait_limit_ns": (_int, [ctypes.c_uint64]),
@@ -228,6 +229,24 @@ def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm
                                 _ptr(gain), flags, eps, norm_eps,
                                 _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
     _check(st, "bitlinear_linear")
+    return out
+
+
+def dense_bf16_forward(W: torch.Tensor, X: torch.Tensor, out_dtype=torch.bfloat16,
+                       out: torch.Tensor = None) -> torch.Tensor:
+    """The dense bf16 layer Y = X W^T the ternary path replaces (context)."""
+    _need(W, torch.bfloat16, "W")
+    _need(X, torch.bfloat16, "X")
+    d_out, d_in = W.shape
+    T = X.shape[0]
+    if X.shape[1] != d_in:
+        raise ValueError("X must be [T][d_in]")
+    if out is None:
+        out = torch.empty((T, d_out), dtype=out_dtype, device=X.device)
+    od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
+    _check(lib().bitlinear_dense_bf16_forward(_ptr(W), d_out, d_in, _ptr(X), T, _ptr(out), od,
+                                              _stream()),
+           "bitlinear_dense_bf16_forward")
     return out
 
 

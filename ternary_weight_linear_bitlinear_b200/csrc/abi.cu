@@ -28,6 +28,9 @@ bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int6
                                 int64_t d_in, const int8_t *Xq, const float *beta,
                                 const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
                                 int32_t *acc_out, cudaStream_t stream);
+bitlinear_status launch_dense_bf16(const uint16_t *W, int64_t d_out, int64_t d_in,
+                                   const uint16_t *X, int64_t T, void *Y, int out_dtype,
+                                   cudaStream_t stream);
 
 // Device error word: set by kernels whose bounded waits expire.
 __device__ uint32_t g_error_word;
@@ -197,6 +200,22 @@ extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int6
     if (st != BITLINEAR_OK) return st;
     return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
                             nullptr, static_weights, stream);
+}
+
+extern "C" int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, int64_t d_in,
+                                            const uint16_t *X, int64_t T, void *Y,
+                                            int out_dtype, cudaStream_t stream) {
+    if (T < 0 || T > (1 << 20)) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (d_out <= 0 || d_out % 16 || d_out > (1 << 22)) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (d_in <= 0 || d_in % 256 || d_in > 65536) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (out_dtype != BITLINEAR_OUT_F32 && out_dtype != BITLINEAR_OUT_BF16)
+        return BITLINEAR_ERR_INVALID_ARG;
+    if (T == 0) return BITLINEAR_OK;
+    if (!W || !X || !Y) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(X, 16) || !aligned(Y, 16)) return BITLINEAR_ERR_MISALIGNED;
+    bitlinear_status st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    return launch_dense_bf16(W, d_out, d_in, X, T, Y, out_dtype, stream);
 }
 
 extern "C" int bitlinear_device_error(cudaStream_t stream, int clear) {

@@ -333,3 +333,34 @@ def test_forward_special_cases():
     xq, beta, _, _ = oracle.quant_act(_bits(x), rmsnorm=False)
     y = oracle.rescale(oracle.int_matmul(wq, xq), g, beta)[0]
     np.testing.assert_allclose(y, g * wq[:, 9] * -1.5, rtol=1e-6)
+
+
+# ------------------------------------------------- dense bf16 (context) ---
+
+def test_dense_bf16_brute_force():
+    """Y = X W^T of bf16 operands against pure-Python loops over exact fractions."""
+    from fractions import Fraction
+    W = _bits(RNG.standard_normal((3, 5)) * 0.5)
+    X = _bits(RNG.standard_normal((2, 5)) * 3.0)
+    Wf = oracle.bf16_bits_to_f32(W).astype(np.float64)
+    Xf = oracle.bf16_bits_to_f32(X).astype(np.float64)
+    y = oracle.dense_bf16(W, X)
+    for t in range(2):
+        for o in range(3):
+            exact = sum(Fraction(float(Wf[o, k])) * Fraction(float(Xf[t, k])) for k in range(5))
+            assert abs(Fraction(y[t, o]) - exact) <= abs(exact) * Fraction(1, 2 ** 50)
+
+
+def test_dense_bf16_against_numpy_and_identity():
+    W = _bits(RNG.standard_normal((16, 256)) * 0.02)
+    X = _bits(RNG.standard_normal((3, 256)))
+    y = oracle.dense_bf16(W, X)
+    ref = oracle.bf16_bits_to_f32(X).astype(np.float64) @ \
+        oracle.bf16_bits_to_f32(W).astype(np.float64).T
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-15)
+    # W = identity rows: Y reproduces X exactly.
+    eye = _bits(np.eye(256, dtype=np.float32)[:16])
+    np.testing.assert_array_equal(oracle.dense_bf16(eye, X),
+                                  oracle.bf16_bits_to_f32(X)[:, :16].astype(np.float64))
+    # One output through the single-dot entry point equals the full product.
+    assert oracle.dense_bf16_dot(W[5], X[2]) == y[2, 5]
