@@ -10,32 +10,33 @@
 //   D[o][t] = sum_k C[o][k] * X~[t][k]     (C = W~ + 1 in {0,1,2}, u8 x s8)
 //
 // with the weight codes as the A operand (M = 128 weight rows per tile) and
-// the tokens as B (N = 128 tokens per tile).  The kernel is persistent: one
-// CTA per SM walks the output tiles, and four roles run concurrently:
-//   * warp 0 (one lane) TMA-loads, per 256-column step, the token tile
-//     X~[n0..n0+128)[k..k+256) (two 128-byte swizzled, K-major halves) and
-//     the eight whole 16x256 packed tiles of the 128 weight rows (8 KiB,
-//     eight contiguous 1 KiB rows) into a ring of shared-memory stages,
-//     signalling `full`;
-//   * warps 2..5 (one thread per weight row = TMEM lane) expand their row's
-//     sixteen packed words into 256 int8 codes and store them straight into
-//     a tensor-memory A slot (tcgen05.st), where the MMA reads its A operand:
-//     the expanded weights never touch shared memory.  They signal `afull`;
-//   * warp 1 (one lane) issues eight tcgen05.mma.kind::i8 (K = 32 each) per
-//     step into one of two TMEM accumulators and commits to `empty`, which
-//     frees the shared-memory stage and the A slot; after a tile's last step
-//     it commits to `acc_full`;
-//   * warps 6..9 read a finished accumulator into registers (tcgen05.ld) and
-//     hand it straight back (`acc_empty`), then subtract each token's code
-//     sum, apply gamma beta / 127, stage 32x32 output blocks in shared memory
-//     and write them with TMA tensor stores -- while the MMA already fills
+// the tokens as B (N = 256 tokens per tile).  The kernel is persistent: one
+// CTA per SM walks the output tiles, and four roles run concurrently, each
+// 128-column step passing through two rings of shared memory:
+//   * warp 0 (one lane) TMA-loads the token tile X~[n0..n0+256)[k..k+128)
+//     (128-byte swizzled, K-major) and the packed 2-bit codes of the 128
+//     weight rows (4 KiB) into the token ring, signalling `full`;
+//   * warps 2..5 (one thread per weight row) expand their row's eight packed
+//     words into 128 int8 codes and store them into the weight ring in the
+//     same 128-byte swizzled K-major layout the TMA gives the tokens, then
+//     signal `afull`;
+//   * warp 1 (one lane) issues four tcgen05.mma.kind::i8 (K = 32 each) with
+//     both operands read from shared memory into one of two TMEM
+//     accumulators, and commits to `empty` (token stage free) and `aempty`
+//     (weight slot free); after a tile's last step it commits to `acc_full`;
+//   * warps 6..9 read a finished accumulator (tcgen05.ld), subtract each
+//     token's code sum, apply gamma beta / 127, stage 32-row x 8-token
+//     blocks in shared memory and write them with TMA tensor stores, then
+//     hand the accumulator back (`acc_empty`) -- while the MMA already fills
 //     the other accumulator with the next tile.
-// Tensor memory: 2 x 128 accumulator columns + 4 A slots x 64 columns = 512.
-// Waiting threads sleep in mbarrier.try_wait (with a suspend-time hint)
-// instead of spinning, leaving issue slots to the producer and MMA lanes.
-// Every mbarrier wait is bounded (see common.cuh); on expiry the CTA stops
-// issuing, waits for its own copies, MMAs and stores in flight, frees its
-// tensor memory and returns with the device error word set.
+// Each expanded weight code feeds 256 tokens of MMA work, so the expansion
+// is a small share of the issue slots.  The token ring is four deep (three
+// measured 8 % slower, five no faster); two weight slots suffice because the
+// expanders run just ahead of the MMA.  Tensor
+// memory holds only the two 256-column accumulators (512 columns).  Waiting
+// threads sleep in mbarrier.try_wait.  Every wait is bounded (see common.cuh); on expiry the
+// CTA stops issuing, waits for its own copies, MMAs and stores in flight,
+// frees its tensor memory and returns with the device error word set.
 #include <cstdint>
 
 #include <cuda.h>
@@ -48,41 +49,44 @@
 namespace bl {
 
 constexpr int kBM = 128;          // weight rows per tile (MMA M = TMEM lanes)
-constexpr int kBN = 128;          // tokens per tile (MMA N)
-constexpr int kBK = 256;          // reduction columns per stage (one packed tile)
-constexpr int kStages = 4;
-constexpr int kBHalf = kBN * 128;            // 16 KiB: one 128-byte swizzle span of tokens
-constexpr int kBTile = 2 * kBHalf;           // 32 KiB token tile
-constexpr int kPTile = kBM * kBK / 4;        // 8 KiB packed tile
-constexpr int kStageBytes = kBTile + kPTile; // 40 KiB (a multiple of 1024)
+constexpr int kBN = 256;          // tokens per tile (MMA N)
+constexpr int kBK = 128;          // reduction columns per step (bytes)
+constexpr int kStages = 4;        // token ring
+constexpr int kASlots = 2;        // weight ring
+constexpr int kBTile = kBN * kBK;            // 32 KiB token tile
+constexpr int kPTile = kBM * kBK / 4;        // 4 KiB packed tile
+constexpr int kStageBytes = kBTile + kPTile; // 36 KiB (a multiple of 1024)
+constexpr int kATile = kBM * kBK;            // 16 KiB expanded weight codes
 constexpr int kAccCols = kBN;                // int32 columns of one accumulator
 constexpr int kAccBufs = 2;
-constexpr int kACols = kBK / 4;              // TMEM columns of one A slot (4 codes each)
 constexpr int kTmemCols = 512;
 constexpr int kEpiWarps = 4;
-constexpr int kChunk = 32;                   // tokens per output block
-constexpr int kOutBufBytes = kChunk * 32 * 4;            // 32 tokens x 32 rows x fp32
+constexpr int kChunk = 8;                    // tokens per output block
+constexpr int kOutBufBytes = kChunk * 32 * 4;            // 8 tokens x 32 rows x fp32
 constexpr int kOutBytes = kEpiWarps * 2 * kOutBufBytes;  // two blocks per epilogue warp
-constexpr int kTokBytes = kEpiWarps * kBN * 8;           // per-warp {scale, code sum} table
+constexpr int kTokBytes = kBN * 8;                       // {scale, code sum} of the tile's tokens
 constexpr int kFirstEpiWarp = 6;
 constexpr int kGemmThreads = 32 * (kFirstEpiWarp + kEpiWarps);   // 10 warps
-static_assert(kAccBufs * kAccCols + kStages * kACols <= kTmemCols, "tensor memory budget");
-static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
-static_assert(kBN % kChunk == 0, "whole output blocks per tile");
+static_assert(kAccBufs * kAccCols <= kTmemCols, "tensor memory budget");
+static_assert(kStageBytes % 1024 == 0 && kATile % 1024 == 0,
+              "ring entries keep the 1024-byte swizzle alignment");
+static_assert(kBN % 32 == 0 && 32 % kChunk == 0, "whole output blocks per tile");
 
 struct __align__(8) GemmBarriers {
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t afull[kStages];
+    uint64_t afull[kASlots];
+    uint64_t aempty[kASlots];
     uint64_t acc_full[kAccBufs];
     uint64_t acc_empty[kAccBufs];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
+    int epi_ok[4];      // per epilogue warp: its wait for the accumulator succeeded
 };
 static_assert(sizeof(GemmBarriers) <= 1024, "barrier block");
-constexpr int kSmemBytes = kStages * kStageBytes + kOutBytes + kTokBytes + 1024 /* barriers */ +
-                           1024 /* alignment slack */;
+constexpr int kSmemBytes = kStages * kStageBytes + kASlots * kATile + kOutBytes + kTokBytes +
+                           1024 /* barriers */ + 1024 /* alignment slack */;
 
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -94,10 +98,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *out_stage = smem + kStages * kStageBytes;
+    uint8_t *a_ring = smem + kStages * kStageBytes;
+    uint8_t *out_stage = a_ring + kASlots * kATile;
     uint8_t *tok_stage = out_stage + kOutBytes;
     GemmBarriers *bars = reinterpret_cast<GemmBarriers *>(tok_stage + kTokBytes);
     const uint32_t smem_base = smem_u32(smem);
+    const uint32_t a_base = smem_u32(a_ring);
     auto stage_x = [&](int s) { return smem_base + s * kStageBytes; };
     auto stage_w = [&](int s) { return smem_base + s * kStageBytes + kBTile; };
 
@@ -111,7 +117,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&bars->full[s]), 1);
             mbar_init(smem_u32(&bars->empty[s]), 1);
+        }
+        for (int s = 0; s < kASlots; ++s) {
             mbar_init(smem_u32(&bars->afull[s]), 4);
+            mbar_init(smem_u32(&bars->aempty[s]), 1);
         }
         for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(smem_u32(&bars->acc_full[b]), 1);
@@ -129,7 +138,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
-    const uint32_t tmem_a = tmem_base + kAccBufs * kAccCols;
     // Everything above overlaps the previous kernel under a programmatic
     // launch; the codes, scales and gamma are read only after this point.
     pdl_wait_primary();
@@ -151,8 +159,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                     const uint32_t fb = smem_u32(&bars->full[s]);
                     mbar_arrive_expect_tx(fb, kStageBytes);
                     tma_load_2d(stage_x(s), &map_x, kt * kBK, n0, fb);
-                    tma_load_2d(stage_x(s) + kBHalf, &map_x, kt * kBK + 128, n0, fb);
-                    tma_load_3d(stage_w(s), &map_w, 0, kt, m0 / 16, fb);
+                    tma_load_4d(stage_w(s), &map_w, (kt & 1) * 8, 0, kt >> 1, m0 / 16, fb);
                     ++step;
                     if (++s == kStages) { s = 0; ph ^= 1u; }
                 }
@@ -166,8 +173,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         // ------------------------------------------------- MMA issuer ---
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_i8(kBM, kBN);
-            int s = 0, i = 0;
-            uint32_t ph = 0;
+            int s = 0, sa = 0, i = 0;
+            uint32_t pha = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++i) {
                 const int buf = i & 1, use = i >> 1;
@@ -178,22 +185,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 const uint32_t tmem_acc = tmem_base + buf * kAccCols;
                 for (int kt = 0; kt < num_k; ++kt) {
                     // `afull` completes only after every expander thread has seen
-                    // `full` (the stage's copies landed) and written its A slot,
-                    // so one wait orders both operands before the MMAs.
-                    if (!wait_or_abort(smem_u32(&bars->afull[s]), ph, ctx, abort_flag)) {
+                    // `full` (the step's copies landed) and written its codes, so
+                    // one wait orders both operands before the MMAs.
+                    if (!wait_or_abort(smem_u32(&bars->afull[sa]), pha, ctx, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     #pragma unroll
-                    for (int kk = 0; kk < kBK / 32; ++kk) {
-                        const uint64_t bdesc =
-                            smem_desc_sw128(stage_x(s) + (kk >> 2) * kBHalf + (kk & 3) * 32);
-                        tc_mma_i8_ts(tmem_acc, tmem_a + s * kACols + kk * 8, bdesc, idesc,
+                    for (int kk = 0; kk < kBK / 32; ++kk)
+                        tc_mma_i8_ss(tmem_acc, smem_desc_sw128(a_base + sa * kATile + kk * 32),
+                                     smem_desc_sw128(stage_x(s) + kk * 32), idesc,
                                      (kt > 0 || kk > 0) ? 1u : 0u);
-                    }
                     tc_commit(smem_u32(&bars->empty[s]));
-                    if (++s == kStages) { s = 0; ph ^= 1u; }
+                    tc_commit(smem_u32(&bars->aempty[sa]));
+                    if (++s == kStages) s = 0;
+                    if (++sa == kASlots) { sa = 0; pha ^= 1u; }
                 }
                 if (ok) tc_commit(smem_u32(&bars->acc_full[buf]));
             }
@@ -204,54 +211,49 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         __syncwarp();
     } else if (warp < kFirstEpiWarp) {
         // ---------------------------------------------------- expander ---
-        // Row m's sixteen words sit contiguously (64 bytes) in the stage; word
-        // kw holds columns 16 kw .. 16 kw + 15, with column 16 kw + 4 s + j in
-        // bits 8 j + 2 s, so (word >> 2 s) & 0x03030303 is the four codes of
-        // columns 16 kw + 4 s + 0..3 -- exactly TMEM column 4 kw + s of the
-        // K-major A operand (four int8 codes per 32-bit column).
-        const int quarter = warp & 3;           // TMEM lanes 32*quarter .. +31
-        const int m = quarter * 32 + lane;      // weight row within the tile
-        const uint32_t lane_field = (uint32_t)(quarter * 32) << 16;
-        int s = 0, step = 0;
-        uint32_t ph = 0;
+        // Row m's eight words of a step sit contiguously (32 bytes) in the
+        // stage; word j holds columns 16 j .. 16 j + 15 of the step, with
+        // column 16 j + 4 s + b in bits 8 b + 2 s, so (word >> 2 s) &
+        // 0x03030303 is the four codes of columns 16 j + 4 s + 0..3: word j
+        // expands to the 16-byte chunk j of the row, which the 128-byte
+        // swizzle places at chunk j ^ (m mod 8) of the row's 128 bytes.
+        const int m = (warp & 3) * 32 + lane;   // weight row within the tile
+        uint8_t *arow = a_ring + m * kBK;
+        int s = 0, sa = 0, step = 0;
+        uint32_t ph = 0, pha = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kt = 0; kt < num_k; ++kt) {
                 ok = wait_or_abort(smem_u32(&bars->full[s]), ph, ctx, abort_flag);
-                uint32_t w[16];
+                uint32_t w[8];
                 if (ok) {
                     const uint4 *src = reinterpret_cast<const uint4 *>(
-                        smem + s * kStageBytes + kBTile + m * 64);
-                    #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 v = src[q];
-                        w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-                    }
-                    // The A slot is free once the MMAs of its previous use completed.
-                    if (step >= kStages)
-                        ok = wait_or_abort(smem_u32(&bars->empty[s]), ph ^ 1u, ctx, abort_flag);
+                        smem + s * kStageBytes + kBTile + m * 32);
+                    const uint4 lo = src[0], hi = src[1];
+                    w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
+                    w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
+                    // The weight slot is free once the MMAs of its previous use completed.
+                    if (step >= kASlots)
+                        ok = wait_or_abort(smem_u32(&bars->aempty[sa]), pha ^ 1u, ctx, abort_flag);
                 }
-                // The warp stays converged: tcgen05.st is a warp-wide instruction.
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
                     break;
                 }
+                uint8_t *dst = arow + sa * kATile;
                 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t a[32];
-                    #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        #pragma unroll
-                        for (int sl = 0; sl < 4; ++sl)
-                            a[4 * j + sl] = (w[8 * h + j] >> (2 * sl)) & 0x03030303u;
-                    tmem_st_32x32b_x32(tmem_a + lane_field + s * kACols + 32 * h, a);
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 c = make_uint4(w[j] & 0x03030303u, (w[j] >> 2) & 0x03030303u,
+                                               (w[j] >> 4) & 0x03030303u, (w[j] >> 6) & 0x03030303u);
+                    *reinterpret_cast<uint4 *>(dst + ((j ^ (m & 7)) << 4)) = c;
                 }
-                tmem_wait_st();
-                tc_fence_before();
+                // The tensor cores read the codes through the async proxy.
+                fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bars->afull[s]));
+                if (lane == 0) mbar_arrive(smem_u32(&bars->afull[sa]));
                 ++step;
                 if (++s == kStages) { s = 0; ph ^= 1u; }
+                if (++sa == kASlots) { sa = 0; pha ^= 1u; }
             }
         }
     } else {
@@ -260,8 +262,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         const uint32_t lane_field = (uint32_t)(quarter * 32) << 16;
         const int ep = warp - kFirstEpiWarp;
         uint8_t *my_out = out_stage + ep * 2 * kOutBufBytes;
-        float2 *tok = reinterpret_cast<float2 *>(tok_stage + ep * kBN * 8);
+        float2 *tok = reinterpret_cast<float2 *>(tok_stage);
         const float4 *tok4 = reinterpret_cast<const float4 *>(tok);
+        // Barrier over the four epilogue warps (they share the token table).
+        auto epi_barrier = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); };
         const float gamma = *gamma_ptr;
         int ob = 0, i = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
@@ -269,75 +273,82 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             const int buf = i & 1, use = i >> 1;
             const bool ok = wait_or_abort(smem_u32(&bars->acc_full[buf]), (uint32_t)use & 1u, ctx,
                                           abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            // The four warps share a barrier, so they leave together: each
+            // posts its result, and after the barrier all read the same four.
+            const bool warp_ok = __all_sync(0xffffffffu, ok);
+            if (lane == 0) bars->epi_ok[ep] = warp_ok ? 1 : 0;
+            epi_barrier();
+            const volatile int *eok = bars->epi_ok;
+            if (!(eok[0] && eok[1] && eok[2] && eok[3])) break;
             tc_fence_after();
             const int r0 = m0 + quarter * 32;   // first output row of this warp
             const int o = r0 + lane;
-            // Output blocks of 32 tokens that exist (warp-uniform).
-            int nblk = r0 < d_out ? (T - n0 + kChunk - 1) / kChunk : 0;
-            if (nblk > kBN / kChunk) nblk = kBN / kChunk;
-            // The whole accumulator row of this lane, in four loads.
-            uint32_t v[kBN / kChunk][kChunk];
+            // Token table of this tile, {gamma beta / 127, code sum}, written by
+            // the four warps together (64 tokens each) and read back as
+            // broadcasts; the barrier above kept it until every warp was done
+            // with the previous tile's.
             #pragma unroll
-            for (int c = 0; c < kBN / kChunk; ++c)
-                if (c < nblk)
-                    tmem_ld_32x32b_x32(tmem_base + lane_field + buf * kAccCols + c * kChunk, v[c]);
-            // Token table of this tile: lane j fills tokens j, j + 32, j + 64, j + 96
-            // with {gamma beta / 127, code sum}; read back as broadcasts.
-            __syncwarp();
-            #pragma unroll
-            for (int q = 0; q < kBN / 32; ++q) {
-                const int t = n0 + q * 32 + lane;
+            for (int q = 0; q < kBN / (32 * kEpiWarps); ++q) {
+                const int tl = (q * kEpiWarps + ep) * 32 + lane;
+                const int t = n0 + tl;
                 float sc = 0.0f;
                 int rs = 0;
                 if (t < T) {
                     sc = __fdiv_rn(__fmul_rn(gamma, beta[t]), 127.0f);
                     rs = rowsum[t];
                 }
-                tok[q * 32 + lane] = make_float2(sc, __int_as_float(rs));
+                tok[tl] = make_float2(sc, __int_as_float(rs));
             }
-            tmem_wait_ld();
-            // Accumulator now in registers: the MMA may refill it.
+            epi_barrier();
+            #pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                const int tc0 = n0 + c * 32;
+                if (tc0 >= T || r0 >= d_out) break;   // uniform: nothing of this block exists
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_field + buf * kAccCols + c * 32, v);
+                tmem_wait_ld();
+                #pragma unroll
+                for (int h = 0; h < 32 / kChunk; ++h) {
+                    const int t0 = tc0 + h * kChunk;
+                    if (t0 < T) {   // uniform
+                        // The block staged two blocks ago has been read by its store.
+                        if (lane == 0) bulk_wait_read_1();
+                        __syncwarp();
+                        uint8_t *stg = my_out + ob * kOutBufBytes;
+                        #pragma unroll
+                        for (int j2 = 0; j2 < kChunk / 2; ++j2) {
+                            const float4 tp = tok4[(c * 32 + h * kChunk) / 2 + j2];
+                            #pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int j = 2 * j2 + e;
+                                const float sc = e ? tp.z : tp.x;
+                                const int rs = __float_as_int(e ? tp.w : tp.y);
+                                const int a = (int)v[h * kChunk + j] - rs;
+                                const float y = __fmul_rn((float)a, sc);
+                                if (OUT_BF16)
+                                    reinterpret_cast<__nv_bfloat16 *>(stg)[j * 32 + lane] =
+                                        __float2bfloat16_rn(y);
+                                else
+                                    reinterpret_cast<float *>(stg)[j * 32 + lane] = y;
+                                if (acc_out && o < d_out && t0 + j < T)
+                                    acc_out[(size_t)(t0 + j) * d_out + o] = a;
+                            }
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            // Rows past d_out and tokens past T are clipped by the copy.
+                            tma_store_2d(&map_y, smem_u32(stg), r0, t0);
+                            bulk_commit_group();
+                        }
+                        ob ^= 1;
+                    }
+                }
+            }
+            // Accumulator drained: the MMA may refill it.
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty[buf]));
-            #pragma unroll
-            for (int c = 0; c < kBN / kChunk; ++c) {
-                if (c < nblk) {
-                    const int t0 = n0 + c * kChunk;
-                    // The block staged two blocks ago has been read by its store.
-                    if (lane == 0) bulk_wait_read_1();
-                    __syncwarp();
-                    uint8_t *stg = my_out + ob * kOutBufBytes;
-                    #pragma unroll
-                    for (int j2 = 0; j2 < kChunk / 2; ++j2) {
-                        const float4 tp = tok4[(c * kChunk) / 2 + j2];
-                        #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int j = 2 * j2 + h;
-                            const float sc = h ? tp.z : tp.x;
-                            const int rs = __float_as_int(h ? tp.w : tp.y);
-                            const int a = (int)v[c][j] - rs;
-                            const float y = __fmul_rn((float)a, sc);
-                            if (OUT_BF16)
-                                reinterpret_cast<__nv_bfloat16 *>(stg)[j * 32 + lane] =
-                                    __float2bfloat16_rn(y);
-                            else
-                                reinterpret_cast<float *>(stg)[j * 32 + lane] = y;
-                            if (acc_out && o < d_out && t0 + j < T)
-                                acc_out[(size_t)(t0 + j) * d_out + o] = a;
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        // Rows past d_out and tokens past T are clipped by the copy.
-                        tma_store_2d(&map_y, smem_u32(stg), r0, t0);
-                        bulk_commit_group();
-                    }
-                    ob ^= 1;
-                }
-            }
         }
         if (lane == 0) bulk_wait_all();
         __syncwarp();
@@ -368,7 +379,7 @@ bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int6
     {
         const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)T};
         const cuuint64_t strides[1] = {(cuuint64_t)d_in};
-        const cuuint32_t box[2] = {128, kBN};
+        const cuuint32_t box[2] = {kBK, kBN};
         const cuuint32_t estr[2] = {1, 1};
         if (encode(&map_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(Xq), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -377,20 +388,21 @@ bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int6
             return BITLINEAR_ERR_CUDA;
     }
     {
-        // Packed words as a 3-D array [row tile][k tile][256 words of one tile].
+        // Packed words as a 4-D array [row tile][k tile][row in tile][word]; a
+        // step takes words 8 (kt & 1) .. +7 of tile kt / 2 for 8 row tiles.
         const cuuint64_t kb = (cuuint64_t)(d_in / 256);
-        const cuuint64_t dims[3] = {256, kb, (cuuint64_t)(d_out / 16)};
-        const cuuint64_t strides[2] = {1024, kb * 1024};
-        const cuuint32_t box[3] = {256, 1, kBM / 16};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        if (encode(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t *>(packed), dims,
+        const cuuint64_t dims[4] = {16, 16, kb, (cuuint64_t)(d_out / 16)};
+        const cuuint64_t strides[3] = {64, 1024, kb * 1024};
+        const cuuint32_t box[4] = {8, 16, 1, kBM / 16};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        if (encode(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint32_t *>(packed), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BITLINEAR_ERR_CUDA;
     }
     {
-        // Output [T][d_out], written in 32-row x 32-token boxes.
+        // Output [T][d_out], written in 32-row x 16-token boxes.
         const cuuint64_t esize = bf ? 2 : 4;
         const cuuint64_t dims[2] = {(cuuint64_t)d_out, (cuuint64_t)T};
         const cuuint64_t strides[1] = {(cuuint64_t)d_out * esize};
