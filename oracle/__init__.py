@@ -74,7 +74,7 @@ def _load():
         lib.oracle_unpack_row.restype = i32
         lib.oracle_inv_rms.argtypes = [vp, i64, f32]
         lib.oracle_inv_rms.restype = f32
-        lib.oracle_quant_act.argtypes = [vp, i64, i64, vp, i32, f32, f32, vp,
+        lib.oracle_quant_act.argtypes = [vp, i64, i64, vp, i32, i32, f32, f32, vp,
                                          vp, vp, vp, vp]
         lib.oracle_quant_act.restype = None
         lib.oracle_int_matmul.argtypes = [vp, vp, i64, i64, i64, vp]
@@ -178,10 +178,12 @@ def inv_rms(x_bf16_bits, norm_eps: float = 1e-5) -> float:
 
 
 def quant_act(X_bf16_bits, gain=None, rmsnorm: bool = True, eps: float = 1e-5,
-              norm_eps: float = 1e-5, inv_rms_in=None):
-    """Per-token absmax int8 quantisation, optional RMSNorm first ([MF] §2).
+              norm_eps: float = 1e-5, inv_rms_in=None, per_tensor: bool = False):
+    """Absmax int8 quantisation, per token (or per tensor), optional RMSNorm
+    first ([MF] §2).
 
-    Returns (xq int8 [T][K], beta f32 [T], rowsum int32 [T], inv_rms f32 [T]).
+    Returns (xq int8 [T][K], beta f32 [T], rowsum int32 [T], inv_rms f32 [T]);
+    with per_tensor every beta[t] is the one absmax of the whole X.
     """
     X = _c(X_bf16_bits, np.uint16)
     T, K = X.shape
@@ -191,9 +193,9 @@ def quant_act(X_bf16_bits, gain=None, rmsnorm: bool = True, eps: float = 1e-5,
     beta = np.empty(T, dtype=np.float32)
     rowsum = np.empty(T, dtype=np.int32)
     rms_out = np.empty(T, dtype=np.float32)
-    _load().oracle_quant_act(_ptr(X), T, K, _ptr(g), int(bool(rmsnorm)), eps,
-                             norm_eps, _ptr(r_in), _ptr(xq), _ptr(beta),
-                             _ptr(rowsum), _ptr(rms_out))
+    _load().oracle_quant_act(_ptr(X), T, K, _ptr(g), int(bool(rmsnorm)),
+                             int(bool(per_tensor)), eps, norm_eps, _ptr(r_in), _ptr(xq),
+                             _ptr(beta), _ptr(rowsum), _ptr(rms_out))
     return xq, beta, rowsum, rms_out
 
 

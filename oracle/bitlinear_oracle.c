@@ -200,52 +200,69 @@ float oracle_inv_rms(const uint16_t *x, int64_t K, float norm_eps)
     return (float)(1.0 / sqrt(ss / (double)K + (double)norm_eps));
 }
 
+/* The normalised value of one element: x * r (times g), or x unchanged. */
+static float normalised(const uint16_t *x, int64_t k, int rmsnorm, float r, const float *gain)
+{
+    float n = oracle_bf16_to_f32(x[k]);
+    if (rmsnorm) {
+        n = n * r;
+        if (gain) n = n * gain[k];
+    }
+    return n;
+}
+
 /*
- * Per-token absmax int8 quantisation with optional RMSNorm in front.
+ * Absmax int8 quantisation with optional RMSNorm in front.
  *   n_k   = x_k * r (binary32 multiplication) with r the token's reciprocal
  *           RMS, times g_k if a gain is given (binary32 multiplication);
  *           n_k = x_k when rmsnorm == 0
- *   beta  = max_k |n_k|
+ *   beta  = max |n| over the token (per_tensor == 0), or over every element
+ *           of every token (per_tensor != 0: [MF] section 2 prints the max
+ *           over all i, j and allows either scope)
  *   q_k   = RoundClip(n_k * 127 / (beta + eps), -127, 127) with the scale
  *           127 / (beta + eps) formed first (binary32 add, then divide) and
  *           applied with one binary32 multiplication
- *   S     = sum_k q_k (the correction term of the offset-code product)
+ *   S     = sum_k q_k per token (the correction term of the offset-code
+ *           product)
  * inv_rms_in, when not NULL, supplies the per-token reciprocal RMS instead of
  * computing it (used to compare integer codes against a GPU that computed
- * its own).
+ * its own).  beta[t] receives the beta token t was quantised with.
  */
 void oracle_quant_act(const uint16_t *X, int64_t T, int64_t K, const float *gain,
-                      int rmsnorm, float eps, float norm_eps, const float *inv_rms_in,
-                      int8_t *xq, float *beta, int32_t *rowsum, float *inv_rms_out)
+                      int rmsnorm, int per_tensor, float eps, float norm_eps,
+                      const float *inv_rms_in, int8_t *xq, float *beta, int32_t *rowsum,
+                      float *inv_rms_out)
 {
+    /* Statistics of every token first. */
     for (int64_t t = 0; t < T; ++t) {
         const uint16_t *x = X + t * K;
         float r = 1.0f;
         if (rmsnorm)
             r = inv_rms_in ? inv_rms_in[t] : oracle_inv_rms(x, K, norm_eps);
         if (inv_rms_out) inv_rms_out[t] = r;
-
         float b = 0.0f;
         for (int64_t k = 0; k < K; ++k) {
-            float n = oracle_bf16_to_f32(x[k]);
-            if (rmsnorm) {
-                n = n * r;
-                if (gain) n = n * gain[k];
-            }
-            float a = fabsf(n);
+            float a = fabsf(normalised(x, k, rmsnorm, r, gain));
             if (a > b) b = a;
         }
         beta[t] = b;
-
-        float scale = (float)ORACLE_QB_MINUS_1 / (b + eps);
+    }
+    if (per_tensor) {
+        float m = 0.0f;
+        for (int64_t t = 0; t < T; ++t)
+            if (beta[t] > m) m = beta[t];
+        for (int64_t t = 0; t < T; ++t) beta[t] = m;
+    }
+    /* Then the codes. */
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *x = X + t * K;
+        float r = 1.0f;
+        if (rmsnorm)
+            r = inv_rms_in ? inv_rms_in[t] : oracle_inv_rms(x, K, norm_eps);
+        float scale = (float)ORACLE_QB_MINUS_1 / (beta[t] + eps);
         int32_t S = 0;
         for (int64_t k = 0; k < K; ++k) {
-            float n = oracle_bf16_to_f32(x[k]);
-            if (rmsnorm) {
-                n = n * r;
-                if (gain) n = n * gain[k];
-            }
-            float v = n * scale;
+            float v = normalised(x, k, rmsnorm, r, gain) * scale;
             int q = (int)round_clip_f32(v, -(float)ORACLE_QB_MINUS_1,
                                         (float)ORACLE_QB_MINUS_1);
             xq[t * K + k] = (int8_t)q;

@@ -364,3 +364,55 @@ def test_dense_bf16_against_numpy_and_identity():
                                   oracle.bf16_bits_to_f32(X)[:, :16].astype(np.float64))
     # One output through the single-dot entry point equals the full product.
     assert oracle.dense_bf16_dot(W[5], X[2]) == y[2, 5]
+
+
+# ------------------------------------------------- per-tensor absmax (NEXT) ---
+
+def test_per_tensor_worked_example():
+    """Hand-derived: X = [[1, -2], [4, 0.5]], no RMSNorm, beta = 4 for both
+    tokens, scale = 127 / (4 + 1e-5) = 31.7499...; 1 -> floor(32.25) = 32,
+    -2 -> floor(-63.0) = -63, 4 -> 127, 0.5 -> floor(16.37) = 16."""
+    X = _bits([[1.0, -2.0], [4.0, 0.5]])
+    xq, beta, rs, _ = oracle.quant_act(X, rmsnorm=False, per_tensor=True)
+    np.testing.assert_array_equal(xq, [[32, -63], [127, 16]])
+    np.testing.assert_array_equal(beta, [4.0, 4.0])
+    np.testing.assert_array_equal(rs, [-31, 143])
+    # Per token the first row would use its own beta = 2 instead.
+    xq1, beta1, _, _ = oracle.quant_act(X, rmsnorm=False, per_tensor=False)
+    np.testing.assert_array_equal(beta1, [2.0, 4.0])
+    assert xq1[0, 1] == -127
+
+
+@pytest.mark.parametrize("rmsnorm", [False, True])
+def test_per_tensor_properties(rmsnorm):
+    W, X = draw(Problem("pt", 512, 16, 6, 0.02, 0.01, 50.0, 9))
+    xb = bf16_bits(X)
+    xq_t, beta_t, _, r_t = oracle.quant_act(xb, rmsnorm=rmsnorm)
+    xq, beta, rs, r = oracle.quant_act(xb, rmsnorm=rmsnorm, per_tensor=True)
+    np.testing.assert_array_equal(r, r_t)                 # the normalisation is per token
+    assert np.all(beta == beta_t.max())                   # one beta: the largest per-token one
+    np.testing.assert_array_equal(rs, xq.astype(np.int64).sum(axis=1))
+    top = int(np.argmax(beta_t))
+    np.testing.assert_array_equal(xq[top], xq_t[top])     # that token is unchanged
+    assert np.abs(xq[top]).max() == 127
+    # Every other token's largest code is its own absmax on the shared scale.
+    scale = np.float32(127.0) / (np.float32(beta[0]) + np.float32(1e-5))
+    for t in range(6):
+        expect = np.floor(np.float64(np.float32(beta_t[t] * scale)) + 0.5)
+        assert np.abs(xq[t]).max() == min(expect, 127)
+    # One token: the two scopes coincide.
+    a = oracle.quant_act(xb[:1], rmsnorm=rmsnorm, per_tensor=True)
+    b = oracle.quant_act(xb[:1], rmsnorm=rmsnorm, per_tensor=False)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+
+
+def test_per_tensor_scale_invariance():
+    """Without RMSNorm and with eps = 0, scaling all of X by 2^m (exact in
+    bf16) leaves the per-tensor codes unchanged."""
+    _, X = draw(Problem("ps", 256, 16, 4, 0.02, 0.02, 30.0, 4))
+    base = oracle.quant_act(bf16_bits(X), rmsnorm=False, eps=0.0, per_tensor=True)[0]
+    for m in (-3, 5):
+        Xs = (X.float() * (2.0 ** m)).to(torch.bfloat16)
+        np.testing.assert_array_equal(
+            oracle.quant_act(bf16_bits(Xs), rmsnorm=False, eps=0.0, per_tensor=True)[0], base)
