@@ -79,6 +79,13 @@ typedef enum {
  * reading them before earlier work completes (decode layers with fixed
  * weights: the next layer's weight stream overlaps the current layer). */
 #define BITLINEAR_STATIC_WEIGHTS 2u
+/* bitlinear_quant_act and bitlinear_linear: one beta for the whole X -- the
+ * largest absmax over all tokens ([MF] section 2 prints beta as the max over
+ * all i, j and allows this scope) -- instead of one per token.  beta[t] then
+ * holds that one value for every t.  Three launches (statistics, max,
+ * codes); bitlinear_linear never fuses the quantiser into the product in
+ * this mode. */
+#define BITLINEAR_PER_TENSOR_ABSMAX 4u
 
 /* Library ABI version (this header: 1). */
 int bitlinear_version(void);

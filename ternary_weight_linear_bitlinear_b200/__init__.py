@@ -27,6 +27,7 @@ OUT_F32 = 0
 OUT_BF16 = 1
 RMSNORM = 1
 STATIC_WEIGHTS = 2
+PER_TENSOR_ABSMAX = 4
 
 OK = 0
 ERR_INVALID_ARG = 1
@@ -160,8 +161,10 @@ def pack_weights(W: torch.Tensor, eps: float = 1e-5, gamma: torch.Tensor = None,
 
 
 def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
-              eps: float = 1e-5, norm_eps: float = 1e-5, inv_rms: torch.Tensor = None):
-    """Fused RMSNorm + per-token absmax int8 codes of bf16 X [T][d_in].
+              eps: float = 1e-5, norm_eps: float = 1e-5, inv_rms: torch.Tensor = None,
+              per_tensor: bool = False):
+    """Fused RMSNorm + absmax int8 codes of bf16 X [T][d_in], with one beta
+    per token (default) or one for the whole tensor (per_tensor).
 
     Returns (Xq int8 [T][d_in], beta f32 [T], rowsum int32 [T], inv_rms f32 [T]),
     inv_rms being the per-token reciprocal RMS used (or given).
@@ -177,7 +180,8 @@ def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
         _need(gain, torch.float32, "gain")
     if inv_rms is not None:
         _need(inv_rms, torch.float32, "inv_rms")
-    st = lib().bitlinear_quant_act(_ptr(X), T, d_in, _ptr(gain), RMSNORM if rmsnorm else 0,
+    flags = (RMSNORM if rmsnorm else 0) | (PER_TENSOR_ABSMAX if per_tensor else 0)
+    st = lib().bitlinear_quant_act(_ptr(X), T, d_in, _ptr(gain), flags,
                                    eps, norm_eps, _ptr(inv_rms), _ptr(Xq), _ptr(beta),
                                    _ptr(rowsum), _ptr(rms_out), _stream())
     _check(st, "bitlinear_quant_act")
@@ -203,12 +207,14 @@ def forward(w: PackedTernary, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torc
 
 def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
            eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.float32,
-           out: torch.Tensor = None, scratch=None, static_weights: bool = False):
+           out: torch.Tensor = None, scratch=None, static_weights: bool = False,
+           per_tensor: bool = False):
     """The whole BitLinear forward from bf16 X: quantise, then product.
 
     static_weights: promise that no work still in flight on the stream
     writes w.packed or w.gamma (the product may then stream the weights
-    before earlier work has finished).  ``scratch`` = (Xq, beta, rowsum)
+    before earlier work has finished).  per_tensor: one activation absmax for
+    the whole X instead of one per token.  ``scratch`` = (Xq, beta, rowsum)
     receives the intermediates.
     """
     _need(X, torch.bfloat16, "X")
@@ -224,7 +230,8 @@ def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm
     od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
     if gain is not None:
         _need(gain, torch.float32, "gain")
-    flags = (RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
+    flags = ((RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
+             | (PER_TENSOR_ABSMAX if per_tensor else 0))
     st = lib().bitlinear_linear(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(X), T,
                                 _ptr(gain), flags, eps, norm_eps,
                                 _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())

@@ -177,7 +177,8 @@ extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int6
                                 cudaStream_t stream) {
     bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, nullptr);
     if (st != BITLINEAR_OK) return st;
-    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_STATIC_WEIGHTS)) return BITLINEAR_ERR_INVALID_ARG;
+    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_STATIC_WEIGHTS | BITLINEAR_PER_TENSOR_ABSMAX))
+        return BITLINEAR_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !std::isfinite(eps) || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps))
         return BITLINEAR_ERR_INVALID_ARG;
     if (T == 0) return BITLINEAR_OK;
@@ -189,14 +190,16 @@ extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int6
     if (st != BITLINEAR_OK) return st;
     const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
     const bool rmsnorm = (flags & BITLINEAR_RMSNORM) != 0;
-    if (decode_can_fuse(T, d_in))
+    const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
+    if (!per_tensor && decode_can_fuse(T, d_in))
         return launch_linear_fused(packed, gamma, d_out, d_in, X, T, norm_gain, rmsnorm, eps,
                                    norm_eps, Xq, beta, rowsum, Y, out_dtype, static_weights,
                                    stream);
     // Quantiser, then the product as its programmatic dependent: with static
     // weights the product streams them while the codes are still being made.
-    st = launch_quant_act(X, T, d_in, norm_gain, flags & BITLINEAR_RMSNORM, eps, norm_eps,
-                          nullptr, Xq, beta, rowsum, nullptr, true, stream);
+    st = launch_quant_act(X, T, d_in, norm_gain,
+                          flags & (BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX), eps,
+                          norm_eps, nullptr, Xq, beta, rowsum, nullptr, true, stream);
     if (st != BITLINEAR_OK) return st;
     return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
                             nullptr, static_weights, stream);

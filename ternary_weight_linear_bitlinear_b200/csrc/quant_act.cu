@@ -1,4 +1,5 @@
-// quant_act.cu -- fused RMSNorm + per-token absmax int8 activation codes.
+// quant_act.cu -- fused RMSNorm + absmax int8 activation codes (per token, or
+// per tensor).
 //
 // "BitNet b1.58: Mathematical Foundations of 1.58-Bit Ternary Quantization,
 // Absmean Scaling, and Multiplication-Free LLM Architectures", section 2,
@@ -8,10 +9,17 @@
 //
 // One CTA of kQuantThreads per token: one pass for the sum of squares and the
 // absmax (one more when a gain vector is set), one pass for the codes; the
-// row is re-read from L1.  RMSNorm multiplies by the token's reciprocal RMS.  Besides the codes the kernel writes the row sum of
-// the codes, which the product kernels use to turn their offset-code sums
-// into W~ X~.  The reduction order is the one of quant_common.cuh, shared
-// with the fused decode kernel.
+// row is re-read from L1.  RMSNorm multiplies by the token's reciprocal RMS.
+// Besides the codes the kernel writes the row sum of the codes, which the
+// product kernels use to turn their offset-code sums into W~ X~.  The
+// reduction order is the one of quant_common.cuh, shared with the fused
+// decode kernel.
+//
+// Per-tensor scope (the same section prints beta as the max over all i, j):
+// three launches -- every token's statistics (beta[t] = its own absmax), one
+// CTA folding them into beta[0] = max_t beta[t], then every token's codes on
+// that one beta (recomputing its reciprocal RMS in the same order), each
+// token's beta[t] set to it.
 #include <cmath>
 #include <cstdint>
 
@@ -21,12 +29,18 @@
 
 namespace bl {
 
+enum QuantMode : int {
+    kQuantPerToken = 0,     // statistics and codes of each token
+    kQuantStatsOnly = 1,    // statistics only: beta[t] = the token's absmax
+    kQuantSharedBeta = 2,   // codes on the one beta held in beta[0]
+};
+
 __global__ void __launch_bounds__(kQuantThreads)
 quant_act_kernel(const uint16_t *__restrict__ X, int d_in, const float *__restrict__ gain,
                  int rmsnorm, float eps, float norm_eps, double inv_k,
                  const float *__restrict__ inv_rms_in,
                  int8_t *__restrict__ Xq, float *__restrict__ beta_out,
-                 int32_t *__restrict__ rowsum, float *__restrict__ inv_rms_out) {
+                 int32_t *__restrict__ rowsum, float *__restrict__ inv_rms_out, int mode) {
     __shared__ QuantShared<1> qs;
     const int64_t t = blockIdx.x;
 
@@ -41,11 +55,44 @@ quant_act_kernel(const uint16_t *__restrict__ X, int d_in, const float *__restri
     const uint16_t *row = X + t * d_in;
     token_stats<1>(row, 1, d_in, gain, rmsnorm != 0, eps, norm_eps, inv_k,
                    inv_rms_in ? inv_rms_in + t : nullptr, qs);
+    if (mode == kQuantStatsOnly) {
+        if (threadIdx.x == 0) {
+            beta_out[t] = qs.beta[0];
+            if (inv_rms_out) inv_rms_out[t] = qs.inv_rms[0];
+        }
+        return;
+    }
+    if (mode == kQuantSharedBeta) {
+        // Every CTA reads the same beta[0] and token 0 rewrites it with the
+        // same value.
+        if (threadIdx.x == 0) {
+            const float b = beta_out[0];
+            qs.beta[0] = b;
+            qs.scale[0] = __fdiv_rn(127.0f, __fadd_rn(b, eps));
+        }
+        quant_barrier();
+    }
     token_codes<1>(row, 1, d_in, gain, rmsnorm != 0, Xq + t * d_in, qs);
     if (threadIdx.x == 0) {
         beta_out[t] = qs.beta[0];
         rowsum[t] = qs.rowsum[0];
         if (inv_rms_out) inv_rms_out[t] = qs.inv_rms[0];
+    }
+}
+
+// beta[0] = max_t beta[t] (non-negative values), one CTA.
+constexpr int kBetaMaxThreads = 1024;
+__global__ void __launch_bounds__(kBetaMaxThreads) beta_max_kernel(float *beta, int64_t T) {
+    __shared__ float part[kBetaMaxThreads / 32];
+    float m = 0.0f;
+    for (int64_t i = threadIdx.x; i < T; i += kBetaMaxThreads) m = fmaxf(m, beta[i]);
+    m = warp_max_f32(m);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        m = part[threadIdx.x];
+        m = warp_max_f32(m);
+        if (threadIdx.x == 0) beta[0] = m;
     }
 }
 
@@ -55,6 +102,7 @@ bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                                   float *beta, int32_t *rowsum, float *inv_rms_out, bool pdl,
                                   cudaStream_t stream) {
     const int rmsnorm = (flags & BITLINEAR_RMSNORM) ? 1 : 0;
+    const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)T);
     cfg.blockDim = dim3(kQuantThreads);
@@ -64,9 +112,24 @@ bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm,
-                                       eps, norm_eps, 1.0 / (double)d_in, inv_rms_in, Xq, beta,
-                                       rowsum, inv_rms_out);
+    const double inv_k = 1.0 / (double)d_in;
+    cudaError_t e;
+    if (!per_tensor) {
+        e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
+                               norm_eps, inv_k, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
+                               (int)kQuantPerToken);
+        return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+    }
+    e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
+                           norm_eps, inv_k, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
+                           (int)kQuantStatsOnly);
+    if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
+    beta_max_kernel<<<1, kBetaMaxThreads, 0, stream>>>(beta, T);
+    if (cudaGetLastError() != cudaSuccess) return BITLINEAR_ERR_CUDA;
+    cfg.numAttrs = 0;   // the codes need the folded beta: an ordinary stream-ordered launch
+    e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
+                           norm_eps, inv_k, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
+                           (int)kQuantSharedBeta);
     return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
@@ -81,7 +144,8 @@ extern "C" int bitlinear_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                                    cudaStream_t stream) {
     if (T < 0 || T > (1 << 20)) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     if (d_in <= 0 || d_in % 256 || d_in > 65536) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-    if (flags & ~BITLINEAR_RMSNORM) return BITLINEAR_ERR_INVALID_ARG;
+    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX))
+        return BITLINEAR_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !std::isfinite(eps)) return BITLINEAR_ERR_INVALID_ARG;
     if (!(norm_eps >= 0.0f) || !std::isfinite(norm_eps)) return BITLINEAR_ERR_INVALID_ARG;
     if (T == 0) return BITLINEAR_OK;

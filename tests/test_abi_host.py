@@ -108,7 +108,9 @@ def test_quant_act_validation(lib):
                  P(a["beta"]), P(a["rs"]), P(a["rmso"]) if a["rmso"] else None, S0)
 
     assert call(X=0) == bl.ERR_INVALID_ARG
-    assert call(flags=4) == bl.ERR_INVALID_ARG
+    assert call(flags=8) == bl.ERR_INVALID_ARG                     # no such flag
+    assert call(flags=2) == bl.ERR_INVALID_ARG                     # bitlinear_linear's only
+    assert call(flags=1 | bl.PER_TENSOR_ABSMAX) != bl.ERR_INVALID_ARG
     assert call(eps=float("nan")) == bl.ERR_INVALID_ARG
     assert call(neps=-1.0) == bl.ERR_INVALID_ARG
     assert call(d_in=300) == bl.ERR_UNSUPPORTED_SHAPE

@@ -164,6 +164,61 @@ def test_quant_act_special_tokens():
     assert (xq[1] == -127).all()
 
 
+PER_TENSOR_CASES = [
+    # (T, K, rmsnorm, gain)
+    (1, 512, True, False), (5, 512, True, True), (40, 1024, False, False),
+    (300, 4096, True, False), (1100, 256, True, False),
+]
+
+
+@pytest.mark.parametrize("T,K,rmsnorm,use_gain", PER_TENSOR_CASES)
+def test_quant_act_per_tensor_matches_oracle(T, K, rmsnorm, use_gain):
+    """One beta for all tokens: statistics, the max over tokens and the codes."""
+    X = draw(Problem("pt", K, 16, T, 0.02, 0.01, 50.0, 21))[1]
+    gain = None
+    if use_gain:
+        gen = torch.Generator().manual_seed(4)
+        gain = (torch.rand(K, generator=gen) * 2).numpy().astype(np.float32)
+    xb = bf16_bits(X)
+    q_ref, b_ref, s_ref, r_ref = oracle.quant_act(xb, gain=gain, rmsnorm=rmsnorm, eps=EPS,
+                                                  norm_eps=NORM_EPS, per_tensor=True)
+    assert np.all(b_ref == b_ref[0])
+    Xd = X.to(dev())
+    gd = None if gain is None else to_dev(gain)
+    _, _, _, r_gpu = bl.quant_act(Xd, gain=gd, rmsnorm=rmsnorm, per_tensor=True)
+    np.testing.assert_allclose(r_gpu.cpu().numpy(), r_ref, rtol=1e-6)
+    xq, beta, rowsum, _ = bl.quant_act(Xd, gain=gd, rmsnorm=rmsnorm, eps=EPS, norm_eps=NORM_EPS,
+                                       inv_rms=to_dev(r_ref), per_tensor=True)
+    np.testing.assert_array_equal(beta.cpu().numpy(), b_ref)
+    np.testing.assert_array_equal(xq.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("T", [1, 3, 40])
+def test_linear_per_tensor_matches_oracle(T):
+    """bitlinear_linear with the per-tensor scope (decode and prefill paths)."""
+    d_out, d_in = 272, 1024
+    W, X = draw(Problem("lpt", d_in, d_out, T, 0.02, 0.01, 50.0, 23))
+    Wn = W.numpy()
+    g = oracle.absmean_gamma(Wn)
+    wq = oracle.ternarize(Wn, g, EPS)
+    xq_ref, b_ref, s_ref, r_ref = oracle.quant_act(bf16_bits(X), eps=EPS, norm_eps=NORM_EPS,
+                                                   per_tensor=True)
+    w = bl.PackedTernary(to_dev(oracle.pack(wq).view(np.int32)), torch.tensor([g], device=dev()),
+                         d_out, d_in)
+    scratch = (torch.empty((T, d_in), dtype=torch.int8, device=dev()),
+               torch.empty(T, dtype=torch.float32, device=dev()),
+               torch.empty(T, dtype=torch.int32, device=dev()))
+    y = bl.linear(w, X.to(dev()), scratch=scratch, per_tensor=True)
+    torch.cuda.synchronize()
+    b_gpu = scratch[1].cpu().numpy()
+    assert np.all(b_gpu == b_gpu[0])
+    np.testing.assert_allclose(b_gpu, b_ref, rtol=2e-6)
+    if np.array_equal(b_gpu, b_ref):
+        np.testing.assert_array_equal(scratch[0].cpu().numpy(), xq_ref)
+        check_y(y, oracle.int_matmul(wq, xq_ref), g, b_ref, False)
+
+
 # ---------------------------------------------------------------- forward ---
 
 def forward_case(d_out, d_in, T, out_dtype, seed=5, frac=0.01, factor=50.0):
