@@ -263,6 +263,19 @@ def test_gemm_bf16_out(T):
     forward_case(256, 1024, T, torch.bfloat16)
 
 
+# Many tiles per CTA (the persistent tile loop and both accumulators in turn).
+LARGE_GEMM_CASES = [
+    (4096, 512, 1201, torch.float32),    # ragged tokens in the last tile
+    (4112, 256, 1100, torch.bfloat16),   # 4112 rows: the last row tile holds 16
+    (9472, 256, 512, torch.float32),
+]
+
+
+@pytest.mark.parametrize("d_out,d_in,T,out_dtype", LARGE_GEMM_CASES)
+def test_gemm_many_tiles_matches_oracle(d_out, d_in, T, out_dtype):
+    forward_case(d_out, d_in, T, out_dtype)
+
+
 def test_forward_zero_inputs():
     for T in (1, 40):
         d_out, d_in = 64, 512
