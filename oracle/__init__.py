@@ -83,6 +83,10 @@ def _load():
         lib.oracle_dot_masked_add.restype = ctypes.c_int32
         lib.oracle_rescale.argtypes = [vp, i64, i64, f32, vp, vp]
         lib.oracle_rescale.restype = None
+        lib.oracle_dequant_act_bf16.argtypes = [ctypes.c_int8, f32]
+        lib.oracle_dequant_act_bf16.restype = ctypes.c_uint16
+        lib.oracle_backward.argtypes = [vp, f32, vp, vp, vp, i64, i64, i64, vp, vp]
+        lib.oracle_backward.restype = None
         lib.oracle_dense_bf16_dot.argtypes = [vp, vp, i64]
         lib.oracle_dense_bf16_dot.restype = ctypes.c_double
         lib.oracle_dense_bf16.argtypes = [vp, vp, i64, i64, i64, vp]
@@ -247,6 +251,29 @@ def dense_bf16_dot(w_bits, x_bits) -> float:
     w = _c(w_bits, np.uint16)
     x = _c(x_bits, np.uint16)
     return float(_load().oracle_dense_bf16_dot(_ptr(w), _ptr(x), w.size))
+
+
+# ------------------------------------------------ backward (STE, [MF] §3) ---
+
+def dequant_act_bf16(q: int, beta: float) -> int:
+    """X^ of one code: bf16 bits of fl32(q * fl32(beta / 127))."""
+    return int(_load().oracle_dequant_act_bf16(int(q), float(beta)))
+
+
+def backward(wq, gamma: float, xq, beta, dY_bits, want_dx: bool = True, want_dw: bool = True):
+    """Straight-through-estimator gradients ([MF] §3): returns (dX [T][K],
+    dW [N][K]) in double, either None when not asked for."""
+    wq = _c(wq, np.int8)
+    xq = _c(xq, np.int8)
+    beta = _c(beta, np.float32)
+    dY = _c(dY_bits, np.uint16)
+    N, K = wq.shape
+    T = xq.shape[0]
+    dX = np.empty((T, K), dtype=np.float64) if want_dx else None
+    dW = np.empty((N, K), dtype=np.float64) if want_dw else None
+    _load().oracle_backward(_ptr(wq), gamma, _ptr(xq), _ptr(beta), _ptr(dY), T, N, K,
+                            _ptr(dX), _ptr(dW))
+    return dX, dW
 
 
 def forward(W, X_bf16_bits, eps: float = 1e-5, norm_eps: float = 1e-5, gain=None,

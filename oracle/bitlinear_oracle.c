@@ -336,3 +336,50 @@ void oracle_dense_bf16(const uint16_t *W, const uint16_t *X, int64_t T, int64_t 
         for (int64_t o = 0; o < N; ++o)
             y[t * N + o] = oracle_dense_bf16_dot(W + o * K, X + t * K, K);
 }
+
+/*
+ * Backward pass with the straight-through estimator ([MF] section 3,
+ * "Training Dynamics and the Straight-Through Estimator"): the rounding of
+ * both quantisers is bypassed, so the layer acts as Y = X^ (gamma W~)^T with
+ * the dequantised activations X^ = X~ * beta / 127, gamma and beta held
+ * constant.  Given dY [T][N] (bf16):
+ *   dX[t][k] = gamma * sum_o dY[t][o] W~[o][k]        (gradient at X^)
+ *   dW[o][k] = gamma * sum_t dY[t][o] X^[t][k]        (gradient at W~, passed
+ *                                                      to the latent weights)
+ * X^ is formed as the GEMM operand is: bf16 of the binary32 product
+ * X~ * (beta / 127) (binary32 divide, binary32 multiply, round to nearest
+ * even).  Sums in double; each product of a bf16 value and a small integer or
+ * of two bf16 values is exact in double.
+ */
+uint16_t oracle_dequant_act_bf16(int8_t q, float beta)
+{
+    float s = beta / (float)ORACLE_QB_MINUS_1;
+    return oracle_f32_to_bf16((float)q * s);
+}
+
+void oracle_backward(const int8_t *wq, float gamma, const int8_t *xq, const float *beta,
+                     const uint16_t *dY, int64_t T, int64_t N, int64_t K, double *dX,
+                     double *dW)
+{
+    if (dX) {
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t k = 0; k < K; ++k) {
+                double s = 0.0;
+                for (int64_t o = 0; o < N; ++o)
+                    s += (double)oracle_bf16_to_f32(dY[t * N + o]) * (double)wq[o * K + k];
+                dX[t * K + k] = (double)gamma * s;
+            }
+    }
+    if (dW) {
+        for (int64_t o = 0; o < N; ++o)
+            for (int64_t k = 0; k < K; ++k) {
+                double s = 0.0;
+                for (int64_t t = 0; t < T; ++t) {
+                    double xh = (double)oracle_bf16_to_f32(
+                        oracle_dequant_act_bf16(xq[t * K + k], beta[t]));
+                    s += (double)oracle_bf16_to_f32(dY[t * N + o]) * xh;
+                }
+                dW[o * K + k] = (double)gamma * s;
+            }
+    }
+}

@@ -416,3 +416,76 @@ def test_per_tensor_scale_invariance():
         Xs = (X.float() * (2.0 ** m)).to(torch.bfloat16)
         np.testing.assert_array_equal(
             oracle.quant_act(bf16_bits(Xs), rmsnorm=False, eps=0.0, per_tensor=True)[0], base)
+
+
+# --------------------------------------------- backward, STE (NEXT-2) ---
+
+def _tiny_backward_case(T=3, N=32, K=256, seed=6):
+    W, X = draw(Problem("bw", K, N, T, 0.02, 0.01, 50.0, seed))
+    Wn = W.numpy()
+    g = oracle.absmean_gamma(Wn)
+    wq = oracle.ternarize(Wn, g, 1e-5)
+    xq, beta, _, _ = oracle.quant_act(bf16_bits(X))
+    dY = bf16_bits(torch.randn(T, N, generator=torch.Generator().manual_seed(seed + 1))
+                   .to(torch.bfloat16))
+    return wq, g, xq, beta, dY
+
+
+def test_dequant_operand_matches_torch_rounding():
+    """X^ = bf16(fl32(q * fl32(beta / 127))) against torch's own bf16 rounding."""
+    for beta in (0.37, 3.1415, 127.0, 1e-3):
+        s = np.float32(beta) / np.float32(127.0)
+        for q in (-127, -64, -1, 0, 1, 5, 99, 127):
+            ref = torch.tensor(np.float32(q) * s, dtype=torch.float32).to(torch.bfloat16)
+            assert oracle.dequant_act_bf16(q, beta) == int(ref.view(torch.int16).item()) & 0xFFFF
+
+
+def test_backward_is_the_gradient_of_the_forward():
+    """The inference forward (int_matmul + rescale) is linear in the codes, so
+    raising one activation code by 1 changes L = sum(dY * Y) by
+    dX[t][k] * beta_t / 127, and raising one weight code by 1 changes it by
+    dW[o][k] up to the bf16 rounding of X^ (2^-8 relative per term)."""
+    wq, g, xq, beta, dY = _tiny_backward_case()
+    dX, dW = oracle.backward(wq, g, xq, beta, dY)
+    dYf = oracle.bf16_bits_to_f32(dY).astype(np.float64)
+
+    def loss(w, x):
+        return float((dYf * oracle.rescale(oracle.int_matmul(w, x), g, beta)).sum())
+
+    base = loss(wq, xq)
+    rng = np.random.default_rng(0)
+    for _ in range(8):
+        t, k = int(rng.integers(0, xq.shape[0])), int(rng.integers(0, xq.shape[1]))
+        x2 = xq.copy()
+        x2[t, k] += 1 if x2[t, k] < 127 else -1
+        step = float(int(x2[t, k]) - int(xq[t, k])) * float(beta[t]) / 127.0
+        assert abs((loss(wq, x2) - base) - dX[t, k] * step) <= 1e-9 * (abs(base) + 1)
+    mag = np.abs(dYf).T @ np.abs(xq.astype(np.float64) * beta[:, None] / 127.0) * g
+    for _ in range(8):
+        o, k = int(rng.integers(0, wq.shape[0])), int(rng.integers(0, wq.shape[1]))
+        w2 = wq.copy()
+        w2[o, k] += 1 if w2[o, k] < 1 else -1
+        step = float(int(w2[o, k]) - int(wq[o, k]))
+        assert abs((loss(w2, xq) - base) - dW[o, k] * step) <= 2.0 ** -8 * mag[o, k] + 1e-12
+
+
+def test_backward_exact_fractions_and_special_cases():
+    from fractions import Fraction
+    wq, g, xq, beta, dY = _tiny_backward_case(T=2, N=16, K=256, seed=9)
+    dX, dW = oracle.backward(wq, g, xq, beta, dY)
+    dYf = oracle.bf16_bits_to_f32(dY)
+    for t, k in ((0, 3), (1, 200)):
+        exact = sum(Fraction(float(dYf[t, o])) * int(wq[o, k]) for o in range(16)) * Fraction(g)
+        assert abs(Fraction(dX[t, k]) - exact) <= abs(exact) * Fraction(1, 2 ** 50)
+    # One-hot dY: dX is gamma times one weight row; dW is gamma times one X^ row.
+    oh = np.zeros_like(dY)
+    oh[1, 5] = 0x3F80                                   # bf16 1.0
+    dX1, dW1 = oracle.backward(wq, g, xq, beta, oh)
+    np.testing.assert_array_equal(dX1[0], 0.0)
+    np.testing.assert_array_equal(dX1[1], g * wq[5].astype(np.float64))
+    xh = np.array([oracle.bf16_bits_to_f32(np.array([oracle.dequant_act_bf16(q, beta[1])],
+                                                     dtype=np.uint16))[0] for q in xq[1]])
+    np.testing.assert_array_equal(dW1[5], g * xh.astype(np.float64))
+    assert not dW1[np.arange(16) != 5].any()
+    z0, z1 = oracle.backward(wq, g, xq, beta, np.zeros_like(dY))
+    assert not z0.any() and not z1.any()
