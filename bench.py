@@ -419,6 +419,64 @@ def measure_prefill(steps, warmup, dev, peaks):
     }
 
 
+# ------------------------------------------------------------ backward ---
+
+def measure_backward(steps, dev, peaks):
+    """The straight-through-estimator backward at the prefill shape (dX and
+    dW: two tcgen05 bf16 GEMMs plus the operand transposes), one call at a
+    time after an L2 flush; beside it the dense bf16 layer's two gradient
+    GEMMs with operands already transposed (its weights kept in bf16)."""
+    import ternary_weight_linear_bitlinear_b200 as bl
+    p = WORKLOADS["prefill_2048x4096x11008"].problems[0]
+    T, N, K = p.tokens, p.d_out, p.d_in
+    W, X = draw(p)
+    w = bl.pack_weights(W.to(dev), EPS)
+    del W
+    xq, beta, _, _ = bl.quant_act(X.to(dev))
+    g = torch.Generator().manual_seed(3)
+    dY = torch.randn(T, N, generator=g).to(torch.bfloat16).to(dev)
+    nbytes = int(bl.lib().bitlinear_backward_workspace_bytes(N, K, T, 1, 1))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dX = torch.empty((T, K), dtype=torch.float32, device=dev)
+    dW = torch.empty((N, K), dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def ours():
+        bl._check(bl.lib().bitlinear_backward(
+            bl._ptr(w.packed), bl._ptr(w.gamma), N, K, bl._ptr(xq), bl._ptr(beta), T,
+            bl._ptr(dY), bl._ptr(dX), bl._ptr(dW), bl.OUT_F32, bl._ptr(ws), nbytes,
+            bl._stream()), "bitlinear_backward")
+
+    for _ in range(3):
+        ours()
+    ms = time_each(ours, steps, flush)
+    flops = 4.0 * T * N * K
+    # The dense bf16 layer's gradient GEMMs on pre-transposed operands.
+    Wt = torch.randn(K, N, generator=g).to(torch.bfloat16).to(dev)
+    Xt = torch.randn(K, T, generator=g).to(torch.bfloat16).to(dev)
+    dYt = dY.t().contiguous()
+
+    def dense():
+        bl.dense_bf16_forward(Wt, dY, out_dtype=torch.float32, out=dX)
+        bl.dense_bf16_forward(Xt, dYt, out_dtype=torch.float32, out=dW)
+
+    for _ in range(3):
+        dense()
+    ms_dense = time_each(dense, steps, flush)
+    del ws, flush, Wt, Xt, dYt
+    torch.cuda.empty_cache()
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"workload": "prefill_2048x4096x11008 backward (dX, dW)",
+            "ms": round(ms, 4), "tflops": round(tflops, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1),
+                         "peak": peaks["bf16"], "unit": "TFLOP/s",
+                         "frac": round(tflops / peaks["bf16"], 4),
+                         "peak_source": peaks["source"] + " bf16 burst"},
+            "dense_bf16_gemms_ms": round(ms_dense, 4),
+            "overhead_vs_dense": round(ms / ms_dense, 3),
+            "gpu_launches": 5 * steps}
+
+
 # ------------------------------------------------------- bf16 context ---
 
 def measure_context_bf16(dev, peaks, decode_us: dict, prefill_ms: float):
@@ -632,6 +690,7 @@ def main():
             torch.cuda.empty_cache()
         extras["decode_other"] = other
         sampler.mark(True)
+        extras["backward_ste"] = measure_backward(10, dev, peaks)
         extras["context_bf16"] = measure_context_bf16(
             dev, peaks,
             {args.workload: ms_step * 1e3 / len(run.layers),

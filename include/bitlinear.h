@@ -255,6 +255,37 @@ int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, int64_t d_in,
                                  cudaStream_t stream);
 
 /*
+ * bitlinear_backward -- gradients of the BitLinear forward with the
+ * straight-through estimator ([MF] section 3, "Training Dynamics and the
+ * Straight-Through Estimator": the rounding is bypassed, so the layer acts
+ * as Y = X^ (gamma W~)^T with X^ = X~ beta / 127, gamma and beta constant):
+ *
+ *   dX = gamma dY W~       [T][d_in]     gradient at X^ (the quantiser input)
+ *   dW = gamma dY^T X^     [d_out][d_in] gradient at W~, passed to the latent
+ *                                        weights
+ *
+ *   packed, gamma   the weights as bitlinear_pack_weights left them.
+ *   Xq, beta        the forward's activation codes [T][d_in] and scales [T];
+ *                   needed for dW only.
+ *   dY              bf16 [T][d_out], row-major, 16-byte aligned.
+ *   dX, dW          out: fp32 or bf16 (out_dtype), row-major, 16-byte aligned;
+ *                   either may be NULL (not computed), not both.
+ *   workspace       device scratch of bitlinear_backward_workspace_bytes()
+ *                   bytes, 256-byte aligned, owned by the caller (the
+ *                   transposed operands: W~^T, X^^T and dY^T in bf16).
+ * X^ enters the dW product as bf16 of fl32(q * fl32(beta / 127)); products
+ * and sums in fp32, gamma applied once to the fp32 sum.  Shapes: d_out a
+ * multiple of 256 and at most 65536, d_in as above, 0 <= T <= 65536 (T = 0
+ * zeroes dW).  Errors as above; a short workspace is BITLINEAR_ERR_INVALID_ARG.
+ */
+size_t bitlinear_backward_workspace_bytes(int64_t d_out, int64_t d_in, int64_t T,
+                                          int want_dx, int want_dw);
+int bitlinear_backward(const uint32_t *packed, const float *gamma, int64_t d_out,
+                       int64_t d_in, const int8_t *Xq, const float *beta, int64_t T,
+                       const uint16_t *dY, void *dX, void *dW, int out_dtype,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * bitlinear_device_error -- synchronises `stream`, then reads the device
  * error word that kernels set when a bounded wait gives up.  Returns
  * BITLINEAR_OK when the word is clear, BITLINEAR_ERR_TIMEOUT when a wait

@@ -264,11 +264,18 @@ def backward(wq, gamma: float, xq, beta, dY_bits, want_dx: bool = True, want_dw:
     """Straight-through-estimator gradients ([MF] §3): returns (dX [T][K],
     dW [N][K]) in double, either None when not asked for."""
     wq = _c(wq, np.int8)
-    xq = _c(xq, np.int8)
-    beta = _c(beta, np.float32)
     dY = _c(dY_bits, np.uint16)
     N, K = wq.shape
-    T = xq.shape[0]
+    T = dY.shape[0]
+    if dY.ndim != 2 or dY.shape[1] != N:
+        raise ValueError("dY must be [T][N] with N = wq.shape[0]")
+    if want_dw:
+        xq = _c(xq, np.int8)
+        beta = _c(beta, np.float32)
+        if xq.shape != (T, K) or beta.shape != (T,):
+            raise ValueError("xq must be [T][K] and beta [T], T = dY.shape[0]")
+    else:
+        xq = beta = None
     dX = np.empty((T, K), dtype=np.float64) if want_dx else None
     dW = np.empty((N, K), dtype=np.float64) if want_dw else None
     _load().oracle_backward(_ptr(wq), gamma, _ptr(xq), _ptr(beta), _ptr(dY), T, N, K,

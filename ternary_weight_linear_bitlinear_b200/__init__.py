@@ -56,6 +56,9 @@ SIGNATURES = {
     "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
                                 _vp, _vp, _vp, _vp, _int, _vp]),
     "bitlinear_dense_bf16_forward": (_int, [_vp, _i64, _i64, _vp, _i64, _vp, _int, _vp]),
+    "bitlinear_backward_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _int, _int]),
+    "bitlinear_backward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _int, _vp,
+                                  ctypes.c_size_t, _vp]),
     "bitlinear_device_error": (_int, [_vp, _int]),
     "bitlinear_get_last_device_error": (_int, [_vp]),
     "bitlinear_set_wait_limit_ns": (_int, [ctypes.c_uint64]),
@@ -237,6 +240,32 @@ def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm
                                 _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
     _check(st, "bitlinear_linear")
     return out
+
+
+def backward(w: PackedTernary, Xq: torch.Tensor, beta: torch.Tensor, dY: torch.Tensor,
+             want_dx: bool = True, want_dw: bool = True, out_dtype=torch.float32,
+             workspace: torch.Tensor = None):
+    """Straight-through-estimator gradients of the forward ([MF] §3):
+    returns (dX [T][d_in], dW [d_out][d_in]), None for the one not asked for."""
+    _need(dY, torch.bfloat16, "dY")
+    T = dY.shape[0]
+    dev = dY.device
+    if want_dw:
+        _need(Xq, torch.int8, "Xq")
+        _need(beta, torch.float32, "beta")
+    nbytes = int(lib().bitlinear_backward_workspace_bytes(w.d_out, w.d_in, T, int(want_dx),
+                                                          int(want_dw)))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    dX = torch.empty((T, w.d_in), dtype=out_dtype, device=dev) if want_dx else None
+    dW = torch.empty((w.d_out, w.d_in), dtype=out_dtype, device=dev) if want_dw else None
+    od = OUT_BF16 if out_dtype == torch.bfloat16 else OUT_F32
+    _check(lib().bitlinear_backward(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in,
+                                    _ptr(Xq) if want_dw else None,
+                                    _ptr(beta) if want_dw else None, T, _ptr(dY), _ptr(dX),
+                                    _ptr(dW), od, _ptr(workspace), workspace.numel(), _stream()),
+           "bitlinear_backward")
+    return dX, dW
 
 
 def dense_bf16_forward(W: torch.Tensor, X: torch.Tensor, out_dtype=torch.bfloat16,

@@ -30,7 +30,7 @@ bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int6
                                 int32_t *acc_out, cudaStream_t stream);
 bitlinear_status launch_dense_bf16(const uint16_t *W, int64_t d_out, int64_t d_in,
                                    const uint16_t *X, int64_t T, void *Y, int out_dtype,
-                                   cudaStream_t stream);
+                                   const float *alpha, cudaStream_t stream);
 
 // Device error word: set by kernels whose bounded waits expire.
 __device__ uint32_t g_error_word;
@@ -218,7 +218,7 @@ extern "C" int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, in
     if (!aligned(W, 16) || !aligned(X, 16) || !aligned(Y, 16)) return BITLINEAR_ERR_MISALIGNED;
     bitlinear_status st = check_device();
     if (st != BITLINEAR_OK) return st;
-    return launch_dense_bf16(W, d_out, d_in, X, T, Y, out_dtype, stream);
+    return launch_dense_bf16(W, d_out, d_in, X, T, Y, out_dtype, nullptr, stream);
 }
 
 extern "C" int bitlinear_device_error(cudaStream_t stream, int clear) {

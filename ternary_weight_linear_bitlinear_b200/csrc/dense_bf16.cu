@@ -56,7 +56,7 @@ __device__ __forceinline__ float dot8_bf16(const uint4 &w, const uint4 &x, float
 template <int TT, bool OUT_BF16>
 __global__ void __launch_bounds__(kDgThreads)
 dense_gemv_kernel(const uint4 *__restrict__ W, const uint4 *__restrict__ X, int d_out, int kv,
-                  int T, void *__restrict__ Y) {
+                  int T, void *__restrict__ Y, const float *__restrict__ alpha) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row0 = (blockIdx.x * (kDgThreads / 32) + warp) * kDgRows;
     if (row0 >= d_out) return;   // whole warp
@@ -91,16 +91,18 @@ dense_gemv_kernel(const uint4 *__restrict__ W, const uint4 *__restrict__ X, int 
             acc[r][t] = v;
         }
     if (lane == 0) {
+        const float a = alpha ? *alpha : 1.0f;
         #pragma unroll
         for (int r = 0; r < kDgRows; ++r)
             #pragma unroll
             for (int t = 0; t < TT; ++t) {
                 if (t < T && row0 + r < d_out) {
                     const size_t yi = (size_t)t * d_out + row0 + r;
+                    const float y = alpha ? __fmul_rn(acc[r][t], a) : acc[r][t];
                     if (OUT_BF16)
-                        reinterpret_cast<__nv_bfloat16 *>(Y)[yi] = __float2bfloat16_rn(acc[r][t]);
+                        reinterpret_cast<__nv_bfloat16 *>(Y)[yi] = __float2bfloat16_rn(y);
                     else
-                        reinterpret_cast<float *>(Y)[yi] = acc[r][t];
+                        reinterpret_cast<float *>(Y)[yi] = y;
                 }
             }
     }
@@ -142,7 +144,7 @@ template <bool OUT_BF16>
 __global__ void __launch_bounds__(kDThreads, 1)
 dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
                   const __grid_constant__ CUtensorMap map_y, int d_out, int d_in, int T,
-                  DeviceCtx ctx) {
+                  const float *__restrict__ alpha, DeviceCtx ctx) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -246,6 +248,7 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
         const int quarter = warp & 3;
         const uint32_t lane_field = (uint32_t)(quarter * 32) << 16;
         uint8_t *my_out = out_stage + (warp - kDFirstEpiWarp) * 2 * kDOutBufBytes;
+        const float a = alpha ? *alpha : 1.0f;
         int ob = 0, i = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
             const int m0 = (tile % m_tiles) * kDM, n0 = (tile / m_tiles) * kDN;
@@ -267,7 +270,8 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
                 uint8_t *stg = my_out + ob * kDOutBufBytes;
                 #pragma unroll
                 for (int j = 0; j < kDChunk; ++j) {
-                    const float y = __uint_as_float(v[j]);
+                    const float y = alpha ? __fmul_rn(__uint_as_float(v[j]), a)
+                                          : __uint_as_float(v[j]);
                     if (OUT_BF16)
                         reinterpret_cast<__nv_bfloat16 *>(stg)[j * 32 + lane] = __float2bfloat16_rn(y);
                     else
@@ -302,19 +306,19 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
 template <int TT>
 static cudaError_t launch_dense_gemv_t(const uint16_t *W, int64_t d_out, int64_t d_in,
                                        const uint16_t *X, int64_t T, void *Y, bool bf,
-                                       cudaStream_t stream) {
+                                       const float *alpha, cudaStream_t stream) {
     const int rows_per_cta = (kDgThreads / 32) * kDgRows;
     const unsigned grid = (unsigned)((d_out + rows_per_cta - 1) / rows_per_cta);
     auto kern = bf ? dense_gemv_kernel<TT, true> : dense_gemv_kernel<TT, false>;
     kern<<<grid, kDgThreads, 0, stream>>>(reinterpret_cast<const uint4 *>(W),
                                           reinterpret_cast<const uint4 *>(X), (int)d_out,
-                                          (int)(d_in / 8), (int)T, Y);
+                                          (int)(d_in / 8), (int)T, Y, alpha);
     return cudaGetLastError();
 }
 
 static bitlinear_status launch_dense_gemm(const uint16_t *W, int64_t d_out, int64_t d_in,
                                           const uint16_t *X, int64_t T, void *Y, bool bf,
-                                          cudaStream_t stream) {
+                                          const float *alpha, cudaStream_t stream) {
     PFN_encodeTiled encode = get_encode_fn();
     if (!encode) return BITLINEAR_ERR_CUDA;
     DeviceCtx ctx;
@@ -362,21 +366,22 @@ static bitlinear_status launch_dense_gemm(const uint16_t *W, int64_t d_out, int6
     const int64_t tiles = ((d_out + kDM - 1) / kDM) * ((T + kDN - 1) / kDN);
     const int grid = (int)(tiles < sms ? tiles : sms);
     kern<<<grid, kDThreads, kDSmemBytes, stream>>>(map_w, map_x, map_y, (int)d_out, (int)d_in,
-                                                   (int)T, ctx);
+                                                   (int)T, alpha, ctx);
     return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
+// alpha: optional device scalar multiplying every output (in fp32, once).
 bitlinear_status launch_dense_bf16(const uint16_t *W, int64_t d_out, int64_t d_in,
                                    const uint16_t *X, int64_t T, void *Y, int out_dtype,
-                                   cudaStream_t stream) {
+                                   const float *alpha, cudaStream_t stream) {
     const bool bf = out_dtype == BITLINEAR_OUT_BF16;
-    if (T > 16) return launch_dense_gemm(W, d_out, d_in, X, T, Y, bf, stream);
+    if (T > 16) return launch_dense_gemm(W, d_out, d_in, X, T, Y, bf, alpha, stream);
     cudaError_t e;
-    if (T <= 1) e = launch_dense_gemv_t<1>(W, d_out, d_in, X, T, Y, bf, stream);
-    else if (T <= 2) e = launch_dense_gemv_t<2>(W, d_out, d_in, X, T, Y, bf, stream);
-    else if (T <= 4) e = launch_dense_gemv_t<4>(W, d_out, d_in, X, T, Y, bf, stream);
-    else if (T <= 8) e = launch_dense_gemv_t<8>(W, d_out, d_in, X, T, Y, bf, stream);
-    else e = launch_dense_gemv_t<16>(W, d_out, d_in, X, T, Y, bf, stream);
+    if (T <= 1) e = launch_dense_gemv_t<1>(W, d_out, d_in, X, T, Y, bf, alpha, stream);
+    else if (T <= 2) e = launch_dense_gemv_t<2>(W, d_out, d_in, X, T, Y, bf, alpha, stream);
+    else if (T <= 4) e = launch_dense_gemv_t<4>(W, d_out, d_in, X, T, Y, bf, alpha, stream);
+    else if (T <= 8) e = launch_dense_gemv_t<8>(W, d_out, d_in, X, T, Y, bf, alpha, stream);
+    else e = launch_dense_gemv_t<16>(W, d_out, d_in, X, T, Y, bf, alpha, stream);
     return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 

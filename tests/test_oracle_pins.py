@@ -489,3 +489,13 @@ def test_backward_exact_fractions_and_special_cases():
     assert not dW1[np.arange(16) != 5].any()
     z0, z1 = oracle.backward(wq, g, xq, beta, np.zeros_like(dY))
     assert not z0.any() and not z1.any()
+
+
+def test_backward_rejects_mismatched_shapes():
+    wq, g, xq, beta, dY = _tiny_backward_case(T=3, N=16, K=256, seed=2)
+    with pytest.raises(ValueError):
+        oracle.backward(wq, g, xq[:2], beta[:2], dY)          # tokens disagree
+    with pytest.raises(ValueError):
+        oracle.backward(wq[:8], g, xq, beta, dY)              # outputs disagree
+    dX, dW = oracle.backward(wq, g, None, None, dY, want_dw=False)
+    assert dW is None and dX.shape == (3, 256)
