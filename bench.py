@@ -534,20 +534,37 @@ def measure_context_bf16(dev, peaks, decode_us: dict, prefill_ms: float):
 
 def measure_e2e(run, steps):
     """Through the public API with host buffers: every step copies its
-    activations host -> device from pinned memory and reads each output
-    back device -> host, inside the timed region."""
+    activations (all layers' X, one pinned host buffer) host -> device and
+    reads all its outputs back device -> host, inside the timed region; the
+    forwards are eager bitlinear_linear calls through the binding's
+    LinearPlan (arguments bound once per layer)."""
     bl = run.bl
-    host_x = [X.cpu().pin_memory() for _, _, X, _, _ in run.layers]
-    host_y = [torch.empty(Y.shape, dtype=Y.dtype).pin_memory() for *_, Y in run.layers]
-    h2d = sum(x.numel() * x.element_size() for x in host_x)
-    d2h = sum(y.numel() * y.element_size() for y in host_y)
+    dev = run.dev
+    xs = [X for _, _, X, _, _ in run.layers]
+    ys = [Y for *_, Y in run.layers]
+    x_elems = [x.numel() for x in xs]
+    y_elems = [y.numel() for y in ys]
+    host_x = torch.cat([x.reshape(-1) for x in xs]).cpu().pin_memory()
+    host_y = torch.empty(sum(y_elems), dtype=ys[0].dtype).pin_memory()
+    dev_x = torch.empty_like(host_x, device=dev)
+    dev_y = torch.empty(sum(y_elems), dtype=ys[0].dtype, device=dev)
+    x_views, y_views, ox, oy = [], [], 0, 0
+    for x, y, nx, ny in zip(xs, ys, x_elems, y_elems):
+        x_views.append(dev_x[ox:ox + nx].view(x.shape))
+        y_views.append(dev_y[oy:oy + ny].view(y.shape))
+        ox += nx
+        oy += ny
+    h2d = host_x.numel() * host_x.element_size()
+    d2h = host_y.numel() * host_y.element_size()
     s = torch.cuda.current_stream()
+    plans = [bl.LinearPlan(w, X.shape[0], out=Y, scratch=scratch, static_weights=True)
+             for (_, w, _, scratch, _), X, Y in zip(run.layers, x_views, y_views)]
 
     def one():
-        for (p, w, X, scratch, Y), hx, hy in zip(run.layers, host_x, host_y):
-            X.copy_(hx, non_blocking=True)
-            bl.linear(w, X, out=Y, scratch=scratch)
-            hy.copy_(Y, non_blocking=True)
+        dev_x.copy_(host_x, non_blocking=True)
+        for plan, X in zip(plans, x_views):
+            plan(X)
+        host_y.copy_(dev_y, non_blocking=True)
 
     one()
     torch.cuda.synchronize()
@@ -748,8 +765,9 @@ def main():
             "e2e": {"value": round(replica_value(nb["step"], world, e2e_ms), 3),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 4),
-                    "how": "public Python API, pinned host X copied in and Y copied out "
-                           "every forward, eager launches"},
+                    "how": "public Python API (LinearPlan per layer: eager bitlinear_linear "
+                           "calls), every step one copy of all its X in from pinned host memory "
+                           "and one of all its Y out"},
             "gpu_launches": (1 if one_kernel else 2) * len(run.layers) * args.steps,
             "clocks": clocks,
             "device_error": run.bl.status_string(status),

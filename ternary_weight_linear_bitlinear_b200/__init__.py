@@ -102,11 +102,12 @@ def _check(status: int, where: str):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # ctypes converts the integer address through the declared c_void_p.
+    return None if t is None else t.data_ptr()
 
 
 def _stream():
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _need(t, dtype, name):
@@ -240,6 +241,47 @@ def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm
                                 _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
     _check(st, "bitlinear_linear")
     return out
+
+
+class LinearPlan:
+    """bitlinear_linear with everything but X bound once: the weights, the
+    scratch (Xq, beta, rowsum), the output, the flags and the CUDA stream
+    current at construction.  Each call passes X's address to the same
+    entry point and returns the bound output tensor (overwritten by the next
+    call).  For a serving loop that calls the same layer shape repeatedly."""
+
+    def __init__(self, w: PackedTernary, T: int, gain: torch.Tensor = None, rmsnorm: bool = True,
+                 eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.bfloat16,
+                 out: torch.Tensor = None, scratch=None, static_weights: bool = False,
+                 per_tensor: bool = False, device=None):
+        dev = device if device is not None else w.packed.device
+        if scratch is None:
+            scratch = (torch.empty((T, w.d_in), dtype=torch.int8, device=dev),
+                       torch.empty(T, dtype=torch.float32, device=dev),
+                       torch.empty(T, dtype=torch.int32, device=dev))
+        if out is None:
+            out = torch.empty((T, w.d_out), dtype=out_dtype, device=dev)
+        if gain is not None:
+            _need(gain, torch.float32, "gain")
+        Xq, beta, rowsum = scratch
+        _need(Xq, torch.int8, "Xq")
+        flags = ((RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
+                 | (PER_TENSOR_ABSMAX if per_tensor else 0))
+        od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
+        self.w, self.scratch, self.out, self.gain = w, scratch, out, gain   # keep alive
+        self._shape = (T, w.d_in)
+        self._fn = lib().bitlinear_linear
+        self._pre = (w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in)
+        self._post = (T, _ptr(gain), flags, eps, norm_eps, Xq.data_ptr(), beta.data_ptr(),
+                      rowsum.data_ptr(), out.data_ptr(), od, _stream())
+
+    def __call__(self, X: torch.Tensor) -> torch.Tensor:
+        if X.dtype != torch.bfloat16 or tuple(X.shape) != self._shape or not X.is_contiguous():
+            raise TypeError("X must be a contiguous bf16 tensor of shape %s" % (self._shape,))
+        st = self._fn(*self._pre, X.data_ptr(), *self._post)
+        if st != OK:
+            raise BitLinearError(st, "bitlinear_linear")
+        return self.out
 
 
 def backward(w: PackedTernary, Xq: torch.Tensor, beta: torch.Tensor, dY: torch.Tensor,

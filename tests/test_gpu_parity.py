@@ -391,3 +391,19 @@ def test_bounded_wait_reports_timeout():
     # The context is still usable afterwards.
     forward_case(48, 512, 3, torch.float32)
     forward_case(144, 512, 40, torch.float32)
+
+
+def test_linear_plan_matches_linear():
+    """The bound-argument call path gives the same bits as bl.linear."""
+    W, X = draw(Problem("lp", 2560, 272, 1, 0.02, 0.01, 50.0, 12))
+    w = bl.pack_weights(W.to(dev()), EPS)
+    Xd = X.to(dev())
+    ref = bl.linear(w, Xd, out_dtype=torch.bfloat16)
+    plan = bl.LinearPlan(w, 1, out_dtype=torch.bfloat16)
+    X2 = torch.empty_like(Xd)
+    X2.copy_(Xd)
+    got = plan(X2)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+    with pytest.raises(TypeError):
+        plan(Xd.float())
