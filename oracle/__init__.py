@@ -72,6 +72,12 @@ def _load():
         lib.oracle_unpack.restype = i32
         lib.oracle_unpack_row.argtypes = [vp, i64, i64, i64, vp]
         lib.oracle_unpack_row.restype = i32
+        lib.oracle_base3_cols.argtypes = [i64]
+        lib.oracle_base3_cols.restype = i64
+        lib.oracle_pack_base3.argtypes = [vp, i64, i64, vp]
+        lib.oracle_pack_base3.restype = i32
+        lib.oracle_unpack_base3.argtypes = [vp, i64, i64, vp]
+        lib.oracle_unpack_base3.restype = i32
         lib.oracle_inv_rms.argtypes = [vp, i64, f32]
         lib.oracle_inv_rms.restype = f32
         lib.oracle_quant_act.argtypes = [vp, i64, i64, vp, i32, i32, f32, f32, vp,
@@ -170,6 +176,35 @@ def unpack_row(packed, d_out: int, d_in: int, o: int) -> np.ndarray:
     rc = _load().oracle_unpack_row(_ptr(packed), d_out, d_in, o, _ptr(out))
     if rc != 0:
         raise ValueError("oracle_unpack_row: invalid code 3 or bad index")
+    return out
+
+
+def base3_cols(d_in: int) -> int:
+    """Row width of the base-3 format: d_in padded to a multiple of 160."""
+    return int(_load().oracle_base3_cols(d_in))
+
+
+def pack_base3(wq) -> np.ndarray:
+    """Ternary codes [d_out][d_in] -> base-3 bytes, five codes per byte
+    ([MF] section 4), in 16 x 160 tiles."""
+    wq = _c(wq, np.int8)
+    n, k = wq.shape
+    out = np.empty(n * base3_cols(k) // 5 if (n % 16 == 0 and k >= 1) else 0, dtype=np.uint8)
+    rc = _load().oracle_pack_base3(_ptr(wq), n, k, _ptr(out) if out.size else None)
+    if rc != 0:
+        raise ValueError("oracle_pack_base3: d_out not a multiple of 16, or a code "
+                         "outside {-1,0,1}")
+    return out
+
+
+def unpack_base3(packed, d_out: int, d_in: int) -> np.ndarray:
+    packed = _c(packed, np.uint8)
+    if d_out % 16 or d_in < 1 or packed.size != d_out * base3_cols(d_in) // 5:
+        raise ValueError("unpack_base3: size does not match the shape")
+    out = np.empty((d_out, d_in), dtype=np.int8)
+    rc = _load().oracle_unpack_base3(_ptr(packed), d_out, d_in, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_unpack_base3: byte above 242 or a nonzero padding code")
     return out
 
 

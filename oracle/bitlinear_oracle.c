@@ -185,6 +185,83 @@ int oracle_unpack_row(const uint32_t *packed, int64_t n_out, int64_t n_in,
     return 0;
 }
 
+/* ------------------------------------ base-3 packed layout ([MF] §4) --- */
+
+/* [MF] §4, "Memory Bandwidth and Latency Bounds": five ternary values fit in
+ * one byte because 3^5 = 243 < 256.  This library's base-3 format (its own;
+ * the page fixes only the five-per-byte count):
+ *   - each row is padded with W~ = 0 to a whole number of 160 columns;
+ *   - the matrix is cut into tiles of 16 rows x 160 columns (512 bytes),
+ *     stored tile-row-major like the 2-bit format, each row of a tile as 32
+ *     consecutive bytes;
+ *   - byte B of a tile row belongs to the 20-column group g = B / 4 and, with
+ *     j = B % 4, holds the codes c_i = W~ + 1 of the columns 20*g + 4*i + j,
+ *     i = 0..4, as the base-3 number c_0 + 3 c_1 + 9 c_2 + 27 c_3 + 81 c_4.
+ * So a byte never exceeds 242, and a full row costs 8/5 = 1.6 bits per
+ * weight. */
+int64_t oracle_base3_cols(int64_t n_in)
+{
+    return (n_in + 159) / 160 * 160;
+}
+
+/* Byte holding weight (o, k) (k < padded width) and the power of 3 of its
+ * digit. */
+static void base3_position(int64_t n_in, int64_t o, int64_t k, int64_t *byte, int *power)
+{
+    int64_t tiles_per_row = oracle_base3_cols(n_in) / 160;
+    int64_t rb = o / 16, r = o % 16;
+    int64_t kb = k / 160, col = k % 160;
+    int64_t g = col / 20, in_group = col % 20;
+    int i = (int)(in_group / 4), j = (int)(in_group % 4);
+    *byte = ((rb * tiles_per_row + kb) * 16 + r) * 32 + g * 4 + j;
+    *power = i;
+}
+
+static const int kPow3[5] = {1, 3, 9, 27, 81};
+
+/* Returns 0, or -1 if d_out is not a multiple of 16, d_in < 1 or a code is
+ * outside {-1, 0, 1}.  packed holds d_out * padded width / 5 bytes. */
+int oracle_pack_base3(const int8_t *wq, int64_t n_out, int64_t n_in, uint8_t *packed)
+{
+    if (n_out % 16 != 0 || n_in < 1) return -1;
+    const int64_t kp = oracle_base3_cols(n_in);
+    memset(packed, 0, (size_t)(n_out * kp / 5));
+    for (int64_t o = 0; o < n_out; ++o) {
+        for (int64_t k = 0; k < kp; ++k) {
+            int v = k < n_in ? wq[o * n_in + k] : 0;
+            if (v < -1 || v > 1) return -1;
+            int64_t byte;
+            int power;
+            base3_position(n_in, o, k, &byte, &power);
+            packed[byte] = (uint8_t)(packed[byte] + (v + 1) * kPow3[power]);
+        }
+    }
+    return 0;
+}
+
+/* Inverse of oracle_pack_base3: digit i of byte b is (b / 3^i) mod 3.
+ * Returns -1 on a byte above 242 or a padding column that is not W~ = 0. */
+int oracle_unpack_base3(const uint8_t *packed, int64_t n_out, int64_t n_in, int8_t *wq)
+{
+    if (n_out % 16 != 0 || n_in < 1) return -1;
+    const int64_t kp = oracle_base3_cols(n_in);
+    for (int64_t b = 0; b < n_out * kp / 5; ++b)
+        if (packed[b] > 242) return -1;
+    for (int64_t o = 0; o < n_out; ++o) {
+        for (int64_t k = 0; k < kp; ++k) {
+            int64_t byte;
+            int power;
+            base3_position(n_in, o, k, &byte, &power);
+            int c = (packed[byte] / kPow3[power]) % 3;
+            if (k < n_in)
+                wq[o * n_in + k] = (int8_t)(c - 1);
+            else if (c != 1)
+                return -1;
+        }
+    }
+    return 0;
+}
+
 /* ---------------------------------------- activation quantisation ([MF] §2) */
 
 /* Reciprocal RMS of one token: 1 / sqrt(mean(x^2) + norm_eps), carried in

@@ -163,6 +163,87 @@ def test_pack_roundtrip(shape):
         np.testing.assert_array_equal(oracle.unpack_row(p, *shape, o), wq[o])
 
 
+# ------------------------------------------------------ base-3 packing ---
+
+def test_base3_layout_golden(golden_dir):
+    ex = json.load(open(os.path.join(golden_dir, "base3_layout.json")))
+    n, k = ex["d_out"], ex["d_in"]
+    zero = oracle.pack_base3(np.zeros((n, k), np.int8))
+    assert zero.size == ex["bytes"] and (zero == 121).all()
+    for c in ex["cases"]:
+        wq = np.zeros((n, k), np.int8)
+        wq[c["o"], c["k"]] = c["w"]
+        p = oracle.pack_base3(wq)
+        expect = np.full(p.shape, 121, dtype=np.uint8)
+        expect[c["byte"]] = c["value"]
+        np.testing.assert_array_equal(p, expect, err_msg=str(c))
+
+
+def test_base3_constant_matrices():
+    """All -1 packs to 0, all +1 to 242 = 2 (1 + 3 + 9 + 27 + 81); with a
+    ragged width the padding columns hold W~ = 0 (digit 1)."""
+    assert (oracle.pack_base3(np.full((16, 320), -1, np.int8)) == 0).all()
+    assert (oracle.pack_base3(np.full((16, 320), 1, np.int8)) == 242).all()
+    # d_in = 256: tile 1 covers columns 160..319, of which 256..319 are padding:
+    # groups 0..3 (columns 160..239) and 4 (240..255 real, 256..259 padding).
+    p = oracle.pack_base3(np.full((16, 256), -1, np.int8)).reshape(2, 16, 32)
+    assert (p[0] == 0).all()
+    assert (p[1][:, :16] == 0).all()                  # groups 0..3: all real
+    # group 4: columns 240 + 4i + j, real for i < 4, padding (digit 1) for i = 4
+    assert (p[1][:, 16:20] == 81).all()
+    assert (p[1][:, 20:] == 121).all()                # groups 5..7: all padding
+
+
+@pytest.mark.parametrize("shape", [(16, 160), (16, 256), (32, 512), (48, 2560), (16, 4096),
+                                   (32, 11008)])
+def test_base3_roundtrip_and_size(shape):
+    wq = RNG.integers(-1, 2, size=shape).astype(np.int8)
+    p = oracle.pack_base3(wq)
+    kp = -(-shape[1] // 160) * 160
+    assert oracle.base3_cols(shape[1]) == kp
+    assert p.size == shape[0] * kp // 5              # 8/5 = 1.6 bits per padded weight
+    assert p.max() <= 242
+    np.testing.assert_array_equal(oracle.unpack_base3(p, *shape), wq)
+    # The code histogram survives packing: count the digits of every byte.
+    digits = np.stack([(p.astype(np.int64) // 3 ** i) % 3 for i in range(5)], axis=-1)
+    counts = np.bincount(digits.ravel(), minlength=3)
+    want = np.bincount((wq + 1).ravel(), minlength=3)
+    want[1] += shape[0] * (kp - shape[1])            # padding columns are W~ = 0
+    np.testing.assert_array_equal(counts, want)
+
+
+def test_base3_is_a_bijection_on_a_tile():
+    """Every (row, column) of a 16 x 160 tile owns its own (byte, digit)."""
+    seen = set()
+    base = oracle.pack_base3(np.zeros((16, 160), np.int8)).astype(np.int64)
+    for o in range(16):
+        for k in range(160):
+            wq = np.zeros((16, 160), np.int8)
+            wq[o, k] = 1
+            d = oracle.pack_base3(wq).astype(np.int64) - base
+            nz = np.flatnonzero(d)
+            assert nz.size == 1
+            power = int(round(math.log(d[nz[0]], 3)))
+            assert 3 ** power == d[nz[0]] and 0 <= power < 5
+            seen.add((int(nz[0]), power))
+    assert len(seen) == 16 * 160
+
+
+def test_base3_rejects_bad_input():
+    with pytest.raises(ValueError):
+        oracle.pack_base3(np.full((16, 160), 2, np.int8))
+    with pytest.raises(ValueError):
+        oracle.pack_base3(np.zeros((8, 160), np.int8))
+    bad = oracle.pack_base3(np.zeros((16, 160), np.int8))
+    bad[7] = 243
+    with pytest.raises(ValueError):
+        oracle.unpack_base3(bad, 16, 160)
+    pad = oracle.pack_base3(np.zeros((16, 256), np.int8))
+    pad[-1] = 0                                      # padding column set to -1
+    with pytest.raises(ValueError):
+        oracle.unpack_base3(pad, 16, 256)
+
+
 def test_pack_exhaustive_groups():
     """All 81 joint values of the four codes that share one byte (same s)
     and of the four that share one 2-bit slot across bytes (same j)."""
