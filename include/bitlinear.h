@@ -236,6 +236,59 @@ int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
                      void *Y, int out_dtype, cudaStream_t stream);
 
 /*
+ * Base-3 weight format ([MF] section 4, "Memory Bandwidth and Latency
+ * Bounds": five ternary values fit in one byte, 3^5 = 243 < 256, so a weight
+ * costs 1.6 bits instead of 2).  This library's own order: each row is padded
+ * with W~ = 0 to Kp = 160 * ceil(d_in / 160) columns; the matrix is cut into
+ * tiles of 16 rows x 160 columns (512 bytes) stored tile-row-major (tile
+ * (rb, kb) at byte 512 * (rb * Kp/160 + kb)); inside a tile the 16 rows follow
+ * one another as 32 bytes each; byte B of a tile row belongs to the
+ * 20-column group g = B / 4 and, with j = B % 4, holds the codes
+ * c_i = W~ + 1 of columns 20*g + 4*i + j (i = 0..4) as the base-3 number
+ * c_0 + 3 c_1 + 9 c_2 + 27 c_3 + 81 c_4 (never above 242).  Four bytes of a
+ * group thus give, digit by digit, the codes of four consecutive columns.
+ * Size: d_out * Kp / 5 bytes.  Decode-only: the entry points below take
+ * 1 <= T <= 16.
+ */
+
+/* Bytes of the base-3 format for d_out x d_in, or 0 if the shape is
+ * unsupported (same shape rules as the 2-bit format). */
+size_t bitlinear_base3_bytes(int64_t d_out, int64_t d_in);
+
+/*
+ * bitlinear_repack_base3 -- convert 2-bit packed weights (as written by
+ * bitlinear_pack_weights) into the base-3 format, exactly.
+ *   packed   in: 2-bit layout, d_out x d_in, 16-byte aligned.
+ *   packed3  out: bitlinear_base3_bytes(d_out, d_in) bytes, 16-byte aligned.
+ * gamma is unchanged and shared by both formats.
+ */
+int bitlinear_repack_base3(const uint32_t *packed, int64_t d_out, int64_t d_in,
+                           uint8_t *packed3, cudaStream_t stream);
+
+/*
+ * bitlinear_forward_base3 -- bitlinear_forward on base-3 weights: the same
+ * arguments, meaning and results (the int32 accumulators are the same exact
+ * integers), for 1 <= T <= 16 (otherwise BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+ * T = 0 is a no-op).  The decode kernel expands each byte to its five codes
+ * in registers and multiplies them on the warp-level int8 tensor-core MMA.
+ */
+int bitlinear_forward_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
+                            int64_t d_in, const int8_t *Xq, const float *beta,
+                            const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                            int32_t *acc_out, cudaStream_t stream);
+
+/*
+ * bitlinear_linear_base3 -- bitlinear_linear on base-3 weights (same
+ * arguments, flags and results), for 1 <= T <= 16.  BITLINEAR_PER_TENSOR_ABSMAX
+ * runs the quantiser first, as in bitlinear_linear.
+ */
+int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
+                           int64_t d_in, const uint16_t *X, int64_t T,
+                           const float *norm_gain, uint32_t flags, float eps,
+                           float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
+                           void *Y, int out_dtype, cudaStream_t stream);
+
+/*
  * bitlinear_dense_bf16_forward -- the dense bf16 linear layer Y = X W^T that
  * BitLinear replaces, kept as the context the measurements compare against
  * ([MF] section 2, "The Linear Transformation and Rescaling", without the

@@ -55,6 +55,12 @@ SIGNATURES = {
                                  _vp, _vp]),
     "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
                                 _vp, _vp, _vp, _vp, _int, _vp]),
+    "bitlinear_base3_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "bitlinear_repack_base3": (_int, [_vp, _i64, _i64, _vp, _vp]),
+    "bitlinear_forward_base3": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int,
+                                       _vp, _vp]),
+    "bitlinear_linear_base3": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
+                                      _vp, _vp, _vp, _vp, _int, _vp]),
     "bitlinear_dense_bf16_forward": (_int, [_vp, _i64, _i64, _vp, _i64, _vp, _int, _vp]),
     "bitlinear_backward_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _int, _int]),
     "bitlinear_backward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _int, _vp,
@@ -128,6 +134,38 @@ class PackedTernary:
     d_in: int
 
 
+@dataclass
+class PackedTernaryBase3:
+    """The same ternary weights in the base-3 format, five codes per byte
+    (layout in bitlinear.h); decode only (1 <= T <= 16)."""
+    packed: torch.Tensor    # uint8 [base3_bytes(d_out, d_in)]
+    gamma: torch.Tensor     # float32 [1], shared with the 2-bit weights
+    d_out: int
+    d_in: int
+
+
+def _entry(w, name: str):
+    """The entry point for w's format: name, or name + '_base3'."""
+    full = name + "_base3" if isinstance(w, PackedTernaryBase3) else name
+    return getattr(lib(), full), full
+
+
+def base3_bytes(d_out: int, d_in: int) -> int:
+    return int(lib().bitlinear_base3_bytes(d_out, d_in))
+
+
+def repack_base3(w: PackedTernary, out: torch.Tensor = None) -> PackedTernaryBase3:
+    """2-bit packed weights -> the base-3 format (exact; gamma shared)."""
+    n = base3_bytes(w.d_out, w.d_in)
+    if n == 0:
+        _check(ERR_UNSUPPORTED_SHAPE, "repack_base3")
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=w.packed.device)
+    st = lib().bitlinear_repack_base3(_ptr(w.packed), w.d_out, w.d_in, _ptr(out), _stream())
+    _check(st, "bitlinear_repack_base3")
+    return PackedTernaryBase3(out, w.gamma, w.d_out, w.d_in)
+
+
 def packed_words(d_out: int, d_in: int) -> int:
     return int(lib().bitlinear_packed_words(d_out, d_in))
 
@@ -192,9 +230,10 @@ def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
     return Xq, beta, rowsum, rms_out
 
 
-def forward(w: PackedTernary, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
+def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
             out_dtype=torch.float32, want_acc: bool = False, out: torch.Tensor = None):
-    """Y = (X~ W~^T) gamma beta / 127; returns Y (and the int32 acc if asked)."""
+    """Y = (X~ W~^T) gamma beta / 127; returns Y (and the int32 acc if asked).
+    w is a PackedTernary or a PackedTernaryBase3."""
     _need(Xq, torch.int8, "Xq")
     T = Xq.shape[0]
     dev = Xq.device
@@ -202,18 +241,19 @@ def forward(w: PackedTernary, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torc
         out = torch.empty((T, w.d_out), dtype=out_dtype, device=dev)
     od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
     acc = torch.empty((T, w.d_out), dtype=torch.int32, device=dev) if want_acc else None
-    st = lib().bitlinear_forward(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq),
-                                 _ptr(beta), _ptr(rowsum), T, _ptr(out), od, _ptr(acc),
-                                 _stream())
-    _check(st, "bitlinear_forward")
+    fn, name = _entry(w, "bitlinear_forward")
+    st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq), _ptr(beta), _ptr(rowsum), T,
+            _ptr(out), od, _ptr(acc), _stream())
+    _check(st, name)
     return (out, acc) if want_acc else out
 
 
-def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
+def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
            eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.float32,
            out: torch.Tensor = None, scratch=None, static_weights: bool = False,
            per_tensor: bool = False):
     """The whole BitLinear forward from bf16 X: quantise, then product.
+    w is a PackedTernary or a PackedTernaryBase3.
 
     static_weights: promise that no work still in flight on the stream
     writes w.packed or w.gamma (the product may then stream the weights
@@ -236,10 +276,10 @@ def linear(w: PackedTernary, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm
         _need(gain, torch.float32, "gain")
     flags = ((RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
              | (PER_TENSOR_ABSMAX if per_tensor else 0))
-    st = lib().bitlinear_linear(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(X), T,
-                                _ptr(gain), flags, eps, norm_eps,
-                                _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
-    _check(st, "bitlinear_linear")
+    fn, name = _entry(w, "bitlinear_linear")
+    st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(X), T, _ptr(gain), flags, eps,
+            norm_eps, _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
+    _check(st, name)
     return out
 
 
@@ -250,7 +290,7 @@ class LinearPlan:
     entry point and returns the bound output tensor (overwritten by the next
     call).  For a serving loop that calls the same layer shape repeatedly."""
 
-    def __init__(self, w: PackedTernary, T: int, gain: torch.Tensor = None, rmsnorm: bool = True,
+    def __init__(self, w, T: int, gain: torch.Tensor = None, rmsnorm: bool = True,
                  eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.bfloat16,
                  out: torch.Tensor = None, scratch=None, static_weights: bool = False,
                  per_tensor: bool = False, device=None):
@@ -270,7 +310,7 @@ class LinearPlan:
         od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
         self.w, self.scratch, self.out, self.gain = w, scratch, out, gain   # keep alive
         self._shape = (T, w.d_in)
-        self._fn = lib().bitlinear_linear
+        self._fn, self._name = _entry(w, "bitlinear_linear")
         self._pre = (w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in)
         self._post = (T, _ptr(gain), flags, eps, norm_eps, Xq.data_ptr(), beta.data_ptr(),
                       rowsum.data_ptr(), out.data_ptr(), od, _stream())
@@ -280,7 +320,7 @@ class LinearPlan:
             raise TypeError("X must be a contiguous bf16 tensor of shape %s" % (self._shape,))
         st = self._fn(*self._pre, X.data_ptr(), *self._post)
         if st != OK:
-            raise BitLinearError(st, "bitlinear_linear")
+            raise BitLinearError(st, self._name)
         return self.out
 
 

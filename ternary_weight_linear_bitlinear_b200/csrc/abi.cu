@@ -14,16 +14,18 @@ bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                                   float norm_eps, const float *inv_rms_in, int8_t *Xq,
                                   float *beta, int32_t *rowsum, float *inv_rms_out, bool pdl,
                                   cudaStream_t stream);
-bitlinear_status launch_gemv(const uint32_t *packed, const float *gamma, int64_t d_out,
+bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_out,
                              int64_t d_in, const int8_t *Xq, const float *beta,
                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                             int32_t *acc_out, bool static_weights, cudaStream_t stream);
+                             int32_t *acc_out, bool static_weights, bool base3,
+                             cudaStream_t stream);
 bool decode_can_fuse(int64_t T, int64_t d_in);
-bitlinear_status launch_linear_fused(const uint32_t *packed, const float *gamma, int64_t d_out,
+bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const uint16_t *X, int64_t T,
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
                                      int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
-                                     int out_dtype, bool static_weights, cudaStream_t stream);
+                                     int out_dtype, bool static_weights, bool base3,
+                                     cudaStream_t stream);
 bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int64_t d_out,
                                 int64_t d_in, const int8_t *Xq, const float *beta,
                                 const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
@@ -107,7 +109,7 @@ cudaError_t ensure_dynamic_smem(const void *kernel, size_t bytes) {
     return cudaSuccess;
 }
 
-static bitlinear_status validate_forward(const uint32_t *packed, const float *gamma,
+static bitlinear_status validate_forward(const void *packed, const float *gamma,
                                          int64_t d_out, int64_t d_in, int64_t T, void *Y,
                                          int out_dtype, int32_t *acc_out) {
     if (T < 0 || T > (1 << 20)) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
@@ -123,16 +125,69 @@ static bitlinear_status validate_forward(const uint32_t *packed, const float *ga
     return BITLINEAR_OK;
 }
 
-static bitlinear_status dispatch_forward(const uint32_t *packed, const float *gamma,
+static bitlinear_status dispatch_forward(const void *packed, const float *gamma,
                                          int64_t d_out, int64_t d_in, const int8_t *Xq,
                                          const float *beta, const int32_t *rowsum, int64_t T,
                                          void *Y, int out_dtype, int32_t *acc_out,
-                                         bool static_weights, cudaStream_t stream) {
-    if (T <= 16)
+                                         bool static_weights, bool base3, cudaStream_t stream) {
+    if (T <= 16 || base3)
         return launch_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                           acc_out, static_weights, stream);
-    return launch_gemm_tc(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype, acc_out,
-                          stream);
+                           acc_out, static_weights, base3, stream);
+    return launch_gemm_tc(static_cast<const uint32_t *>(packed), gamma, d_out, d_in, Xq, beta,
+                          rowsum, T, Y, out_dtype, acc_out, stream);
+}
+
+static bitlinear_status forward_common(const void *packed, const float *gamma, int64_t d_out,
+                                       int64_t d_in, const int8_t *Xq, const float *beta,
+                                       const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                                       int32_t *acc_out, bool base3, cudaStream_t stream) {
+    bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, acc_out);
+    if (st != BITLINEAR_OK) return st;
+    if (base3 && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return BITLINEAR_OK;
+    if (!Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4))
+        return BITLINEAR_ERR_MISALIGNED;
+    st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
+                            acc_out, false, base3, stream);
+}
+
+static bitlinear_status linear_common(const void *packed, const float *gamma, int64_t d_out,
+                                      int64_t d_in, const uint16_t *X, int64_t T,
+                                      const float *norm_gain, uint32_t flags, float eps,
+                                      float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
+                                      void *Y, int out_dtype, bool base3, cudaStream_t stream) {
+    bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, nullptr);
+    if (st != BITLINEAR_OK) return st;
+    if (base3 && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_STATIC_WEIGHTS | BITLINEAR_PER_TENSOR_ABSMAX))
+        return BITLINEAR_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !std::isfinite(eps) || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps))
+        return BITLINEAR_ERR_INVALID_ARG;
+    if (T == 0) return BITLINEAR_OK;
+    if (!X || !Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4) ||
+        (norm_gain && !aligned(norm_gain, 4)))
+        return BITLINEAR_ERR_MISALIGNED;
+    st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
+    const bool rmsnorm = (flags & BITLINEAR_RMSNORM) != 0;
+    const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
+    if (!per_tensor && decode_can_fuse(T, d_in))
+        return launch_linear_fused(packed, gamma, d_out, d_in, X, T, norm_gain, rmsnorm, eps,
+                                   norm_eps, Xq, beta, rowsum, Y, out_dtype, static_weights,
+                                   base3, stream);
+    // Quantiser, then the product as its programmatic dependent: with static
+    // weights the product streams them while the codes are still being made.
+    st = launch_quant_act(X, T, d_in, norm_gain,
+                          flags & (BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX), eps,
+                          norm_eps, nullptr, Xq, beta, rowsum, nullptr, true, stream);
+    if (st != BITLINEAR_OK) return st;
+    return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
+                            nullptr, static_weights, base3, stream);
 }
 
 }  // namespace bl
@@ -158,16 +213,16 @@ extern "C" int bitlinear_forward(const uint32_t *packed, const float *gamma, int
                                  int64_t d_in, const int8_t *Xq, const float *beta,
                                  const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
                                  int32_t *acc_out, cudaStream_t stream) {
-    bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, acc_out);
-    if (st != BITLINEAR_OK) return st;
-    if (T == 0) return BITLINEAR_OK;
-    if (!Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
-    if (!aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4))
-        return BITLINEAR_ERR_MISALIGNED;
-    st = check_device();
-    if (st != BITLINEAR_OK) return st;
-    return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                            acc_out, false, stream);
+    return forward_common(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype, acc_out,
+                          false, stream);
+}
+
+extern "C" int bitlinear_forward_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
+                                       int64_t d_in, const int8_t *Xq, const float *beta,
+                                       const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                                       int32_t *acc_out, cudaStream_t stream) {
+    return forward_common(packed3, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
+                          acc_out, true, stream);
 }
 
 extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
@@ -175,34 +230,17 @@ extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int6
                                 const float *norm_gain, uint32_t flags, float eps, float norm_eps,
                                 int8_t *Xq, float *beta, int32_t *rowsum, void *Y, int out_dtype,
                                 cudaStream_t stream) {
-    bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, nullptr);
-    if (st != BITLINEAR_OK) return st;
-    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_STATIC_WEIGHTS | BITLINEAR_PER_TENSOR_ABSMAX))
-        return BITLINEAR_ERR_INVALID_ARG;
-    if (!(eps >= 0.0f) || !std::isfinite(eps) || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps))
-        return BITLINEAR_ERR_INVALID_ARG;
-    if (T == 0) return BITLINEAR_OK;
-    if (!X || !Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
-    if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4) ||
-        (norm_gain && !aligned(norm_gain, 4)))
-        return BITLINEAR_ERR_MISALIGNED;
-    st = check_device();
-    if (st != BITLINEAR_OK) return st;
-    const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
-    const bool rmsnorm = (flags & BITLINEAR_RMSNORM) != 0;
-    const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
-    if (!per_tensor && decode_can_fuse(T, d_in))
-        return launch_linear_fused(packed, gamma, d_out, d_in, X, T, norm_gain, rmsnorm, eps,
-                                   norm_eps, Xq, beta, rowsum, Y, out_dtype, static_weights,
-                                   stream);
-    // Quantiser, then the product as its programmatic dependent: with static
-    // weights the product streams them while the codes are still being made.
-    st = launch_quant_act(X, T, d_in, norm_gain,
-                          flags & (BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX), eps,
-                          norm_eps, nullptr, Xq, beta, rowsum, nullptr, true, stream);
-    if (st != BITLINEAR_OK) return st;
-    return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                            nullptr, static_weights, stream);
+    return linear_common(packed, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps, Xq,
+                         beta, rowsum, Y, out_dtype, false, stream);
+}
+
+extern "C" int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
+                                      int64_t d_in, const uint16_t *X, int64_t T,
+                                      const float *norm_gain, uint32_t flags, float eps,
+                                      float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
+                                      void *Y, int out_dtype, cudaStream_t stream) {
+    return linear_common(packed3, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps, Xq,
+                         beta, rowsum, Y, out_dtype, true, stream);
 }
 
 extern "C" int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, int64_t d_in,

@@ -44,12 +44,26 @@
 // declared them static (not written by work still in flight): then the
 // weight stream of this layer overlaps the tail of the previous one.
 //
+// BASE-3 variant (section 4 of the same page, "Memory Bandwidth and Latency
+// Bounds": five ternary values per byte, 1.6 bits per weight).  Tiles of 16
+// rows x 160 columns (512 bytes); lane (g, q) reads 8 bytes of rows g and
+// g+8 (bytes 8 lane.. and 256 + 8 lane.., conflict-free) = two 20-column
+// groups = columns 40q .. 40q+39 of the tile.  A byte b is expanded with
+// packed half-precision arithmetic, exact for every b < 243: the halves
+// v = 1024 + b (bit pattern 0x6400 | b) give the quotient by 3 as
+// v' = RN(v * fp16(1/3) + 682.5) = 1024 + floor(b / 3) and the digit as
+// e = v - 3 v' = d - 2048, whose low byte is -d as an int8.  Four bytes of a
+// group thus yield, digit by digit, the s8 values -c of four consecutive
+// columns -- an A-operand register of an s8 MMA whose activation fragment is
+// eight consecutive code bytes.  The accumulator is -sum c x.
+//
 // Every mbarrier wait is bounded; on expiry the CTA stops consuming, the
 // producer waits (bounded) for the copies it issued, and the error word is
 // set.
 #include <cstdint>
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "bitlinear.h"
 #include "common.cuh"
@@ -63,10 +77,11 @@ constexpr int kDecMaxStages = 4;
 static_assert(kDecWarps * 32 == kQuantThreads, "fused quantiser runs on the consumer warps");
 
 struct DecodeArgs {
-    const uint4 *packed;
+    const uint8_t *packed;   // 2-bit tiles (1 KiB) or base-3 tiles (512 B)
     const float *gamma;
     int d_out;
-    int kb_total;            // d_in / 256
+    int d_in;
+    int kb_total;            // k-tiles per row: d_in / 256, or ceil(d_in / 160) in base 3
     int T;
     // product-only inputs (written by the stand-alone quantiser)
     const int8_t *Xq;
@@ -105,6 +120,44 @@ __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_s8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ __half2 h2_bits(uint32_t u) {
+    return *reinterpret_cast<const __half2 *>(&u);
+}
+__device__ __forceinline__ uint32_t h2_u32(__half2 h) {
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Four base-3 bytes (one 20-column group) -> d[i] = the int8 values -c of
+// columns 4i .. 4i+3 of the group (byte j -> column 4i + j), i = 0..4.
+__device__ __forceinline__ void base3_neg_codes(uint32_t w, uint32_t *d) {
+    const __half2 third = h2_bits(0x35553555u);    // fp16(1/3) = 0.33325195
+    const __half2 bias = h2_bits(0x61556155u);     // 682.5
+    const __half2 minus3 = h2_bits(0xC200C200u);   // -3
+    const __half2 m3072 = h2_bits(0xEA00EA00u);    // -3072
+    __half2 ve = h2_bits(__byte_perm(w, 0x64646464u, 0x4240));   // 1024 + b0, 1024 + b2
+    __half2 vo = h2_bits(__byte_perm(w, 0x64646464u, 0x4341));   // 1024 + b1, 1024 + b3
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 qe = __hfma2(ve, third, bias);   // 1024 + floor(v / 3)
+        const __half2 qo = __hfma2(vo, third, bias);
+        const uint32_t ee = h2_u32(__hfma2(qe, minus3, ve));   // digit - 2048
+        const uint32_t eo = h2_u32(__hfma2(qo, minus3, vo));
+        d[i] = __byte_perm(ee, eo, 0x6240);
+        ve = qe;
+        vo = qo;
+    }
+    d[4] = __byte_perm(h2_u32(__hadd2(ve, m3072)), h2_u32(__hadd2(vo, m3072)), 0x6240);
+}
+
 // Bulk (TMA-engine) copy of `bytes` contiguous bytes global -> shared,
 // completing on an mbarrier.  Both addresses 16-byte aligned, bytes % 16 == 0.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
@@ -135,10 +188,12 @@ __device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, const De
     }
 }
 
-template <int NT, int R, bool FUSED, bool OUT_BF16>
+template <int NT, int R, bool FUSED, bool OUT_BF16, bool B3>
 __global__ void __launch_bounds__(kDecThreads)
 decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx ctx) {
     constexpr int TMAX = NT * 8;
+    constexpr int kTileBytes = B3 ? 512 : 1024;
+    constexpr int kTileCols = B3 ? 160 : 256;
     extern __shared__ __align__(128) uint8_t dsm[];
     __shared__ __align__(8) uint64_t full_bar[kDecMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kDecMaxStages];
@@ -150,7 +205,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     __shared__ int s_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KB = a.kb_total, K = KB * 256, T = a.T;
+    const int KB = a.kb_total, K = a.d_in, T = a.T;
     const int n_rt = a.d_out >> 4;
     const int n_groups = (n_rt + R - 1) / R;
     const int grp0 = (int)(((long long)n_groups * blockIdx.x) / gridDim.x);
@@ -182,6 +237,11 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
         if (lane == 0) {
             // Unit (gi, sl): group grp0 + gi, slab sl; units run gi-major.
             auto slab_kb = [&](int sl) { return KB - sl * ks < ks ? KB - sl * ks : ks; };
+            // Activation columns of a slab (the last base-3 tile may overhang d_in).
+            auto slab_cols = [&](int sl) {
+                const int c = slab_kb(sl) * kTileCols, left = K - sl * ks * kTileCols;
+                return c < left ? c : left;
+            };
             auto issue_w = [&](int gi, int sl, int st) {
                 const uint32_t bar = smem_u32(&full_bar[st]);
                 const int rt = (grp0 + gi) * R;
@@ -189,21 +249,20 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 int nrow = 0;
                 #pragma unroll
                 for (int r = 0; r < R; ++r) nrow += rt + r < n_rt ? 1 : 0;
-                const uint32_t xbytes = FUSED ? 0u : (uint32_t)(T * nkb * 256);
-                mbar_arrive_expect_tx(bar, (uint32_t)(nrow * nkb * 1024) + xbytes);
+                const uint32_t xbytes = FUSED ? 0u : (uint32_t)(T * slab_cols(sl));
+                mbar_arrive_expect_tx(bar, (uint32_t)(nrow * nkb * kTileBytes) + xbytes);
                 for (int r = 0; r < nrow; ++r)
-                    bulk_g2s(ring_s + st * stage_bytes + r * ks * 1024,
-                             a.packed + ((size_t)(rt + r) * KB + (size_t)sl * ks) * 64,
-                             (uint32_t)(nkb * 1024), bar);
+                    bulk_g2s(ring_s + st * stage_bytes + r * ks * kTileBytes,
+                             a.packed + ((size_t)(rt + r) * KB + (size_t)sl * ks) * kTileBytes,
+                             (uint32_t)(nkb * kTileBytes), bar);
             };
             auto issue_x = [&](int sl, int st) {
                 if (FUSED) return;
                 const uint32_t bar = smem_u32(&full_bar[st]);
-                const int nkb = slab_kb(sl);
                 for (int t = 0; t < T; ++t)
-                    bulk_g2s(ring_s + st * stage_bytes + R * ks * 1024 + t * ks * 256,
-                             a.Xq + (size_t)t * K + (size_t)sl * ks * 256, (uint32_t)(nkb * 256),
-                             bar);
+                    bulk_g2s(ring_s + st * stage_bytes + R * ks * kTileBytes + t * ks * kTileCols,
+                             a.Xq + (size_t)t * K + (size_t)sl * ks * kTileCols,
+                             (uint32_t)slab_cols(sl), bar);
             };
             const int first = units < stages ? units : stages;
             if (a.static_weights) {
@@ -285,7 +344,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                     }
                     const uint4 *xrow = reinterpret_cast<const uint4 *>(xb + (size_t)t * K);
                     uint2 *qrow = reinterpret_cast<uint2 *>(xs + (size_t)t * K);
-                    for (int kb = warp; kb < KB; kb += kDecWarps) {
+                    for (int kb = warp; kb < (K >> 8); kb += kDecWarps) {
                         const int v = kb * 32 + lane;
                         qrow[v] = codes8(xrow[v], rmsnorm, ts.inv_rms, ts.scale, &sums[t]);
                     }
@@ -299,6 +358,9 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 }
             }
             __syncwarp();
+            // Base-3 tiles do not line up with the quantiser's 256-column
+            // blocks: every warp needs every code.
+            if constexpr (B3) consumer_barrier();
         } else {
             token_stats<TMAX, true>(xb, T, K, a.gain, a.rmsnorm != 0, a.eps, a.norm_eps,
                                     a.inv_k, nullptr, qs);
@@ -347,6 +409,45 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             const uint8_t *stage = ring + st * stage_bytes;
             const int nkb = KB - sl * ks < ks ? KB - sl * ks : ks;
+            if constexpr (B3) {
+                for (int kk = warp; kk < nkb; kk += kDecWarps) {
+                    // This lane's 40 columns of the tile: 40q .. 40q+39.
+                    const int col0 = (sl * ks + kk) * 160 + 40 * q;
+                    uint32_t dg[R][10], dh[R][10];   // rows g and g + 8
+                    #pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const uint8_t *tile = stage + (r * ks + kk) * 512;
+                        const uint2 lo = *reinterpret_cast<const uint2 *>(tile + lane * 8);
+                        const uint2 hi = *reinterpret_cast<const uint2 *>(tile + 256 + lane * 8);
+                        base3_neg_codes(lo.x, &dg[r][0]);
+                        base3_neg_codes(lo.y, &dg[r][5]);
+                        base3_neg_codes(hi.x, &dh[r][0]);
+                        base3_neg_codes(hi.y, &dh[r][5]);
+                    }
+                    #pragma unroll
+                    for (int m = 0; m < 5; ++m) {
+                        const bool in_k = col0 + 8 * m < K;   // d_in is a multiple of 8
+                        uint2 xr[NT];
+                        #pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const int t = nt * 8 + g;
+                            const uint8_t *xsrc =
+                                FUSED ? reinterpret_cast<const uint8_t *>(xs) + (size_t)t * K +
+                                            col0 + 8 * m
+                                      : stage + R * ks * 512 + t * ks * 160 + kk * 160 + 40 * q +
+                                            8 * m;
+                            xr[nt] = make_uint2(0, 0);
+                            if (t < T && in_k) xr[nt] = *reinterpret_cast<const uint2 *>(xsrc);
+                        }
+                        #pragma unroll
+                        for (int r = 0; r < R; ++r)
+                            #pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                mma_s8s8(acc[r][nt][0], dg[r][2 * m], dh[r][2 * m],
+                                         dg[r][2 * m + 1], dh[r][2 * m + 1], xr[nt].x, xr[nt].y);
+                    }
+                }
+            } else
             for (int kk = warp; kk < nkb; kk += kDecWarps) {
                 uint32_t w0[R][4], w1[R][4];
                 #pragma unroll
@@ -405,8 +506,9 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 int c[4];
                 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    c[e] = acc[r][nt][0][e] + (acc[r][nt][1][e] >> 2) +
-                           (acc[r][nt][2][e] >> 4) + (acc[r][nt][3][e] >> 6);
+                    c[e] = B3 ? -acc[r][nt][0][e]
+                              : acc[r][nt][0][e] + (acc[r][nt][1][e] >> 2) +
+                                    (acc[r][nt][2][e] >> 4) + (acc[r][nt][3][e] >> 6);
                 red[warp][r][nt][lane] = make_int4(c[0], c[1], c[2], c[3]);
             }
         consumer_barrier();
@@ -492,16 +594,19 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
 #endif
 constexpr int kFusedMaxCodeBytes = BL_FUSED_MAX_CODE_BYTES;
 
-template <int NT, int R, bool FUSED, bool OUT_BF16>
+template <int NT, int R, bool FUSED, bool OUT_BF16, bool B3>
 static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
                                    cudaStream_t stream) {
+    constexpr int kTileBytes = B3 ? 512 : 1024;
+    constexpr int kTileCols = B3 ? 160 : 256;
     const int n_rt = args.d_out / 16;
     const int n_groups = (n_rt + R - 1) / R;
-    const int KB = args.kb_total, K = KB * 256;
+    const int KB = args.kb_total, K = args.d_in;
     DecodePlan plan;
     plan.xs_bytes = FUSED ? ((args.T * K + 127) & ~127) : 0;
     const int xb_bytes = FUSED ? ((args.T * K * 2 + 127) & ~127) : 0;
-    const int per_kb = R * 1024 + (FUSED ? 0 : args.T * 256);   // bytes per k-block column
+    // bytes per k-tile column of a stage
+    const int per_kb = R * kTileBytes + (FUSED ? 0 : args.T * kTileCols);
     plan.ks = BL_DEC_STAGE_BYTES / per_kb;
     if (plan.ks > KB) plan.ks = KB;
     // With several slabs keep ks a multiple of the warp count, so that warp w
@@ -518,7 +623,7 @@ static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
     if (plan.stages < 2) plan.stages = 2;
     const size_t smem =
         (size_t)xb_bytes + (size_t)plan.xs_bytes + (size_t)plan.stages * plan.stage_bytes;
-    auto kern = decode_kernel<NT, R, FUSED, OUT_BF16>;
+    auto kern = decode_kernel<NT, R, FUSED, OUT_BF16, B3>;
     cudaError_t e = ensure_dynamic_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148, per_sm = 1;
@@ -546,7 +651,7 @@ static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
     return cudaLaunchKernelEx(&cfg, kern, args, plan, ctx);
 }
 
-template <bool FUSED, bool OUT_BF16>
+template <bool FUSED, bool OUT_BF16, bool B3>
 static cudaError_t launch_decode_r(const DecodeArgs &args, const DeviceCtx &ctx,
                                    cudaStream_t stream) {
     // One row tile per group while that still leaves a few CTAs per SM;
@@ -554,42 +659,49 @@ static cudaError_t launch_decode_r(const DecodeArgs &args, const DeviceCtx &ctx,
     const int n_rt = args.d_out / 16;
     const bool wide = n_rt >= BL_DEC_WIDE_ROW_TILES;
     if (args.T <= 8)
-        return wide ? launch_decode_t<1, 2, FUSED, OUT_BF16>(args, ctx, stream)
-                    : launch_decode_t<1, 1, FUSED, OUT_BF16>(args, ctx, stream);
+        return wide ? launch_decode_t<1, 2, FUSED, OUT_BF16, B3>(args, ctx, stream)
+                    : launch_decode_t<1, 1, FUSED, OUT_BF16, B3>(args, ctx, stream);
     if constexpr (FUSED) return cudaErrorInvalidValue;   // fused path is T <= 8 only
-    return wide ? launch_decode_t<2, 2, false, OUT_BF16>(args, ctx, stream)
-                : launch_decode_t<2, 1, false, OUT_BF16>(args, ctx, stream);
+    return wide ? launch_decode_t<2, 2, false, OUT_BF16, B3>(args, ctx, stream)
+                : launch_decode_t<2, 1, false, OUT_BF16, B3>(args, ctx, stream);
 }
 
 bool decode_can_fuse(int64_t T, int64_t d_in) {
     return T >= 1 && T <= 8 && T * d_in <= kFusedMaxCodeBytes;
 }
 
-bitlinear_status launch_decode(const DecodeArgs &args, bool fused, int out_dtype,
+template <bool B3>
+static cudaError_t launch_decode_f(const DecodeArgs &args, bool fused, bool bf,
+                                   const DeviceCtx &ctx, cudaStream_t stream) {
+    if (fused)
+        return bf ? launch_decode_r<true, true, B3>(args, ctx, stream)
+                  : launch_decode_r<true, false, B3>(args, ctx, stream);
+    return bf ? launch_decode_r<false, true, B3>(args, ctx, stream)
+              : launch_decode_r<false, false, B3>(args, ctx, stream);
+}
+
+bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, bool base3,
                                cudaStream_t stream) {
     DeviceCtx ctx;
     bitlinear_status st = get_ctx(&ctx);
     if (st != BITLINEAR_OK) return st;
-    cudaError_t e;
     const bool bf = out_dtype == BITLINEAR_OUT_BF16;
-    if (fused)
-        e = bf ? launch_decode_r<true, true>(args, ctx, stream)
-               : launch_decode_r<true, false>(args, ctx, stream);
-    else
-        e = bf ? launch_decode_r<false, true>(args, ctx, stream)
-               : launch_decode_r<false, false>(args, ctx, stream);
+    args.kb_total = base3 ? (args.d_in + 159) / 160 : args.d_in / 256;
+    const cudaError_t e = base3 ? launch_decode_f<true>(args, fused, bf, ctx, stream)
+                                : launch_decode_f<false>(args, fused, bf, ctx, stream);
     return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
-bitlinear_status launch_gemv(const uint32_t *packed, const float *gamma, int64_t d_out,
+bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_out,
                              int64_t d_in, const int8_t *Xq, const float *beta,
                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                             int32_t *acc_out, bool static_weights, cudaStream_t stream) {
+                             int32_t *acc_out, bool static_weights, bool base3,
+                             cudaStream_t stream) {
     DecodeArgs a = {};
-    a.packed = reinterpret_cast<const uint4 *>(packed);
+    a.packed = static_cast<const uint8_t *>(packed);
     a.gamma = gamma;
     a.d_out = (int)d_out;
-    a.kb_total = (int)(d_in / 256);
+    a.d_in = (int)d_in;
     a.T = (int)T;
     a.Xq = Xq;
     a.beta = beta;
@@ -597,19 +709,20 @@ bitlinear_status launch_gemv(const uint32_t *packed, const float *gamma, int64_t
     a.Y = Y;
     a.acc_out = acc_out;
     a.static_weights = static_weights ? 1 : 0;
-    return launch_decode(a, false, out_dtype, stream);
+    return launch_decode(a, false, out_dtype, base3, stream);
 }
 
-bitlinear_status launch_linear_fused(const uint32_t *packed, const float *gamma, int64_t d_out,
+bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const uint16_t *X, int64_t T,
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
                                      int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
-                                     int out_dtype, bool static_weights, cudaStream_t stream) {
+                                     int out_dtype, bool static_weights, bool base3,
+                                     cudaStream_t stream) {
     DecodeArgs a = {};
-    a.packed = reinterpret_cast<const uint4 *>(packed);
+    a.packed = static_cast<const uint8_t *>(packed);
     a.gamma = gamma;
     a.d_out = (int)d_out;
-    a.kb_total = (int)(d_in / 256);
+    a.d_in = (int)d_in;
     a.T = (int)T;
     a.X = X;
     a.gain = gain;
@@ -622,7 +735,7 @@ bitlinear_status launch_linear_fused(const uint32_t *packed, const float *gamma,
     a.rowsum_out = rowsum;
     a.Y = Y;
     a.static_weights = static_weights ? 1 : 0;
-    return launch_decode(a, true, out_dtype, stream);
+    return launch_decode(a, true, out_dtype, base3, stream);
 }
 
 }  // namespace bl

@@ -98,6 +98,48 @@ pack_kernel(const float *__restrict__ W, int64_t d_out, int64_t d_in, float eps,
     }
 }
 
+// Base-3 format (section 4 of the same page, "Memory Bandwidth and Latency
+// Bounds": five ternary values per byte, 3^5 = 243 < 256).  Tiles of 16 rows
+// x 160 columns (512 bytes), rows padded with W~ = 0; byte B of a tile row
+// covers the 20-column group g = B / 4 and, with j = B % 4, holds the codes
+// c_i = W~ + 1 of columns 20 g + 4 i + j as sum_i c_i 3^i.  The repacker
+// reads the 2-bit tiles, so the conversion is exact; one thread per 32-bit
+// word (one 20-column group of one row).  Offline, like the packer.
+__global__ void __launch_bounds__(256)
+repack_base3_kernel(const uint32_t *__restrict__ packed, int64_t d_out, int64_t d_in,
+                    uint32_t *__restrict__ packed3) {
+    const int64_t tiles2 = d_in >> 8;
+    const int64_t tiles3 = (d_in + 159) / 160;
+    const int64_t nwords = d_out * tiles3 * 8;        // 16 rows x 8 words per tile
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < nwords;
+         wi += stride) {
+        const int64_t tile = wi >> 7;
+        const int within = (int)(wi & 127);
+        const int r = within >> 3, g = within & 7;
+        const int64_t rb = tile / tiles3, kb = tile - rb * tiles3;
+        const int64_t k0 = kb * 160 + g * 20;
+        uint32_t word = 0;
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t b = 0;
+            #pragma unroll
+            for (int i = 4; i >= 0; --i) {            // Horner, highest digit first
+                const int64_t k = k0 + 4 * i + j;
+                uint32_t c = 1;                       // padding: W~ = 0
+                if (k < d_in) {
+                    const int64_t w2 =
+                        ((rb * tiles2 + (k >> 8)) * 16 + r) * 16 + ((k & 255) >> 4);
+                    c = (__ldg(packed + w2) >> (8 * (k & 3) + 2 * ((k & 15) >> 2))) & 3u;
+                }
+                b = b * 3u + c;
+            }
+            word |= b << (8 * j);
+        }
+        packed3[wi] = word;
+    }
+}
+
 }  // namespace bl
 
 using namespace bl;
@@ -230,5 +272,25 @@ extern "C" int bitlinear_pack_weights_noalloc(const float *W, int64_t d_out, int
     if (pblocks > 148 * 16) pblocks = 148 * 16;
     pack_kernel<<<(int)pblocks, 256, 0, stream>>>(W, d_out, d_in, eps, gamma_out, packed,
                                                   gamma_out);
+    return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+extern "C" size_t bitlinear_base3_bytes(int64_t d_out, int64_t d_in) {
+    if (bitlinear_packed_words(d_out, d_in) == 0) return 0;
+    return (size_t)(d_out * ((d_in + 159) / 160) * 32);
+}
+
+extern "C" int bitlinear_repack_base3(const uint32_t *packed, int64_t d_out, int64_t d_in,
+                                      uint8_t *packed3, cudaStream_t stream) {
+    if (bitlinear_packed_words(d_out, d_in) == 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (!packed || !packed3) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(packed, 16) || !aligned(packed3, 16)) return BITLINEAR_ERR_MISALIGNED;
+    bitlinear_status st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    const int64_t nwords = (int64_t)(bitlinear_base3_bytes(d_out, d_in) / 4);
+    int64_t blocks = (nwords + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    repack_base3_kernel<<<(int)blocks, 256, 0, stream>>>(packed, d_out, d_in,
+                                                          reinterpret_cast<uint32_t *>(packed3));
     return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }

@@ -96,6 +96,35 @@ def test_forward_validation(lib):
     assert _fwd(lib, T=0, xq=0, beta=0, rowsum=0) == bl.OK
 
 
+def test_base3_sizes_and_validation(lib):
+    """Five codes per byte on rows padded to 160 columns; base-3 entry points
+    take 1 <= T <= 16 and validate like their 2-bit counterparts."""
+    assert bl.base3_bytes(6912, 2560) == 6912 * 2560 // 5          # 2560 = 16 x 160
+    assert bl.base3_bytes(28672, 8192) == 28672 * 8320 // 5        # 8192 -> 8320 columns
+    assert bl.base3_bytes(16, 256) == 16 * 320 // 5
+    assert bl.base3_bytes(15, 256) == 0 and bl.base3_bytes(16, 128) == 0
+    f = lib.bitlinear_forward_base3
+
+    def fwd(T=4, packed=0x10000, d_in=256, xq=0x30000):
+        return f(P(packed), P(0x20000), 64, d_in, P(xq), P(0x40000), P(0x50000), T, P(0x60000),
+                 0, None, S0)
+
+    assert fwd(T=17) == bl.ERR_UNSUPPORTED_SHAPE
+    assert fwd(d_in=200) == bl.ERR_UNSUPPORTED_SHAPE
+    assert fwd(packed=0) == bl.ERR_INVALID_ARG
+    assert fwd(packed=0x10008) == bl.ERR_MISALIGNED
+    assert fwd(T=0, xq=0) == bl.OK
+    lin = lib.bitlinear_linear_base3
+    assert lin(P(0x10000), P(0x20000), 64, 256, P(0x30000), 17, None, 1, 1e-5, 1e-5,
+               P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0) == bl.ERR_UNSUPPORTED_SHAPE
+    assert lin(P(0x10000), P(0x20000), 64, 256, P(0x30000), 4, None, 8, 1e-5, 1e-5,
+               P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0) == bl.ERR_INVALID_ARG
+    rp = lib.bitlinear_repack_base3
+    assert rp(P(0x10000), 16, 128, P(0x20000), S0) == bl.ERR_UNSUPPORTED_SHAPE
+    assert rp(P(0x10000), 16, 256, None, S0) == bl.ERR_INVALID_ARG
+    assert rp(P(0x10000), 16, 256, P(0x20008), S0) == bl.ERR_MISALIGNED
+
+
 def test_quant_act_validation(lib):
     q = lib.bitlinear_quant_act
     args = dict(X=0x10000, T=2, d_in=512, gain=None, flags=1, eps=1e-5, neps=1e-5, rms=None,
