@@ -196,14 +196,15 @@ def fused(p: Problem) -> bool:
     return p.tokens <= 8 and p.tokens * p.d_in <= FUSED_MAX_CODE_BYTES
 
 
-def decode_bytes(p: Problem, out_bytes: int = 2) -> dict:
+def decode_bytes(p: Problem, out_bytes: int = 2, base3: bool = False) -> dict:
     """Algorithmic bytes of one decode BitLinear forward (quantise + product).
 
     Fused (one kernel): packed W + bf16 X read + codes, beta, row sums written
     once + gamma + Y.  Two kernels: the codes, beta and row sums are also read
-    back once by the product."""
+    back once by the product.  base3: five codes per byte on rows padded to
+    160 columns instead of four per byte."""
     T, K, N = p.tokens, p.d_in, p.d_out
-    w = N * K // 4                   # packed 2-bit weights
+    w = N * ((K + 159) // 160 * 160) // 5 if base3 else N * K // 4
     x = T * K * 2                    # bf16 activations
     inter = T * K + 8 * T            # codes, beta, row sums written
     y = T * N * out_bytes
@@ -272,9 +273,10 @@ def profile_traffic(summary_name: str, source):
 class DecodeRun:
     """`layers` forwards per step over distinct packed weight copies."""
 
-    def __init__(self, problems, layers, dev, out_dtype=torch.bfloat16):
+    def __init__(self, problems, layers, dev, out_dtype=torch.bfloat16, base3=False):
         import ternary_weight_linear_bitlinear_b200 as bl
         self.bl = bl
+        self.base3 = base3
         self.problems = problems
         self.dev = dev
         self.out_dtype = out_dtype
@@ -283,6 +285,8 @@ class DecodeRun:
         for p in problems:
             W, X = draw(p)
             w = bl.pack_weights(W.to(dev), EPS)
+            if base3:
+                w = bl.repack_base3(w)
             base.append((p, w, X.to(dev)))
             del W
         reps = max(1, layers // len(problems))
@@ -291,7 +295,7 @@ class DecodeRun:
                 if r == 0:
                     w = w0
                 else:
-                    w = bl.PackedTernary(w0.packed.clone(), w0.gamma.clone(), w0.d_out, w0.d_in)
+                    w = type(w0)(w0.packed.clone(), w0.gamma.clone(), w0.d_out, w0.d_in)
                 T = p.tokens
                 scratch = (torch.empty((T, p.d_in), dtype=torch.int8, device=dev),
                            torch.empty(T, dtype=torch.float32, device=dev),
@@ -319,12 +323,12 @@ class DecodeRun:
         ob = 2 if self.out_dtype == torch.bfloat16 else 4
         tot = dict(step=0, gemv=0, weights=0, weights_and_acts=0)
         for p, *_ in self.layers:
-            for k, v in decode_bytes(p, ob).items():
+            for k, v in decode_bytes(p, ob, self.base3).items():
                 tot[k] += v
         return tot
 
     def weight_bytes_resident(self):
-        return sum(w.packed.numel() * 4 for _, w, *_ in self.layers)
+        return sum(w.packed.numel() * w.packed.element_size() for _, w, *_ in self.layers)
 
 
 def run_decode(name, steps, warmup, dev, layers, world):
@@ -355,6 +359,46 @@ def measure_product_only(run, steps):
     ms = time_graph(g)
     launches = steps * len(run.layers)
     return ms / launches, launches
+
+
+def measure_base3(dev, peaks, reps=5):
+    """The base-3 weight format (five codes per byte) against the 2-bit one on
+    the decode workloads, each over distinct weight copies of at least 4x the
+    L2: microseconds per forward of the whole fused forward and of the product
+    alone (codes precomputed), and the GB/s of each format's own bytes."""
+    out = {}
+    for name in ("decode_gemv_2560x6912_t1", "decode_block_4096_t1",
+                 "large_gemv_8192x28672_t1", "large_gemv_8192x28672_t8"):
+        wl = WORKLOADS[name]
+        res = {}
+        for fmt in ("2bit", "base3"):
+            b3 = fmt == "base3"
+            per = sum(decode_bytes(p, base3=b3)["weights"] for p in wl.problems)
+            layers = max(len(wl.problems), int(np.ceil(4 * L2_BYTES / per)) * len(wl.problems))
+            r = DecodeRun(wl.problems, layers, dev, base3=b3)
+            g = capture(lambda: [r.step() for _ in range(reps)])
+            time_graph(g)
+            t = time_graph(g) / reps / len(r.layers)
+            gp = capture(lambda: [r.product_only() for _ in range(reps)])
+            time_graph(gp)
+            tp = time_graph(gp) / reps / len(r.layers)
+            b = r.bytes()
+            n = len(r.layers)
+            res[fmt] = {"us_per_forward": round(t * 1e3, 3),
+                        "gbs_forward": round(b["step"] / n / (t * 1e-3) / 1e9, 1),
+                        "us_product_only": round(tp * 1e3, 3),
+                        "gbs_product_only": round(b["gemv"] / n / (tp * 1e-3) / 1e9, 1),
+                        "frac_of_hbm_product_only": round(
+                            b["gemv"] / n / (tp * 1e-3) / 1e9 / peaks["hbm"], 4),
+                        "weight_bytes_per_forward": b["weights"] // n}
+            del r, g, gp
+            torch.cuda.empty_cache()
+        res["speedup_forward"] = round(res["2bit"]["us_per_forward"] /
+                                       res["base3"]["us_per_forward"], 3)
+        res["speedup_product_only"] = round(res["2bit"]["us_product_only"] /
+                                            res["base3"]["us_product_only"], 3)
+        out[name] = res
+    return out
 
 
 # ----------------------------------------------------- prefill workload ---
@@ -625,6 +669,8 @@ def main():
                     help="headline only (no prefill / other decode workloads)")
     ap.add_argument("--only-prefill", action="store_true",
                     help="time the prefill forward alone and print its JSON object")
+    ap.add_argument("--only-base3", action="store_true",
+                    help="time the base-3 and 2-bit decode formats alone, print their JSON")
     args = ap.parse_args()
     warmup = max(args.warmup, 3)
     rank, world, local = dist_init(args.gpus)
@@ -643,6 +689,15 @@ def main():
         res = measure_prefill(max(3, args.steps), warmup, dev, peaks)
         if rank == 0:
             print(json.dumps({"prefill": res}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            barrier(world)
+            dist.destroy_process_group()
+        return
+    if args.only_base3:
+        res = measure_base3(dev, peaks)
+        if rank == 0:
+            print(json.dumps({"base3": res}), flush=True)
         if world > 1:
             import torch.distributed as dist
             barrier(world)
@@ -706,6 +761,9 @@ def main():
             del r2, g2
             torch.cuda.empty_cache()
         extras["decode_other"] = other
+        sampler.mark(True)
+        extras["base3"] = measure_base3(dev, peaks)
+        sampler.mark(False)
         sampler.mark(True)
         extras["backward_ste"] = measure_backward(10, dev, peaks)
         extras["context_bf16"] = measure_context_bf16(
