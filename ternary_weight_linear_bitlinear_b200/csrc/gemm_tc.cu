@@ -14,25 +14,32 @@
 // CTA per SM walks the output tiles, and four roles run concurrently, each
 // 128-column step passing through two rings of shared memory:
 //   * warp 0 (one lane) TMA-loads the token tile X~[n0..n0+256)[k..k+128)
-//     (128-byte swizzled, K-major) and the packed 2-bit codes of the 128
-//     weight rows (4 KiB) into the token ring, signalling `full`;
-//   * warps 2..5 (one thread per weight row) expand their row's eight packed
-//     words into 128 int8 codes and store them into the weight ring in the
-//     same 128-byte swizzled K-major layout the TMA gives the tokens, then
-//     signal `afull`;
-//   * warp 1 (one lane) issues four tcgen05.mma.kind::i8 (K = 32 each) with
-//     both operands read from shared memory into one of two TMEM
-//     accumulators, and commits to `empty` (token stage free) and `aempty`
-//     (weight slot free); after a tile's last step it commits to `acc_full`;
+//     (128-byte swizzled, K-major) into the token ring, signalling `full`,
+//     and, five steps ahead, the packed 2-bit codes of the 128 weight rows
+//     (4 KiB) into a separate packed ring, signalling `pfull`;
+//   * warps 2..5 (one thread per weight row) read their row's eight packed
+//     words from the packed ring, expand them into 128 int8 codes and store
+//     those into the weight ring in the same 128-byte swizzled K-major
+//     layout the TMA gives the tokens, then signal `afull` (and `pempty`);
+//   * warp 1 (one lane) waits for both operands of a step, issues four
+//     tcgen05.mma.kind::i8 (K = 32 each) with both operands read from shared
+//     memory into one of two TMEM accumulators, and commits to `empty`
+//     (token stage free) and `aempty` (weight slot free); after a tile's
+//     last step it commits to `acc_full`;
 //   * warps 6..9 read a finished accumulator (tcgen05.ld), subtract each
 //     token's code sum, apply gamma beta / 127, stage 32-row x 8-token
 //     blocks in shared memory and write them with TMA tensor stores, then
 //     hand the accumulator back (`acc_empty`) -- while the MMA already fills
 //     the other accumulator with the next tile.
 // Each expanded weight code feeds 256 tokens of MMA work, so the expansion
-// is a small share of the issue slots.  The token ring is four deep (three
-// measured 8 % slower, five no faster); two weight slots suffice because the
-// expanders run just ahead of the MMA.  Tensor
+// is a small share of the issue slots.  A step's critical loop is: MMA
+// completion frees a token stage -> its next TMA (~1200 cycles under load)
+// -> the MMA issue, which four token stages cover.  The expansion runs off
+// that loop: its packed words arrive steps early in their own ring (the
+// expanders never wait for a token stage), and three weight slots let it
+// run ahead of the MMA.  (Loading the packed words with per-thread global
+// loads instead was slower: the proxy fence each expander thread needs
+// before signalling `afull` also waits for its loads in flight.)  Tensor
 // memory holds only the two 256-column accumulators (512 columns).  Waiting
 // threads sleep in mbarrier.try_wait.  Every wait is bounded (see common.cuh); on expiry the
 // CTA stops issuing, waits for its own copies, MMAs and stores in flight,
@@ -52,10 +59,12 @@ constexpr int kBM = 128;          // weight rows per tile (MMA M = TMEM lanes)
 constexpr int kBN = 256;          // tokens per tile (MMA N)
 constexpr int kBK = 128;          // reduction columns per step (bytes)
 constexpr int kStages = 4;        // token ring
-constexpr int kASlots = 2;        // weight ring
+constexpr int kASlots = 3;        // weight ring
+constexpr int kPSlots = 8;        // packed ring
+constexpr int kPAhead = 5;        // steps the packed loads run ahead of the token loads
 constexpr int kBTile = kBN * kBK;            // 32 KiB token tile
-constexpr int kPTile = kBM * kBK / 4;        // 4 KiB packed tile
-constexpr int kStageBytes = kBTile + kPTile; // 36 KiB (a multiple of 1024)
+constexpr int kStageBytes = kBTile;          // a multiple of 1024
+constexpr int kPTile = kBM * kBK / 4;        // 4 KiB packed codes of a step
 constexpr int kATile = kBM * kBK;            // 16 KiB expanded weight codes
 constexpr int kAccCols = kBN;                // int32 columns of one accumulator
 constexpr int kAccBufs = 2;
@@ -77,6 +86,8 @@ struct __align__(8) GemmBarriers {
     uint64_t empty[kStages];
     uint64_t afull[kASlots];
     uint64_t aempty[kASlots];
+    uint64_t pfull[kPSlots];
+    uint64_t pempty[kPSlots];
     uint64_t acc_full[kAccBufs];
     uint64_t acc_empty[kAccBufs];
     uint64_t drain;
@@ -85,7 +96,8 @@ struct __align__(8) GemmBarriers {
     int epi_ok[4];      // per epilogue warp: its wait for the accumulator succeeded
 };
 static_assert(sizeof(GemmBarriers) <= 1024, "barrier block");
-constexpr int kSmemBytes = kStages * kStageBytes + kASlots * kATile + kOutBytes + kTokBytes +
+constexpr int kSmemBytes = kStages * kStageBytes + kASlots * kATile + kPSlots * kPTile +
+                           kOutBytes + kTokBytes +
                            1024 /* barriers */ + 1024 /* alignment slack */;
 
 template <bool OUT_BF16>
@@ -99,13 +111,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *a_ring = smem + kStages * kStageBytes;
-    uint8_t *out_stage = a_ring + kASlots * kATile;
+    uint8_t *p_ring = a_ring + kASlots * kATile;
+    uint8_t *out_stage = p_ring + kPSlots * kPTile;
     uint8_t *tok_stage = out_stage + kOutBytes;
     GemmBarriers *bars = reinterpret_cast<GemmBarriers *>(tok_stage + kTokBytes);
     const uint32_t smem_base = smem_u32(smem);
     const uint32_t a_base = smem_u32(a_ring);
     auto stage_x = [&](int s) { return smem_base + s * kStageBytes; };
-    auto stage_w = [&](int s) { return smem_base + s * kStageBytes + kBTile; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = (d_out + kBM - 1) / kBM;
@@ -121,6 +133,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         for (int s = 0; s < kASlots; ++s) {
             mbar_init(smem_u32(&bars->afull[s]), 4);
             mbar_init(smem_u32(&bars->aempty[s]), 1);
+        }
+        for (int s = 0; s < kPSlots; ++s) {
+            mbar_init(smem_u32(&bars->pfull[s]), 1);
+            mbar_init(smem_u32(&bars->pempty[s]), 4);
         }
         for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(smem_u32(&bars->acc_full[b]), 1);
@@ -144,12 +160,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer ---
+        // Steps are numbered over this CTA's tiles in order; step g is
+        // (tile blockIdx.x + (g / num_k) gridDim.x, kt = g mod num_k).  The
+        // packed codes of step g are issued with the tokens of g - kPAhead.
         if (lane == 0) {
+            const int my_tiles = blockIdx.x < num_tiles
+                                     ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
+                                     : 0;
+            const int total = my_tiles * num_k;
+            auto issue_packed = [&](int g) {
+                const int tile = (int)blockIdx.x + (g / num_k) * (int)gridDim.x;
+                const int kt = g - (g / num_k) * num_k;
+                const int m0 = (tile % m_tiles) * kBM;
+                const uint32_t pb = smem_u32(&bars->pfull[g % kPSlots]);
+                mbar_arrive_expect_tx(pb, kPTile);
+                tma_load_4d(smem_u32(p_ring + (g % kPSlots) * kPTile), &map_w, (kt & 1) * 8, 0,
+                            kt >> 1, m0 / 16, pb);
+            };
+            int p_issued = 0;
+            for (; p_issued < kPAhead && p_issued < total; ++p_issued) issue_packed(p_issued);
             int s = 0, step = 0;
             uint32_t ph = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m0 = (tile % m_tiles) * kBM, n0 = (tile / m_tiles) * kBN;
+                const int n0 = (tile / m_tiles) * kBN;
                 for (int kt = 0; kt < num_k; ++kt) {
                     if (step >= kStages &&
                         !wait_or_abort(smem_u32(&bars->empty[s]), ph ^ 1u, ctx, abort_flag)) {
@@ -159,22 +193,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                     const uint32_t fb = smem_u32(&bars->full[s]);
                     mbar_arrive_expect_tx(fb, kStageBytes);
                     tma_load_2d(stage_x(s), &map_x, kt * kBK, n0, fb);
-                    tma_load_4d(stage_w(s), &map_w, (kt & 1) * 8, 0, kt >> 1, m0 / 16, fb);
                     ++step;
                     if (++s == kStages) { s = 0; ph ^= 1u; }
+                    if (p_issued < total) {
+                        // The packed slot was last used by step p_issued - kPSlots.
+                        if (p_issued >= kPSlots &&
+                            !wait_or_abort(smem_u32(&bars->pempty[p_issued % kPSlots]),
+                                           (uint32_t)(p_issued / kPSlots - 1) & 1u, ctx,
+                                           abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        issue_packed(p_issued++);
+                    }
                 }
             }
             // Drain: every copy issued must land before the CTA may exit.
             for (int q = step > kStages ? step - kStages : 0; q < step; ++q)
                 mbar_wait_bounded(smem_u32(&bars->full[q % kStages]),
                                   (uint32_t)(q / kStages) & 1u, ctx);
+            for (int q = p_issued > kPSlots ? p_issued - kPSlots : 0; q < p_issued; ++q)
+                mbar_wait_bounded(smem_u32(&bars->pfull[q % kPSlots]),
+                                  (uint32_t)(q / kPSlots) & 1u, ctx);
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ---
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_i8(kBM, kBN);
             int s = 0, sa = 0, i = 0;
-            uint32_t pha = 0;
+            uint32_t ph = 0, pha = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++i) {
                 const int buf = i & 1, use = i >> 1;
@@ -184,10 +231,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 tc_fence_after();
                 const uint32_t tmem_acc = tmem_base + buf * kAccCols;
                 for (int kt = 0; kt < num_k; ++kt) {
-                    // `afull` completes only after every expander thread has seen
-                    // `full` (the step's copies landed) and written its codes, so
-                    // one wait orders both operands before the MMAs.
-                    if (!wait_or_abort(smem_u32(&bars->afull[sa]), pha, ctx, abort_flag)) {
+                    // Both operands of the step: the expanded weight codes and
+                    // the token tile.
+                    if (!wait_or_abort(smem_u32(&bars->afull[sa]), pha, ctx, abort_flag) ||
+                        !wait_or_abort(smem_u32(&bars->full[s]), ph, ctx, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -199,7 +246,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                                      (kt > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(smem_u32(&bars->empty[s]));
                     tc_commit(smem_u32(&bars->aempty[sa]));
-                    if (++s == kStages) s = 0;
+                    if (++s == kStages) { s = 0; ph ^= 1u; }
                     if (++sa == kASlots) { sa = 0; pha ^= 1u; }
                 }
                 if (ok) tc_commit(smem_u32(&bars->acc_full[buf]));
@@ -212,23 +259,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     } else if (warp < kFirstEpiWarp) {
         // ---------------------------------------------------- expander ---
         // Row m's eight words of a step sit contiguously (32 bytes) in the
-        // stage; word j holds columns 16 j .. 16 j + 15 of the step, with
-        // column 16 j + 4 s + b in bits 8 b + 2 s, so (word >> 2 s) &
+        // packed slot; word j holds columns 16 j .. 16 j + 15 of the step,
+        // with column 16 j + 4 s + b in bits 8 b + 2 s, so (word >> 2 s) &
         // 0x03030303 is the four codes of columns 16 j + 4 s + 0..3: word j
         // expands to the 16-byte chunk j of the row, which the 128-byte
         // swizzle places at chunk j ^ (m mod 8) of the row's 128 bytes.
         const int m = (warp & 3) * 32 + lane;   // weight row within the tile
         uint8_t *arow = a_ring + m * kBK;
-        int s = 0, sa = 0, step = 0;
-        uint32_t ph = 0, pha = 0;
+        int sa = 0, sp = 0, step = 0;
+        uint32_t pha = 0, php = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kt = 0; kt < num_k; ++kt) {
-                ok = wait_or_abort(smem_u32(&bars->full[s]), ph, ctx, abort_flag);
+                ok = wait_or_abort(smem_u32(&bars->pfull[sp]), php, ctx, abort_flag);
                 uint32_t w[8];
                 if (ok) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(
-                        smem + s * kStageBytes + kBTile + m * 32);
+                    const uint4 *src = reinterpret_cast<const uint4 *>(p_ring + sp * kPTile + m * 32);
                     const uint4 lo = src[0], hi = src[1];
                     w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
                     w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
@@ -250,10 +296,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 // The tensor cores read the codes through the async proxy.
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bars->afull[sa]));
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&bars->afull[sa]));
+                    mbar_arrive(smem_u32(&bars->pempty[sp]));   // packed words consumed
+                }
                 ++step;
-                if (++s == kStages) { s = 0; ph ^= 1u; }
                 if (++sa == kASlots) { sa = 0; pha ^= 1u; }
+                if (++sp == kPSlots) { sp = 0; php ^= 1u; }
             }
         }
     } else {
