@@ -85,11 +85,13 @@ __device__ __forceinline__ float inv_rms_from_ss(double ss, double inv_k, float 
 // 2^-24).  When that sum is not finite or below 2^-100 (huge or tiny inputs)
 // the squares are formed and added sequentially in double instead.
 __device__ __forceinline__ double sq_sum8(const float (&x)[8]) {
-    float p[8];
+    // fma(x1, x1, x0 * x0) is fl(p0 + p1) itself, since both squares are
+    // exact: the pairs of the tree cost one multiply and one fma.
+    float p[4];
     #pragma unroll
-    for (int j = 0; j < 8; ++j) p[j] = __fmul_rn(x[j], x[j]);
-    const float s = __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3])),
-                              __fadd_rn(__fadd_rn(p[4], p[5]), __fadd_rn(p[6], p[7])));
+    for (int j = 0; j < 4; ++j)
+        p[j] = __fmaf_rn(x[2 * j + 1], x[2 * j + 1], __fmul_rn(x[2 * j], x[2 * j]));
+    const float s = __fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3]));
     if (s >= 0x1p-100f && s <= 3.40282347e38f) return (double)s;
     double d = 0.0;
     #pragma unroll
@@ -102,15 +104,32 @@ __device__ __forceinline__ double warp_sum_f64(double v) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
+// Maximum over the warp of non-negative finite floats: their bit patterns
+// order as unsigned integers, so one integer reduction gives it exactly.
 __device__ __forceinline__ float warp_max_f32(float v) {
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(v)));
 }
 __device__ __forceinline__ int warp_sum_i32(int v) {
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
+    return __reduce_add_sync(0xffffffffu, v);
+}
+
+// The activation code floor(v + 0.5) as the bit pattern of the binary32
+// value 1.5 * 2^23 + code.  u = fl_rd(v + 0.5) keeps floor(v + 0.5) (see
+// round_half_up_int); adding 1.5 * 2^23 rounding down lands in [2^23, 2^24),
+// where the spacing is 1, exactly at 1.5 * 2^23 + floor(u).  The low byte is
+// then the code in two's complement, and the pattern minus kCodeBias is the
+// code itself.  Valid for |v| < 2^22; the quantiser's v never exceeds
+// 127.00001 in magnitude: |n| <= beta because beta is the absmax of the same
+// rounded products, and fl(127 / (beta + eps)) <= (127 / beta)(1 + 2^-24),
+// so floor(v + 0.5) already lies in [-127, 127] and the clip is a no-op.
+constexpr uint32_t kCodeBias = 0x4B400000u;   // bit pattern of 1.5 * 2^23
+__device__ __forceinline__ uint32_t code_bits(float v) {
+    return __float_as_uint(__fadd_rd(__fadd_rd(v, 0.5f), 12582912.0f));
+}
+// Low bytes of four code patterns, little-endian.
+__device__ __forceinline__ uint32_t pack_code_bytes(uint32_t b0, uint32_t b1, uint32_t b2,
+                                                    uint32_t b3) {
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
 // Statistics of tokens 0..T-1 (T <= TMAX) of X [T][K] (bf16 bits).  Threads
@@ -181,17 +200,16 @@ __device__ __forceinline__ uint2 codes8(const uint4 &v, bool rmsnorm, float r, f
                                         int *sum) {
     float x[8];
     unpack8(v, x);
-    uint32_t lo = 0, hi = 0;
+    uint32_t b[8];
     #pragma unroll
     for (int j = 0; j < 8; ++j) {
         float n = x[j];
         if (rmsnorm) n = __fmul_rn(n, r);
-        const int qi = min(max(round_half_up_int(__fmul_rn(n, scale)), -127), 127);
-        *sum += qi;
-        const uint32_t b = (uint32_t)(qi & 0xff);
-        if (j < 4) lo |= b << (8 * j); else hi |= b << (8 * (j - 4));
+        b[j] = code_bits(__fmul_rn(n, scale));
+        *sum += (int)(b[j] - kCodeBias);
     }
-    return make_uint2(lo, hi);
+    return make_uint2(pack_code_bytes(b[0], b[1], b[2], b[3]),
+                      pack_code_bytes(b[4], b[5], b[6], b[7]));
 }
 
 // Row loads: read-only global path, or plain loads when X was staged in
@@ -322,18 +340,17 @@ __device__ __forceinline__ void token_codes(const uint16_t *__restrict__ X, int 
                         #pragma unroll
                         for (int j = 0; j < 8; ++j) g[j] = __ldg(gain + 8 * v + j);
                     }
-                    uint32_t lo = 0, hi = 0;
+                    uint32_t bb[8];
                     #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         float n = x[j];
                         if (rmsnorm) n = __fmul_rn(n, r);
                         if (use_gain) n = __fmul_rn(n, g[j]);
-                        const int qi = min(max(round_half_up_int(__fmul_rn(n, scale)), -127), 127);
-                        sum += qi;
-                        const uint32_t bb = (uint32_t)(qi & 0xff);
-                        if (j < 4) lo |= bb << (8 * j); else hi |= bb << (8 * (j - 4));
+                        bb[j] = code_bits(__fmul_rn(n, scale));
+                        sum += (int)(bb[j] - kCodeBias);
                     }
-                    out[v] = make_uint2(lo, hi);
+                    out[v] = make_uint2(pack_code_bytes(bb[0], bb[1], bb[2], bb[3]),
+                                        pack_code_bytes(bb[4], bb[5], bb[6], bb[7]));
                 }
             }
         }
