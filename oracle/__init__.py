@@ -78,6 +78,19 @@ def _load():
         lib.oracle_pack_base3.restype = i32
         lib.oracle_unpack_base3.argtypes = [vp, i64, i64, vp]
         lib.oracle_unpack_base3.restype = i32
+        lib.oracle_binarize.argtypes = [vp, i64, vp]
+        lib.oracle_binarize.restype = None
+        lib.oracle_w1_cols.argtypes = [i64]
+        lib.oracle_w1_cols.restype = i64
+        lib.oracle_pack_w1.argtypes = [vp, i64, i64, vp]
+        lib.oracle_pack_w1.restype = i32
+        lib.oracle_unpack_w1.argtypes = [vp, i64, i64, vp]
+        lib.oracle_unpack_w1.restype = i32
+        lib.oracle_quant_act_bits.argtypes = [vp, i64, i64, vp, i32, i32, i32, f32, f32, vp,
+                                              vp, vp, vp, vp]
+        lib.oracle_quant_act_bits.restype = None
+        lib.oracle_rescale_bits.argtypes = [vp, i64, i64, f32, vp, i32, vp]
+        lib.oracle_rescale_bits.restype = None
         lib.oracle_inv_rms.argtypes = [vp, i64, f32]
         lib.oracle_inv_rms.restype = f32
         lib.oracle_quant_act.argtypes = [vp, i64, i64, vp, i32, i32, f32, f32, vp,
@@ -179,6 +192,43 @@ def unpack_row(packed, d_out: int, d_in: int, o: int) -> np.ndarray:
     return out
 
 
+def binarize(W) -> np.ndarray:
+    """W1 codes: +1 where W >= 0, -1 elsewhere (the sign code of [MF] section 1
+    read for the W1A4 regime)."""
+    W = _c(W, np.float32)
+    out = np.empty(W.shape, dtype=np.int8)
+    _load().oracle_binarize(_ptr(W), W.size, _ptr(out))
+    return out
+
+
+def w1_cols(d_in: int) -> int:
+    """Row width of the 1-bit format: d_in padded to a multiple of 512."""
+    return int(_load().oracle_w1_cols(d_in))
+
+
+def pack_w1(wq) -> np.ndarray:
+    """Binary codes [d_out][d_in] in {-1, +1} -> uint32 words, one bit per
+    weight, in 16 x 512 tiles."""
+    wq = _c(wq, np.int8)
+    n, k = wq.shape
+    out = np.empty(n * w1_cols(k) // 32 if (n % 16 == 0 and k >= 1) else 0, dtype=np.uint32)
+    rc = _load().oracle_pack_w1(_ptr(wq), n, k, _ptr(out) if out.size else None)
+    if rc != 0:
+        raise ValueError("oracle_pack_w1: d_out not a multiple of 16, or a code not +-1")
+    return out
+
+
+def unpack_w1(packed, d_out: int, d_in: int) -> np.ndarray:
+    packed = _c(packed, np.uint32)
+    if d_out % 16 or d_in < 1 or packed.size != d_out * w1_cols(d_in) // 32:
+        raise ValueError("unpack_w1: size does not match the shape")
+    out = np.empty((d_out, d_in), dtype=np.int8)
+    rc = _load().oracle_unpack_w1(_ptr(packed), d_out, d_in, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_unpack_w1: a padding bit is set")
+    return out
+
+
 def base3_cols(d_in: int) -> int:
     """Row width of the base-3 format: d_in padded to a multiple of 160."""
     return int(_load().oracle_base3_cols(d_in))
@@ -217,13 +267,16 @@ def inv_rms(x_bf16_bits, norm_eps: float = 1e-5) -> float:
 
 
 def quant_act(X_bf16_bits, gain=None, rmsnorm: bool = True, eps: float = 1e-5,
-              norm_eps: float = 1e-5, inv_rms_in=None, per_tensor: bool = False):
-    """Absmax int8 quantisation, per token (or per tensor), optional RMSNorm
-    first ([MF] §2).
+              norm_eps: float = 1e-5, inv_rms_in=None, per_tensor: bool = False,
+              act_bits: int = 8):
+    """Absmax quantisation to act_bits-bit codes (8: [-127, 127]; 4: [-7, 7]),
+    per token (or per tensor), optional RMSNorm first ([MF] §2).
 
     Returns (xq int8 [T][K], beta f32 [T], rowsum int32 [T], inv_rms f32 [T]);
     with per_tensor every beta[t] is the one absmax of the whole X.
     """
+    if act_bits not in (4, 8):
+        raise ValueError("act_bits must be 4 or 8")
     X = _c(X_bf16_bits, np.uint16)
     T, K = X.shape
     g = None if gain is None else _c(gain, np.float32)
@@ -232,9 +285,9 @@ def quant_act(X_bf16_bits, gain=None, rmsnorm: bool = True, eps: float = 1e-5,
     beta = np.empty(T, dtype=np.float32)
     rowsum = np.empty(T, dtype=np.int32)
     rms_out = np.empty(T, dtype=np.float32)
-    _load().oracle_quant_act(_ptr(X), T, K, _ptr(g), int(bool(rmsnorm)),
-                             int(bool(per_tensor)), eps, norm_eps, _ptr(r_in), _ptr(xq),
-                             _ptr(beta), _ptr(rowsum), _ptr(rms_out))
+    _load().oracle_quant_act_bits(_ptr(X), T, K, _ptr(g), int(bool(rmsnorm)),
+                                  int(bool(per_tensor)), act_bits, eps, norm_eps, _ptr(r_in),
+                                  _ptr(xq), _ptr(beta), _ptr(rowsum), _ptr(rms_out))
     return xq, beta, rowsum, rms_out
 
 
@@ -258,13 +311,14 @@ def dot_masked_add(wrow, xrow) -> int:
     return int(_load().oracle_dot_masked_add(_ptr(w), _ptr(x), w.size))
 
 
-def rescale(acc, gamma: float, beta) -> np.ndarray:
-    """Y = acc * beta * gamma / (Q_b - 1), in float64 ([MF] §2)."""
+def rescale(acc, gamma: float, beta, act_bits: int = 8) -> np.ndarray:
+    """Y = acc * beta * gamma / (Q_b - 1), Q_b = 2^(act_bits - 1), in float64
+    ([MF] §2)."""
     acc = _c(acc, np.int32)
     beta = _c(beta, np.float32)
     T, N = acc.shape
     y = np.empty((T, N), dtype=np.float64)
-    _load().oracle_rescale(_ptr(acc), T, N, gamma, _ptr(beta), _ptr(y))
+    _load().oracle_rescale_bits(_ptr(acc), T, N, gamma, _ptr(beta), act_bits, _ptr(y))
     return y
 
 

@@ -262,6 +262,81 @@ int oracle_unpack_base3(const uint8_t *packed, int64_t n_out, int64_t n_in, int8
     return 0;
 }
 
+/* ----------------------------------------- binary weights (W1A4, [EoMM]) */
+
+/* W1: the binary alphabet {-1, +1} of [MF] section 1 (BitNet b1), used by the
+ * W1A4 regime that "The End of Matrix Multiplications: Welcome to Addition"
+ * names (1-bit weights, 4-bit activations).  The pages give no binarisation
+ * rule; the reading taken: W~ = +1 where W >= 0 and -1 elsewhere (so +0 and
+ * -0 both map to +1), scaled by the same absmean gamma as the ternary layer,
+ * which is the least-squares scale of a sign code: d/da sum (W - a sign W)^2
+ * = 0 at a = mean |W|. */
+void oracle_binarize(const float *W, int64_t count, int8_t *wq)
+{
+    for (int64_t i = 0; i < count; ++i) wq[i] = (int8_t)(W[i] >= 0.0f ? 1 : -1);
+}
+
+/* This library's 1-bit format: rows padded with W~ = -1 to a multiple of 512
+ * columns; tiles of 16 rows x 512 columns (1 KiB), tile-row-major; each tile
+ * row is 16 little-endian 32-bit words; word kw covers columns 32 kw .. 32 kw
+ * + 31, and the bit c = (W~ + 1) / 2 of column 32 kw + 4 s + j sits at bit
+ * 8 j + s.  So (word >> s) & 0x01010101 is the four bits of four consecutive
+ * columns. */
+int64_t oracle_w1_cols(int64_t n_in)
+{
+    return (n_in + 511) / 512 * 512;
+}
+
+static void w1_position(int64_t n_in, int64_t o, int64_t k, int64_t *word, int *bit)
+{
+    int64_t tiles_per_row = oracle_w1_cols(n_in) / 512;
+    int64_t rb = o / 16, r = o % 16;
+    int64_t kb = k / 512, kw = (k % 512) / 32;
+    int s = (int)((k % 32) / 4), j = (int)(k % 4);
+    *word = ((rb * tiles_per_row + kb) * 16 + r) * 16 + kw;
+    *bit = 8 * j + s;
+}
+
+/* Returns 0, or -1 if d_out is not a multiple of 16, d_in < 1 or a code is
+ * not -1 or +1.  packed holds d_out * padded width / 32 words. */
+int oracle_pack_w1(const int8_t *wq, int64_t n_out, int64_t n_in, uint32_t *packed)
+{
+    if (n_out % 16 != 0 || n_in < 1) return -1;
+    const int64_t kp = oracle_w1_cols(n_in);
+    memset(packed, 0, (size_t)(n_out * kp / 32) * sizeof(uint32_t));
+    for (int64_t o = 0; o < n_out; ++o) {
+        for (int64_t k = 0; k < n_in; ++k) {
+            int v = wq[o * n_in + k];
+            if (v != -1 && v != 1) return -1;
+            int64_t word;
+            int bit;
+            w1_position(n_in, o, k, &word, &bit);
+            if (v == 1) packed[word] |= 1u << bit;
+        }
+    }
+    return 0;
+}
+
+/* Inverse of oracle_pack_w1.  Returns -1 if a padding bit is set. */
+int oracle_unpack_w1(const uint32_t *packed, int64_t n_out, int64_t n_in, int8_t *wq)
+{
+    if (n_out % 16 != 0 || n_in < 1) return -1;
+    const int64_t kp = oracle_w1_cols(n_in);
+    for (int64_t o = 0; o < n_out; ++o) {
+        for (int64_t k = 0; k < kp; ++k) {
+            int64_t word;
+            int bit;
+            w1_position(n_in, o, k, &word, &bit);
+            int c = (int)((packed[word] >> bit) & 1u);
+            if (k < n_in)
+                wq[o * n_in + k] = (int8_t)(2 * c - 1);
+            else if (c)
+                return -1;
+        }
+    }
+    return 0;
+}
+
 /* ---------------------------------------- activation quantisation ([MF] §2) */
 
 /* Reciprocal RMS of one token: 1 / sqrt(mean(x^2) + norm_eps), carried in
@@ -305,11 +380,14 @@ static float normalised(const uint16_t *x, int64_t k, int rmsnorm, float r, cons
  * computing it (used to compare integer codes against a GPU that computed
  * its own).  beta[t] receives the beta token t was quantised with.
  */
-void oracle_quant_act(const uint16_t *X, int64_t T, int64_t K, const float *gain,
-                      int rmsnorm, int per_tensor, float eps, float norm_eps,
-                      const float *inv_rms_in, int8_t *xq, float *beta, int32_t *rowsum,
-                      float *inv_rms_out)
+void oracle_quant_act_bits(const uint16_t *X, int64_t T, int64_t K, const float *gain,
+                           int rmsnorm, int per_tensor, int act_bits, float eps,
+                           float norm_eps, const float *inv_rms_in, int8_t *xq, float *beta,
+                           int32_t *rowsum, float *inv_rms_out)
 {
+    /* Q_b = 2^(k-1) levels for k-bit activations ([MF] section 2); the
+     * multiplier and the clip bound are Q_b - 1. */
+    const int qmax = (1 << (act_bits - 1)) - 1;
     /* Statistics of every token first. */
     for (int64_t t = 0; t < T; ++t) {
         const uint16_t *x = X + t * K;
@@ -336,17 +414,26 @@ void oracle_quant_act(const uint16_t *X, int64_t T, int64_t K, const float *gain
         float r = 1.0f;
         if (rmsnorm)
             r = inv_rms_in ? inv_rms_in[t] : oracle_inv_rms(x, K, norm_eps);
-        float scale = (float)ORACLE_QB_MINUS_1 / (beta[t] + eps);
+        float scale = (float)qmax / (beta[t] + eps);
         int32_t S = 0;
         for (int64_t k = 0; k < K; ++k) {
             float v = normalised(x, k, rmsnorm, r, gain) * scale;
-            int q = (int)round_clip_f32(v, -(float)ORACLE_QB_MINUS_1,
-                                        (float)ORACLE_QB_MINUS_1);
+            int q = (int)round_clip_f32(v, -(float)qmax, (float)qmax);
             xq[t * K + k] = (int8_t)q;
             S += q;
         }
         rowsum[t] = S;
     }
+}
+
+/* The int8 quantiser of [MF] section 2: 8-bit activations, Q_b - 1 = 127. */
+void oracle_quant_act(const uint16_t *X, int64_t T, int64_t K, const float *gain,
+                      int rmsnorm, int per_tensor, float eps, float norm_eps,
+                      const float *inv_rms_in, int8_t *xq, float *beta, int32_t *rowsum,
+                      float *inv_rms_out)
+{
+    oracle_quant_act_bits(X, T, K, gain, rmsnorm, per_tensor, 8, eps, norm_eps, inv_rms_in, xq,
+                          beta, rowsum, inv_rms_out);
 }
 
 /* ---------------------------------- product and rescale ([MF] §2 and §6) */
@@ -381,14 +468,21 @@ int32_t oracle_dot_masked_add(const int8_t *wrow, const int8_t *xrow, int64_t K)
 }
 
 /* Y = (X~ W~^T) * beta * gamma / (Q_b - 1), in double ([MF] §2). */
-void oracle_rescale(const int32_t *acc, int64_t T, int64_t N, float gamma,
-                    const float *beta, double *y)
+void oracle_rescale_bits(const int32_t *acc, int64_t T, int64_t N, float gamma,
+                         const float *beta, int act_bits, double *y)
 {
+    const double qmax = (double)((1 << (act_bits - 1)) - 1);
     for (int64_t t = 0; t < T; ++t) {
-        double scale = (double)beta[t] * (double)gamma / (double)ORACLE_QB_MINUS_1;
+        double scale = (double)beta[t] * (double)gamma / qmax;
         for (int64_t o = 0; o < N; ++o)
             y[t * N + o] = (double)acc[t * N + o] * scale;
     }
+}
+
+void oracle_rescale(const int32_t *acc, int64_t T, int64_t N, float gamma,
+                    const float *beta, double *y)
+{
+    oracle_rescale_bits(acc, T, N, gamma, beta, 8, y);
 }
 
 /*

@@ -244,6 +244,120 @@ def test_base3_rejects_bad_input():
         oracle.unpack_base3(pad, 16, 256)
 
 
+# ------------------------------------------------------- W1A4 (binary) ---
+
+def test_binarize_signs():
+    """Sign code of the W1 regime: +1 for W >= 0 (both zeros), -1 below."""
+    W = np.array([0.0, -0.0, 1e-38, -1e-38, 3.5, -2.0, 1e-45, -1e-45], np.float32)
+    np.testing.assert_array_equal(oracle.binarize(W), [1, 1, 1, -1, 1, -1, 1, -1])
+    G = (RNG.standard_normal(100000) * 0.02).astype(np.float32)
+    b = oracle.binarize(G)
+    assert set(np.unique(b)) == {-1, 1}
+    assert abs((b == 1).mean() - 0.5) < 0.01                # symmetric distribution
+
+
+def test_absmean_is_least_squares_scale_of_sign_code():
+    """The absmean gamma minimises sum (W - a sign W)^2 over a: the derivative
+    sum |W| - N a vanishes at a = gamma, and nearby scales fit worse."""
+    W = (RNG.standard_normal((64, 512)) * 0.02).astype(np.float32)
+    g = oracle.absmean_gamma(W)
+    s = oracle.binarize(W).astype(np.float64)
+    w = W.astype(np.float64)
+    f = lambda a: float(((w - a * s) ** 2).sum())
+    assert abs(float((s * (w - g * s)).sum())) <= 1e-6 * float(np.abs(w).sum())
+    assert f(g) < f(g * 1.01) and f(g) < f(g * 0.99)
+
+
+def test_w1_layout_golden(golden_dir):
+    ex = json.load(open(os.path.join(golden_dir, "w1_layout.json")))
+    n, k = ex["d_out"], ex["d_in"]
+    zero = oracle.pack_w1(np.full((n, k), -1, np.int8))
+    assert zero.size == ex["words"] and not zero.any()
+    for c in ex["cases"]:
+        wq = np.full((n, k), -1, np.int8)
+        wq[c["o"], c["k"]] = 1
+        p = oracle.pack_w1(wq)
+        expect = np.zeros(p.shape, dtype=np.uint32)
+        expect[c["word"]] = int(c["value"], 16)
+        np.testing.assert_array_equal(p, expect, err_msg=str(c))
+
+
+@pytest.mark.parametrize("shape", [(16, 256), (32, 512), (48, 2560), (16, 4096), (32, 11008)])
+def test_w1_roundtrip_and_size(shape):
+    wq = (RNG.integers(0, 2, size=shape) * 2 - 1).astype(np.int8)
+    p = oracle.pack_w1(wq)
+    kp = -(-shape[1] // 512) * 512
+    assert oracle.w1_cols(shape[1]) == kp
+    assert p.size == shape[0] * kp // 32                 # one bit per padded weight
+    np.testing.assert_array_equal(oracle.unpack_w1(p, *shape), wq)
+    # The number of +1 codes survives packing.
+    ones = sum(bin(int(v)).count("1") for v in p)
+    assert ones == int((wq == 1).sum())
+    if shape[1] % 512 == 0:                               # no padding: every bit set
+        assert (oracle.pack_w1(np.ones(shape, np.int8)) == 0xFFFFFFFF).all()
+
+
+def test_w1_is_a_bijection_on_a_tile():
+    seen = set()
+    for o in range(16):
+        for k in range(512):
+            wq = np.full((16, 512), -1, np.int8)
+            wq[o, k] = 1
+            p = oracle.pack_w1(wq)
+            nz = np.flatnonzero(p)
+            assert nz.size == 1 and bin(int(p[nz[0]])).count("1") == 1
+            seen.add((int(nz[0]), int(p[nz[0]]).bit_length() - 1))
+    assert len(seen) == 16 * 512
+
+
+def test_w1_rejects_bad_input():
+    with pytest.raises(ValueError):
+        oracle.pack_w1(np.zeros((16, 512), np.int8))          # 0 is not a binary code
+    pad = oracle.pack_w1(np.full((16, 256), -1, np.int8))
+    pad[15] = 1                                               # column 480: padding
+    with pytest.raises(ValueError):
+        oracle.unpack_w1(pad, 16, 256)
+
+
+def test_quant_act_4bit():
+    """A4: Q_b = 2^3 levels, codes in [-7, 7], the absmax element of a token at
+    +-7, q the integer nearest to v = fl32(n * fl32(7 / (beta + eps))) with ties
+    upward; act_bits = 8 is the default quantiser."""
+    X = draw(Problem("a4", 512, 16, 5, 0.02, 0.01, 50.0, 4))[1]
+    bits = bf16_bits(X)
+    xq, beta, rowsum, r = oracle.quant_act(bits, act_bits=4)
+    assert xq.min() >= -7 and xq.max() <= 7
+    np.testing.assert_array_equal(rowsum, xq.astype(np.int64).sum(axis=1))
+    xf = X.float().numpy()
+    for t in range(5):
+        n = xf[t] * np.float32(r[t])
+        assert abs(int(xq[t][np.argmax(np.abs(n))])) == 7
+        s = np.float32(7.0) / (np.float32(beta[t]) + np.float32(1e-5))
+        v = (n * s).astype(np.float64)
+        cand = np.stack([np.floor(v), np.floor(v) + 1])
+        d = np.abs(v[None] - cand)
+        q = np.where(d[1] <= d[0], cand[1], cand[0])
+        np.testing.assert_array_equal(xq[t], np.clip(q, -7, 7).astype(np.int8))
+    q8 = oracle.quant_act(bits, act_bits=8)
+    q0 = oracle.quant_act(bits)
+    for a, b in zip(q8, q0):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_w1a4_forward_against_dequantised_product():
+    """Y = (X~ W~^T) beta gamma / 7 equals the fp64 product of the dequantised
+    operands (X~ beta / 7) and (gamma W~)."""
+    W, X = draw(Problem("w1a4", 256, 16, 3, 0.02, 0.01, 50.0, 7))
+    Wn = W.numpy()
+    g = oracle.absmean_gamma(Wn)
+    wq = oracle.binarize(Wn)
+    xq, beta, _, _ = oracle.quant_act(bf16_bits(X), act_bits=4)
+    y = oracle.rescale(oracle.int_matmul(wq, xq), g, beta, act_bits=4)
+    ref = (xq.astype(np.float64) * beta.astype(np.float64)[:, None] / 7.0) @ \
+          (float(g) * wq.astype(np.float64)).T
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-15)
+
+
 def test_pack_exhaustive_groups():
     """All 81 joint values of the four codes that share one byte (same s)
     and of the four that share one 2-bit slot across bytes (same j)."""
