@@ -87,6 +87,13 @@ typedef enum {
  * this mode. */
 #define BITLINEAR_PER_TENSOR_ABSMAX 4u
 
+/* Flag of bitlinear_quant_act and bitlinear_linear_w1: 4-bit activation codes,
+ * the A4 of the W1A4 regime ("The End of Matrix Multiplications: Welcome to
+ * Addition", Technical Details).  [MF] section 2 defines Q_b = 2^(k-1) for
+ * k-bit activations; with k = 4 the multiplier and the clip bound are
+ * Q_b - 1 = 7, codes in [-7, 7] (still stored one per int8). */
+#define BITLINEAR_ACT_4BIT 8u
+
 /* Library ABI version (this header: 1). */
 int bitlinear_version(void);
 
@@ -165,7 +172,10 @@ int bitlinear_pack_weights_noalloc(const float *W, int64_t d_out, int64_t d_in,
  *
  *   X          bf16 [T][d_in], row-major, as raw uint16 bit patterns.
  *   norm_gain  fp32 [d_in] RMSNorm gain, or NULL for all ones.
- *   flags      BITLINEAR_RMSNORM to normalise first, 0 to quantise X as is.
+ *   flags      BITLINEAR_RMSNORM to normalise first, 0 to quantise X as is;
+ *              BITLINEAR_PER_TENSOR_ABSMAX for one beta over all of X;
+ *              BITLINEAR_ACT_4BIT for 4-bit codes (multiplier and clip 7
+ *              instead of 127).
  *   eps        the epsilon of 127 / (beta + eps); finite, >= 0.
  *   norm_eps   the epsilon inside the RMS; finite, >= 0.  The reciprocal RMS
  *              r = 1 / sqrt(mean(x^2) + norm_eps): sum of squares in double in
@@ -287,6 +297,65 @@ int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma, int64_t d
                            const float *norm_gain, uint32_t flags, float eps,
                            float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
                            void *Y, int out_dtype, cudaStream_t stream);
+
+/*
+ * W1A4: binary weights with 4-bit activations, the regime "The End of Matrix
+ * Multiplications: Welcome to Addition" names (Technical Details).  The pages
+ * give no binarisation rule; this library takes the binary alphabet
+ * {-1, +1} of [MF] section 1 as W~ = +1 where W >= 0 and -1 elsewhere, with
+ * the same absmean gamma as scale (the least-squares scale of a sign code),
+ * and the A4 codes of BITLINEAR_ACT_4BIT:
+ *
+ *   Y = (X~ W~^T) * beta * gamma / (Q_b - 1),  Q_b - 1 = 7 (4-bit) or 127
+ *
+ * 1-bit weight format (this library's own): rows padded with W~ = -1 to a
+ * multiple of 512 columns; tiles of 16 rows x 512 columns (1 KiB) stored
+ * tile-row-major (tile (rb, kb) at byte 1024 * (rb * ceil(d_in/512) + kb));
+ * each tile row is 16 little-endian uint32 words; word kw covers columns
+ * 32 kw .. 32 kw + 31 and the bit c = (W~ + 1) / 2 of column 32 kw + 4 s + j
+ * sits at bit 8 j + s.  Size: d_out * ceil(d_in / 512) * 64 bytes (one bit
+ * per weight).  Decode only: the product takes 1 <= T <= 16.
+ */
+
+/* Bytes of the 1-bit format for d_out x d_in, or 0 for an unsupported shape. */
+size_t bitlinear_w1_packed_bytes(int64_t d_out, int64_t d_in);
+
+/*
+ * bitlinear_pack_weights_w1 -- binarise and pack fp32 latent weights.
+ *   W, gamma_in, workspace, workspace_bytes, gamma_out: as in
+ *   bitlinear_pack_weights (gamma = mean |W| unless gamma_in is given; it
+ *   scales the outputs and does not enter the codes).
+ *   packed1   out: bitlinear_w1_packed_bytes(d_out, d_in) bytes, 16-byte aligned.
+ */
+int bitlinear_pack_weights_w1(const float *W, int64_t d_out, int64_t d_in,
+                              const float *gamma_in, void *workspace, size_t workspace_bytes,
+                              uint32_t *packed1, float *gamma_out, cudaStream_t stream);
+
+/*
+ * bitlinear_forward_w1 -- the product on 1-bit weights with the fused
+ * rescale: acc[t][o] = sum_k W~[o][k] Xq[t][k] exactly in int32 (the kernel
+ * multiplies the bits c = (W~ + 1) / 2 and forms 2 sum c x - rowsum[t]),
+ * Y = acc * (gamma * beta[t] / (2^(act_bits-1) - 1)).  act_bits is 4 or 8 and
+ * must be the width the codes were made with (bitlinear_quant_act, with or
+ * without BITLINEAR_ACT_4BIT).  1 <= T <= 16; other arguments as in
+ * bitlinear_forward.
+ */
+int bitlinear_forward_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
+                         int64_t d_in, const int8_t *Xq, const float *beta,
+                         const int32_t *rowsum, int64_t T, int act_bits, void *Y, int out_dtype,
+                         int32_t *acc_out, cudaStream_t stream);
+
+/*
+ * bitlinear_linear_w1 -- bitlinear_linear on 1-bit weights: quantise (with
+ * BITLINEAR_ACT_4BIT: 4-bit codes, the W1A4 forward), then the product; one
+ * kernel for T <= 8 with T * d_in <= 32768.  flags: BITLINEAR_RMSNORM,
+ * BITLINEAR_STATIC_WEIGHTS, BITLINEAR_PER_TENSOR_ABSMAX, BITLINEAR_ACT_4BIT.
+ * 1 <= T <= 16.
+ */
+int bitlinear_linear_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
+                        int64_t d_in, const uint16_t *X, int64_t T, const float *norm_gain,
+                        uint32_t flags, float eps, float norm_eps, int8_t *Xq, float *beta,
+                        int32_t *rowsum, void *Y, int out_dtype, cudaStream_t stream);
 
 /*
  * bitlinear_dense_bf16_forward -- the dense bf16 linear layer Y = X W^T that

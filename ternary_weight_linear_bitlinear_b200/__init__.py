@@ -28,6 +28,7 @@ OUT_BF16 = 1
 RMSNORM = 1
 STATIC_WEIGHTS = 2
 PER_TENSOR_ABSMAX = 4
+ACT_4BIT = 8
 
 OK = 0
 ERR_INVALID_ARG = 1
@@ -61,6 +62,13 @@ SIGNATURES = {
                                        _vp, _vp]),
     "bitlinear_linear_base3": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
                                       _vp, _vp, _vp, _vp, _int, _vp]),
+    "bitlinear_w1_packed_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "bitlinear_pack_weights_w1": (_int, [_vp, _i64, _i64, _vp, _vp, ctypes.c_size_t, _vp, _vp,
+                                         _vp]),
+    "bitlinear_forward_w1": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _int,
+                                    _vp, _vp]),
+    "bitlinear_linear_w1": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
+                                   _vp, _vp, _vp, _vp, _int, _vp]),
     "bitlinear_dense_bf16_forward": (_int, [_vp, _i64, _i64, _vp, _i64, _vp, _int, _vp]),
     "bitlinear_backward_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _int, _int]),
     "bitlinear_backward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _int, _vp,
@@ -144,10 +152,51 @@ class PackedTernaryBase3:
     d_in: int
 
 
+@dataclass
+class PackedBinary:
+    """Sign-binarised weights of the W1A4 regime, one bit per weight (layout
+    in bitlinear.h); decode only (1 <= T <= 16)."""
+    packed: torch.Tensor    # int32 [w1_packed_bytes(d_out, d_in) / 4] (uint32 patterns)
+    gamma: torch.Tensor     # float32 [1], absmean scale
+    d_out: int
+    d_in: int
+
+
 def _entry(w, name: str):
-    """The entry point for w's format: name, or name + '_base3'."""
-    full = name + "_base3" if isinstance(w, PackedTernaryBase3) else name
+    """The entry point for w's format: name, name + '_base3' or name + '_w1'."""
+    if isinstance(w, PackedTernaryBase3):
+        full = name + "_base3"
+    elif isinstance(w, PackedBinary):
+        full = name + "_w1"
+    else:
+        full = name
     return getattr(lib(), full), full
+
+
+def w1_packed_bytes(d_out: int, d_in: int) -> int:
+    return int(lib().bitlinear_w1_packed_bytes(d_out, d_in))
+
+
+def pack_weights_w1(W: torch.Tensor, gamma: torch.Tensor = None) -> PackedBinary:
+    """Sign-binarise and pack fp32 latent weights [d_out][d_in] (W1)."""
+    _need(W, torch.float32, "W")
+    d_out, d_in = W.shape
+    n = w1_packed_bytes(d_out, d_in)
+    if n == 0:
+        _check(ERR_UNSUPPORTED_SHAPE, "pack_weights_w1")
+    out = PackedBinary(torch.empty(n // 4, dtype=torch.int32, device=W.device),
+                       torch.empty(1, dtype=torch.float32, device=W.device), d_out, d_in)
+    ws = None
+    if gamma is None:
+        ws = torch.empty(max(pack_workspace_bytes(d_out, d_in), 8), dtype=torch.uint8,
+                         device=W.device)
+    else:
+        _need(gamma, torch.float32, "gamma")
+    st = lib().bitlinear_pack_weights_w1(_ptr(W), d_out, d_in, _ptr(gamma), _ptr(ws),
+                                         0 if ws is None else ws.numel(), _ptr(out.packed),
+                                         _ptr(out.gamma), _stream())
+    _check(st, "bitlinear_pack_weights_w1")
+    return out
 
 
 def base3_bytes(d_out: int, d_in: int) -> int:
@@ -204,7 +253,7 @@ def pack_weights(W: torch.Tensor, eps: float = 1e-5, gamma: torch.Tensor = None,
 
 def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
               eps: float = 1e-5, norm_eps: float = 1e-5, inv_rms: torch.Tensor = None,
-              per_tensor: bool = False):
+              per_tensor: bool = False, act_bits: int = 8):
     """Fused RMSNorm + absmax int8 codes of bf16 X [T][d_in], with one beta
     per token (default) or one for the whole tensor (per_tensor).
 
@@ -222,7 +271,8 @@ def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
         _need(gain, torch.float32, "gain")
     if inv_rms is not None:
         _need(inv_rms, torch.float32, "inv_rms")
-    flags = (RMSNORM if rmsnorm else 0) | (PER_TENSOR_ABSMAX if per_tensor else 0)
+    flags = ((RMSNORM if rmsnorm else 0) | (PER_TENSOR_ABSMAX if per_tensor else 0)
+             | (ACT_4BIT if act_bits == 4 else 0))
     st = lib().bitlinear_quant_act(_ptr(X), T, d_in, _ptr(gain), flags,
                                    eps, norm_eps, _ptr(inv_rms), _ptr(Xq), _ptr(beta),
                                    _ptr(rowsum), _ptr(rms_out), _stream())
@@ -231,9 +281,11 @@ def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
 
 
 def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
-            out_dtype=torch.float32, want_acc: bool = False, out: torch.Tensor = None):
-    """Y = (X~ W~^T) gamma beta / 127; returns Y (and the int32 acc if asked).
-    w is a PackedTernary or a PackedTernaryBase3."""
+            out_dtype=torch.float32, want_acc: bool = False, out: torch.Tensor = None,
+            act_bits: int = 8):
+    """Y = (X~ W~^T) gamma beta / (Q_b - 1); returns Y (and the int32 acc if
+    asked).  w is a PackedTernary, PackedTernaryBase3 or PackedBinary; act_bits
+    (4 or 8, the width the codes were made with) applies to PackedBinary."""
     _need(Xq, torch.int8, "Xq")
     T = Xq.shape[0]
     dev = Xq.device
@@ -242,8 +294,14 @@ def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
     od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
     acc = torch.empty((T, w.d_out), dtype=torch.int32, device=dev) if want_acc else None
     fn, name = _entry(w, "bitlinear_forward")
-    st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq), _ptr(beta), _ptr(rowsum), T,
-            _ptr(out), od, _ptr(acc), _stream())
+    if isinstance(w, PackedBinary):
+        st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq), _ptr(beta),
+                _ptr(rowsum), T, act_bits, _ptr(out), od, _ptr(acc), _stream())
+    else:
+        if act_bits != 8:
+            raise ValueError("act_bits != 8 needs binary weights")
+        st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq), _ptr(beta),
+                _ptr(rowsum), T, _ptr(out), od, _ptr(acc), _stream())
     _check(st, name)
     return (out, acc) if want_acc else out
 
@@ -251,9 +309,10 @@ def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
 def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
            eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.float32,
            out: torch.Tensor = None, scratch=None, static_weights: bool = False,
-           per_tensor: bool = False):
+           per_tensor: bool = False, act_bits: int = 8):
     """The whole BitLinear forward from bf16 X: quantise, then product.
-    w is a PackedTernary or a PackedTernaryBase3.
+    w is a PackedTernary, PackedTernaryBase3 or PackedBinary; act_bits = 4
+    (PackedBinary only) makes it the W1A4 forward.
 
     static_weights: promise that no work still in flight on the stream
     writes w.packed or w.gamma (the product may then stream the weights
@@ -275,7 +334,7 @@ def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
     if gain is not None:
         _need(gain, torch.float32, "gain")
     flags = ((RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
-             | (PER_TENSOR_ABSMAX if per_tensor else 0))
+             | (PER_TENSOR_ABSMAX if per_tensor else 0) | (ACT_4BIT if act_bits == 4 else 0))
     fn, name = _entry(w, "bitlinear_linear")
     st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(X), T, _ptr(gain), flags, eps,
             norm_eps, _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
@@ -293,7 +352,7 @@ class LinearPlan:
     def __init__(self, w, T: int, gain: torch.Tensor = None, rmsnorm: bool = True,
                  eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.bfloat16,
                  out: torch.Tensor = None, scratch=None, static_weights: bool = False,
-                 per_tensor: bool = False, device=None):
+                 per_tensor: bool = False, device=None, act_bits: int = 8):
         dev = device if device is not None else w.packed.device
         if scratch is None:
             scratch = (torch.empty((T, w.d_in), dtype=torch.int8, device=dev),
@@ -306,7 +365,7 @@ class LinearPlan:
         Xq, beta, rowsum = scratch
         _need(Xq, torch.int8, "Xq")
         flags = ((RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
-                 | (PER_TENSOR_ABSMAX if per_tensor else 0))
+                 | (PER_TENSOR_ABSMAX if per_tensor else 0) | (ACT_4BIT if act_bits == 4 else 0))
         od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
         self.w, self.scratch, self.out, self.gain = w, scratch, out, gain   # keep alive
         self._shape = (T, w.d_in)

@@ -17,14 +17,14 @@ bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
 bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_out,
                              int64_t d_in, const int8_t *Xq, const float *beta,
                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                             int32_t *acc_out, bool static_weights, bool base3,
+                             int32_t *acc_out, bool static_weights, int fmt, float qmax,
                              cudaStream_t stream);
 bool decode_can_fuse(int64_t T, int64_t d_in);
 bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const uint16_t *X, int64_t T,
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
                                      int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
-                                     int out_dtype, bool static_weights, bool base3,
+                                     int out_dtype, bool static_weights, int fmt, float qmax,
                                      cudaStream_t stream);
 bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int64_t d_out,
                                 int64_t d_in, const int8_t *Xq, const float *beta,
@@ -129,10 +129,11 @@ static bitlinear_status dispatch_forward(const void *packed, const float *gamma,
                                          int64_t d_out, int64_t d_in, const int8_t *Xq,
                                          const float *beta, const int32_t *rowsum, int64_t T,
                                          void *Y, int out_dtype, int32_t *acc_out,
-                                         bool static_weights, bool base3, cudaStream_t stream) {
-    if (T <= 16 || base3)
+                                         bool static_weights, int fmt, float qmax,
+                                         cudaStream_t stream) {
+    if (T <= 16 || fmt != kFmt2Bit)
         return launch_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                           acc_out, static_weights, base3, stream);
+                           acc_out, static_weights, fmt, qmax, stream);
     return launch_gemm_tc(static_cast<const uint32_t *>(packed), gamma, d_out, d_in, Xq, beta,
                           rowsum, T, Y, out_dtype, acc_out, stream);
 }
@@ -140,10 +141,11 @@ static bitlinear_status dispatch_forward(const void *packed, const float *gamma,
 static bitlinear_status forward_common(const void *packed, const float *gamma, int64_t d_out,
                                        int64_t d_in, const int8_t *Xq, const float *beta,
                                        const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                                       int32_t *acc_out, bool base3, cudaStream_t stream) {
+                                       int32_t *acc_out, int fmt, float qmax,
+                                       cudaStream_t stream) {
     bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, acc_out);
     if (st != BITLINEAR_OK) return st;
-    if (base3 && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (fmt != kFmt2Bit && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     if (T == 0) return BITLINEAR_OK;
     if (!Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
     if (!aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4))
@@ -151,19 +153,21 @@ static bitlinear_status forward_common(const void *packed, const float *gamma, i
     st = check_device();
     if (st != BITLINEAR_OK) return st;
     return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                            acc_out, false, base3, stream);
+                            acc_out, false, fmt, qmax, stream);
 }
 
 static bitlinear_status linear_common(const void *packed, const float *gamma, int64_t d_out,
                                       int64_t d_in, const uint16_t *X, int64_t T,
                                       const float *norm_gain, uint32_t flags, float eps,
                                       float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
-                                      void *Y, int out_dtype, bool base3, cudaStream_t stream) {
+                                      void *Y, int out_dtype, int fmt, cudaStream_t stream) {
     bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, nullptr);
     if (st != BITLINEAR_OK) return st;
-    if (base3 && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_STATIC_WEIGHTS | BITLINEAR_PER_TENSOR_ABSMAX))
-        return BITLINEAR_ERR_INVALID_ARG;
+    if (fmt != kFmt2Bit && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    uint32_t allowed = BITLINEAR_RMSNORM | BITLINEAR_STATIC_WEIGHTS | BITLINEAR_PER_TENSOR_ABSMAX;
+    if (fmt == kFmt1Bit) allowed |= BITLINEAR_ACT_4BIT;   // the A4 of W1A4
+    if (flags & ~allowed) return BITLINEAR_ERR_INVALID_ARG;
+    const float qmax = (flags & BITLINEAR_ACT_4BIT) ? 7.0f : 127.0f;
     if (!(eps >= 0.0f) || !std::isfinite(eps) || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps))
         return BITLINEAR_ERR_INVALID_ARG;
     if (T == 0) return BITLINEAR_OK;
@@ -179,15 +183,16 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
     if (!per_tensor && decode_can_fuse(T, d_in))
         return launch_linear_fused(packed, gamma, d_out, d_in, X, T, norm_gain, rmsnorm, eps,
                                    norm_eps, Xq, beta, rowsum, Y, out_dtype, static_weights,
-                                   base3, stream);
+                                   fmt, qmax, stream);
     // Quantiser, then the product as its programmatic dependent: with static
     // weights the product streams them while the codes are still being made.
     st = launch_quant_act(X, T, d_in, norm_gain,
-                          flags & (BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX), eps,
-                          norm_eps, nullptr, Xq, beta, rowsum, nullptr, true, stream);
+                          flags & (BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX |
+                                   BITLINEAR_ACT_4BIT),
+                          eps, norm_eps, nullptr, Xq, beta, rowsum, nullptr, true, stream);
     if (st != BITLINEAR_OK) return st;
     return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                            nullptr, static_weights, base3, stream);
+                            nullptr, static_weights, fmt, qmax, stream);
 }
 
 }  // namespace bl
@@ -214,7 +219,7 @@ extern "C" int bitlinear_forward(const uint32_t *packed, const float *gamma, int
                                  const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
                                  int32_t *acc_out, cudaStream_t stream) {
     return forward_common(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype, acc_out,
-                          false, stream);
+                          kFmt2Bit, 127.0f, stream);
 }
 
 extern "C" int bitlinear_forward_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
@@ -222,7 +227,16 @@ extern "C" int bitlinear_forward_base3(const uint8_t *packed3, const float *gamm
                                        const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
                                        int32_t *acc_out, cudaStream_t stream) {
     return forward_common(packed3, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                          acc_out, true, stream);
+                          acc_out, kFmtBase3, 127.0f, stream);
+}
+
+extern "C" int bitlinear_forward_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
+                                    int64_t d_in, const int8_t *Xq, const float *beta,
+                                    const int32_t *rowsum, int64_t T, int act_bits, void *Y,
+                                    int out_dtype, int32_t *acc_out, cudaStream_t stream) {
+    if (act_bits != 4 && act_bits != 8) return BITLINEAR_ERR_INVALID_ARG;
+    return forward_common(packed1, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
+                          acc_out, kFmt1Bit, act_bits == 4 ? 7.0f : 127.0f, stream);
 }
 
 extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
@@ -231,7 +245,7 @@ extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int6
                                 int8_t *Xq, float *beta, int32_t *rowsum, void *Y, int out_dtype,
                                 cudaStream_t stream) {
     return linear_common(packed, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps, Xq,
-                         beta, rowsum, Y, out_dtype, false, stream);
+                         beta, rowsum, Y, out_dtype, kFmt2Bit, stream);
 }
 
 extern "C" int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
@@ -240,7 +254,16 @@ extern "C" int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma
                                       float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
                                       void *Y, int out_dtype, cudaStream_t stream) {
     return linear_common(packed3, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps, Xq,
-                         beta, rowsum, Y, out_dtype, true, stream);
+                         beta, rowsum, Y, out_dtype, kFmtBase3, stream);
+}
+
+extern "C" int bitlinear_linear_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
+                                   int64_t d_in, const uint16_t *X, int64_t T,
+                                   const float *norm_gain, uint32_t flags, float eps,
+                                   float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
+                                   void *Y, int out_dtype, cudaStream_t stream) {
+    return linear_common(packed1, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps, Xq,
+                         beta, rowsum, Y, out_dtype, kFmt1Bit, stream);
 }
 
 extern "C" int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, int64_t d_in,

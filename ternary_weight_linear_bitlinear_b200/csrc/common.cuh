@@ -8,6 +8,12 @@
 
 namespace bl {
 
+// Weight formats of the decode kernel: 2-bit ternary tiles, base-3 ternary
+// tiles (five codes per byte), 1-bit binary tiles.
+constexpr int kFmt2Bit = 0;
+constexpr int kFmtBase3 = 1;
+constexpr int kFmt1Bit = 2;
+
 // Bits of the device error word.
 constexpr uint32_t kErrTimeout = 1u;
 

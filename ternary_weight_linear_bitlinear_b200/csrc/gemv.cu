@@ -57,6 +57,17 @@
 // columns -- an A-operand register of an s8 MMA whose activation fragment is
 // eight consecutive code bytes.  The accumulator is -sum c x.
 //
+// 1-BIT variant (the W1 of the W1A4 regime on "The End of Matrix
+// Multiplications: Welcome to Addition"; binary alphabet of [MF] section 1):
+// tiles of 16 rows x 512 columns (1 KiB), word kw of a row holding columns
+// 32 kw .. 32 kw + 31 with the bit c = (W~ + 1) / 2 of column 32 kw + 4 s + j
+// at bit 8 j + s.  The lane reads the same 16-byte pieces as in the 2-bit
+// tile; word & (0x01010101 << s) is four codes of four consecutive columns
+// scaled by 2^s (one accumulator per slot, combined exactly), or, with two
+// token groups, (word >> s) & 0x01010101 into a single accumulator.  The sum
+// is sum c x, and W~ X~ = 2 sum c x - S.  The rescale divides by Q_b - 1 of
+// the activation codes (127, or 7 for 4-bit codes).
+//
 // Every mbarrier wait is bounded; on expiry the CTA stops consuming, the
 // producer waits (bounded) for the copies it issued, and the error word is
 // set.
@@ -81,7 +92,8 @@ struct DecodeArgs {
     const float *gamma;
     int d_out;
     int d_in;
-    int kb_total;            // k-tiles per row: d_in / 256, or ceil(d_in / 160) in base 3
+    int kb_total;            // k-tiles per row: d_in / 256, ceil(d_in / 160) (base 3), ceil(d_in / 512) (1 bit)
+    float qmax;              // Q_b - 1 of the activation codes: 127, or 7 for 4-bit codes
     int T;
     // product-only inputs (written by the stand-alone quantiser)
     const int8_t *Xq;
@@ -188,12 +200,18 @@ __device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, const De
     }
 }
 
-template <int NT, int R, bool FUSED, bool OUT_BF16, bool B3>
+template <int NT, int R, bool FUSED, bool OUT_BF16, int FMT>
 __global__ void __launch_bounds__(kDecThreads)
 decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx ctx) {
     constexpr int TMAX = NT * 8;
+    constexpr bool B3 = FMT == kFmtBase3;
+    constexpr bool W1 = FMT == kFmt1Bit;
     constexpr int kTileBytes = B3 ? 512 : 1024;
-    constexpr int kTileCols = B3 ? 160 : 256;
+    constexpr int kTileCols = B3 ? 160 : (W1 ? 512 : 256);
+    // Accumulators per (row tile, token group): one per 2-bit slot, one per
+    // 1-bit slot with a single token group, else one.
+    constexpr bool kW1Shift = W1 && NT > 1;
+    constexpr int kSlots = B3 ? 1 : (W1 ? (kW1Shift ? 1 : 8) : 4);
     extern __shared__ __align__(128) uint8_t dsm[];
     __shared__ __align__(8) uint64_t full_bar[kDecMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kDecMaxStages];
@@ -337,9 +355,9 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 sums[t] = 0;
                 if (t < T) {
                     const TokenScale ts =
-                        token_finalize<TMAX>(t, rmsnorm, a.eps, a.norm_eps, a.inv_k, qs);
+                        token_finalize<TMAX>(t, rmsnorm, a.eps, a.norm_eps, a.inv_k, a.qmax, qs);
                     if (threadIdx.x == 0) {
-                        s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, ts.beta), 127.0f);
+                        s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, ts.beta), a.qmax);
                         if (blockIdx.x == 0 && a.beta_out) a.beta_out[t] = ts.beta;
                     }
                     const uint4 *xrow = reinterpret_cast<const uint4 *>(xb + (size_t)t * K);
@@ -358,16 +376,16 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 }
             }
             __syncwarp();
-            // Base-3 tiles do not line up with the quantiser's 256-column
-            // blocks: every warp needs every code.
-            if constexpr (B3) consumer_barrier();
+            // Base-3 and 1-bit tiles do not line up with the quantiser's
+            // 256-column blocks: every warp needs every code.
+            if constexpr (FMT != kFmt2Bit) consumer_barrier();
         } else {
             token_stats<TMAX, true>(xb, T, K, a.gain, a.rmsnorm != 0, a.eps, a.norm_eps,
-                                    a.inv_k, nullptr, qs);
+                                    a.inv_k, a.qmax, nullptr, qs);
             token_codes<TMAX, true>(xb, T, K, a.gain, a.rmsnorm != 0, xs, qs);
             if (threadIdx.x < T) {
                 const int t = threadIdx.x;
-                s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, qs.beta[t]), 127.0f);
+                s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, qs.beta[t]), a.qmax);
                 s_rowsum[t] = qs.rowsum[t];
                 if (blockIdx.x == 0) {
                     if (a.beta_out) a.beta_out[t] = qs.beta[t];
@@ -384,7 +402,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     } else {
         if (threadIdx.x < T) {
             const int t = threadIdx.x;
-            s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, a.beta[t]), 127.0f);
+            s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, a.beta[t]), a.qmax);
             s_rowsum[t] = a.rowsum[t];
         }
         consumer_barrier();
@@ -394,13 +412,13 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     int st = 0;
     uint32_t fph = 0;
     for (int gi = 0; gi < ngrp; ++gi) {
-        int acc[R][NT][4][4];
+        int acc[R][NT][kSlots][4];
         #pragma unroll
         for (int r = 0; r < R; ++r)
             #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
                 #pragma unroll
-                for (int s = 0; s < 4; ++s)
+                for (int s = 0; s < kSlots; ++s)
                     #pragma unroll
                     for (int e = 0; e < 4; ++e) acc[r][nt][s][e] = 0;
 
@@ -445,6 +463,60 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                             for (int nt = 0; nt < NT; ++nt)
                                 mma_s8s8(acc[r][nt][0], dg[r][2 * m], dh[r][2 * m],
                                          dg[r][2 * m + 1], dh[r][2 * m + 1], xr[nt].x, xr[nt].y);
+                    }
+                }
+            } else if constexpr (W1) {
+                for (int kk = warp; kk < nkb; kk += kDecWarps) {
+                    // This lane's 128 columns of the tile: 128q .. 128q+127.
+                    const int col0 = (sl * ks + kk) * 512 + 128 * q;
+                    uint32_t w0[R][4], w1[R][4];   // words 4q..4q+3 of rows g and g + 8
+                    #pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const uint8_t *tile = stage + (r * ks + kk) * 1024;
+                        const uint4 lo = *reinterpret_cast<const uint4 *>(tile + lane * 16);
+                        const uint4 hi = *reinterpret_cast<const uint4 *>(tile + 512 + lane * 16);
+                        w0[r][0] = lo.x; w0[r][1] = lo.y; w0[r][2] = lo.z; w0[r][3] = lo.w;
+                        w1[r][0] = hi.x; w1[r][1] = hi.y; w1[r][2] = hi.z; w1[r][3] = hi.w;
+                    }
+                    #pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        // Activation bytes of columns col0 + 64p .. +63 of each token.
+                        uint32_t xr[NT][16];
+                        #pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const int t = nt * 8 + g;
+                            const uint8_t *xsrc =
+                                FUSED ? reinterpret_cast<const uint8_t *>(xs) + (size_t)t * K +
+                                            col0 + 64 * p
+                                      : stage + R * ks * 1024 + t * ks * 512 + kk * 512 +
+                                            128 * q + 64 * p;
+                            #pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                uint4 x = make_uint4(0, 0, 0, 0);
+                                if (t < T && col0 + 64 * p + 16 * v < K)   // d_in % 256 == 0
+                                    x = *reinterpret_cast<const uint4 *>(xsrc + 16 * v);
+                                xr[nt][4 * v + 0] = x.x;
+                                xr[nt][4 * v + 1] = x.y;
+                                xr[nt][4 * v + 2] = x.z;
+                                xr[nt][4 * v + 3] = x.w;
+                            }
+                        }
+                        #pragma unroll
+                        for (int r = 0; r < R; ++r) {
+                            #pragma unroll
+                            for (int s = 0; s < 8; ++s) {
+                                auto slot = [&](uint32_t w) {
+                                    return kW1Shift ? (w >> s) & 0x01010101u
+                                                    : w & (0x01010101u << s);
+                                };
+                                const uint32_t a0 = slot(w0[r][2 * p]), a2 = slot(w0[r][2 * p + 1]);
+                                const uint32_t a1 = slot(w1[r][2 * p]), a3 = slot(w1[r][2 * p + 1]);
+                                #pragma unroll
+                                for (int nt = 0; nt < NT; ++nt)
+                                    mma_u8s8(acc[r][nt][kW1Shift ? 0 : s], a0, a1, a2, a3,
+                                             xr[nt][s], xr[nt][8 + s]);
+                            }
+                        }
                     }
                 }
             } else
@@ -505,10 +577,19 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             for (int nt = 0; nt < NT; ++nt) {
                 int c[4];
                 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    c[e] = B3 ? -acc[r][nt][0][e]
-                              : acc[r][nt][0][e] + (acc[r][nt][1][e] >> 2) +
-                                    (acc[r][nt][2][e] >> 4) + (acc[r][nt][3][e] >> 6);
+                for (int e = 0; e < 4; ++e) {
+                    if constexpr (B3) {
+                        c[e] = -acc[r][nt][0][e];
+                    } else if constexpr (W1) {
+                        // Slot s summed c 2^s x; every term is a multiple of 2^s.
+                        c[e] = acc[r][nt][0][e];
+                        #pragma unroll
+                        for (int s2 = 1; s2 < kSlots; ++s2) c[e] += acc[r][nt][s2][e] >> s2;
+                    } else {
+                        c[e] = acc[r][nt][0][e] + (acc[r][nt][1 % kSlots][e] >> 2) +
+                               (acc[r][nt][2 % kSlots][e] >> 4) + (acc[r][nt][3 % kSlots][e] >> 6);
+                    }
+                }
                 red[warp][r][nt][lane] = make_int4(c[0], c[1], c[2], c[3]);
             }
         consumer_barrier();
@@ -559,7 +640,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             } else {
                 rsum = s_rowsum[t];
             }
-            const int accv = v - rsum;
+            // Offset codes: W~ = c - 1 (2-bit, base 3) or 2c - 1 (1 bit).
+            const int accv = W1 ? 2 * v - rsum : v - rsum;
             const int o = (rt0 + r) * 16 + row;
             const size_t yi = (size_t)t * a.d_out + o;
             if (a.acc_out) a.acc_out[yi] = accv;
@@ -594,11 +676,11 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
 #endif
 constexpr int kFusedMaxCodeBytes = BL_FUSED_MAX_CODE_BYTES;
 
-template <int NT, int R, bool FUSED, bool OUT_BF16, bool B3>
+template <int NT, int R, bool FUSED, bool OUT_BF16, int FMT>
 static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
                                    cudaStream_t stream) {
-    constexpr int kTileBytes = B3 ? 512 : 1024;
-    constexpr int kTileCols = B3 ? 160 : 256;
+    constexpr int kTileBytes = FMT == kFmtBase3 ? 512 : 1024;
+    constexpr int kTileCols = FMT == kFmtBase3 ? 160 : (FMT == kFmt1Bit ? 512 : 256);
     const int n_rt = args.d_out / 16;
     const int n_groups = (n_rt + R - 1) / R;
     const int KB = args.kb_total, K = args.d_in;
@@ -623,7 +705,7 @@ static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
     if (plan.stages < 2) plan.stages = 2;
     const size_t smem =
         (size_t)xb_bytes + (size_t)plan.xs_bytes + (size_t)plan.stages * plan.stage_bytes;
-    auto kern = decode_kernel<NT, R, FUSED, OUT_BF16, B3>;
+    auto kern = decode_kernel<NT, R, FUSED, OUT_BF16, FMT>;
     cudaError_t e = ensure_dynamic_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148, per_sm = 1;
@@ -651,7 +733,7 @@ static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
     return cudaLaunchKernelEx(&cfg, kern, args, plan, ctx);
 }
 
-template <bool FUSED, bool OUT_BF16, bool B3>
+template <bool FUSED, bool OUT_BF16, int FMT>
 static cudaError_t launch_decode_r(const DecodeArgs &args, const DeviceCtx &ctx,
                                    cudaStream_t stream) {
     // One row tile per group while that still leaves a few CTAs per SM;
@@ -659,43 +741,51 @@ static cudaError_t launch_decode_r(const DecodeArgs &args, const DeviceCtx &ctx,
     const int n_rt = args.d_out / 16;
     const bool wide = n_rt >= BL_DEC_WIDE_ROW_TILES;
     if (args.T <= 8)
-        return wide ? launch_decode_t<1, 2, FUSED, OUT_BF16, B3>(args, ctx, stream)
-                    : launch_decode_t<1, 1, FUSED, OUT_BF16, B3>(args, ctx, stream);
+        return wide ? launch_decode_t<1, 2, FUSED, OUT_BF16, FMT>(args, ctx, stream)
+                    : launch_decode_t<1, 1, FUSED, OUT_BF16, FMT>(args, ctx, stream);
     if constexpr (FUSED) return cudaErrorInvalidValue;   // fused path is T <= 8 only
-    return wide ? launch_decode_t<2, 2, false, OUT_BF16, B3>(args, ctx, stream)
-                : launch_decode_t<2, 1, false, OUT_BF16, B3>(args, ctx, stream);
+    return wide ? launch_decode_t<2, 2, false, OUT_BF16, FMT>(args, ctx, stream)
+                : launch_decode_t<2, 1, false, OUT_BF16, FMT>(args, ctx, stream);
 }
 
 bool decode_can_fuse(int64_t T, int64_t d_in) {
     return T >= 1 && T <= 8 && T * d_in <= kFusedMaxCodeBytes;
 }
 
-template <bool B3>
+template <int FMT>
 static cudaError_t launch_decode_f(const DecodeArgs &args, bool fused, bool bf,
                                    const DeviceCtx &ctx, cudaStream_t stream) {
     if (fused)
-        return bf ? launch_decode_r<true, true, B3>(args, ctx, stream)
-                  : launch_decode_r<true, false, B3>(args, ctx, stream);
-    return bf ? launch_decode_r<false, true, B3>(args, ctx, stream)
-              : launch_decode_r<false, false, B3>(args, ctx, stream);
+        return bf ? launch_decode_r<true, true, FMT>(args, ctx, stream)
+                  : launch_decode_r<true, false, FMT>(args, ctx, stream);
+    return bf ? launch_decode_r<false, true, FMT>(args, ctx, stream)
+              : launch_decode_r<false, false, FMT>(args, ctx, stream);
 }
 
-bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, bool base3,
+bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, int fmt,
                                cudaStream_t stream) {
     DeviceCtx ctx;
     bitlinear_status st = get_ctx(&ctx);
     if (st != BITLINEAR_OK) return st;
     const bool bf = out_dtype == BITLINEAR_OUT_BF16;
-    args.kb_total = base3 ? (args.d_in + 159) / 160 : args.d_in / 256;
-    const cudaError_t e = base3 ? launch_decode_f<true>(args, fused, bf, ctx, stream)
-                                : launch_decode_f<false>(args, fused, bf, ctx, stream);
+    cudaError_t e;
+    if (fmt == kFmtBase3) {
+        args.kb_total = (args.d_in + 159) / 160;
+        e = launch_decode_f<kFmtBase3>(args, fused, bf, ctx, stream);
+    } else if (fmt == kFmt1Bit) {
+        args.kb_total = (args.d_in + 511) / 512;
+        e = launch_decode_f<kFmt1Bit>(args, fused, bf, ctx, stream);
+    } else {
+        args.kb_total = args.d_in / 256;
+        e = launch_decode_f<kFmt2Bit>(args, fused, bf, ctx, stream);
+    }
     return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
 bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_out,
                              int64_t d_in, const int8_t *Xq, const float *beta,
                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                             int32_t *acc_out, bool static_weights, bool base3,
+                             int32_t *acc_out, bool static_weights, int fmt, float qmax,
                              cudaStream_t stream) {
     DecodeArgs a = {};
     a.packed = static_cast<const uint8_t *>(packed);
@@ -709,14 +799,15 @@ bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_o
     a.Y = Y;
     a.acc_out = acc_out;
     a.static_weights = static_weights ? 1 : 0;
-    return launch_decode(a, false, out_dtype, base3, stream);
+    a.qmax = qmax;
+    return launch_decode(a, false, out_dtype, fmt, stream);
 }
 
 bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const uint16_t *X, int64_t T,
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
                                      int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
-                                     int out_dtype, bool static_weights, bool base3,
+                                     int out_dtype, bool static_weights, int fmt, float qmax,
                                      cudaStream_t stream) {
     DecodeArgs a = {};
     a.packed = static_cast<const uint8_t *>(packed);
@@ -735,7 +826,8 @@ bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int
     a.rowsum_out = rowsum;
     a.Y = Y;
     a.static_weights = static_weights ? 1 : 0;
-    return launch_decode(a, true, out_dtype, base3, stream);
+    a.qmax = qmax;
+    return launch_decode(a, true, out_dtype, fmt, stream);
 }
 
 }  // namespace bl

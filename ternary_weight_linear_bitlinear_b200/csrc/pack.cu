@@ -140,6 +140,57 @@ repack_base3_kernel(const uint32_t *__restrict__ packed, int64_t d_out, int64_t 
     }
 }
 
+// gamma = mean |W| into *gamma_out: the two-stage fixed-order reduction.
+static void launch_absmean(const float *W, int64_t n, double *partial, float *gamma_out,
+                           cudaStream_t stream) {
+    const int64_t n4 = n / 4;
+    int blocks = (int)((n4 + kRedThreads * 8 - 1) / (kRedThreads * 8));
+    if (blocks > kRedMaxBlocks) blocks = kRedMaxBlocks;
+    if (blocks < 1) blocks = 1;
+    absmean_partial_kernel<<<blocks, kRedThreads, 0, stream>>>(
+        reinterpret_cast<const float4 *>(W), n4, partial);
+    absmean_final_kernel<<<1, kRedThreads, 0, stream>>>(partial, blocks, (double)n, gamma_out);
+}
+
+// 1-bit format (the W1 of the W1A4 regime on "The End of Matrix
+// Multiplications: Welcome to Addition"; the binary alphabet {-1, +1} of
+// section 1 of the b1.58 page): W~ = +1 where W >= 0, else -1, with the same
+// absmean gamma as scale.  Tiles of 16 rows x 512 columns (1 KiB), rows
+// padded with W~ = -1 (bit 0); word kw of a tile row covers columns 32 kw ..
+// 32 kw + 31 and the bit c = (W~ + 1) / 2 of column 32 kw + 4 s + j sits at
+// bit 8 j + s.  One thread per output word.
+__global__ void __launch_bounds__(256)
+pack_w1_kernel(const float *__restrict__ W, int64_t d_out, int64_t d_in,
+               uint32_t *__restrict__ packed, const float *__restrict__ gamma_src,
+               float *gamma_out) {
+    const int64_t tiles = (d_in + 511) / 512;
+    const int64_t nwords = d_out * tiles * 16;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    if (blockIdx.x == 0 && threadIdx.x == 0 && gamma_src && gamma_src != gamma_out)
+        *gamma_out = *gamma_src;
+    for (int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < nwords; wi += stride) {
+        const int64_t tile = wi >> 8;
+        const int within = (int)(wi & 255);
+        const int r = within >> 4, kw = within & 15;
+        const int64_t rb = tile / tiles, kb = tile - rb * tiles;
+        const int64_t o = rb * 16 + r;
+        const int64_t k0 = kb * 512 + kw * 32;
+        uint32_t word = 0;
+        if (k0 < d_in) {   // d_in % 256 == 0, so a word is all real or all padding
+            const float4 *src = reinterpret_cast<const float4 *>(W + o * d_in + k0);
+            #pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const float4 v = __ldg(src + s);
+                const float e[4] = {v.x, v.y, v.z, v.w};
+                #pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (e[j] >= 0.0f) word |= 1u << (8 * j + s);
+            }
+        }
+        packed[wi] = word;
+    }
+}
+
 }  // namespace bl
 
 using namespace bl;
@@ -181,15 +232,7 @@ extern "C" int bitlinear_pack_weights(const float *W, int64_t d_out, int64_t d_i
     const int64_t n = d_out * d_in;
     const float *gptr = gamma_in;
     if (!gamma_in) {
-        const int64_t n4 = n / 4;
-        int blocks = (int)((n4 + kRedThreads * 8 - 1) / (kRedThreads * 8));
-        if (blocks > kRedMaxBlocks) blocks = kRedMaxBlocks;
-        if (blocks < 1) blocks = 1;
-        double *partial = static_cast<double *>(workspace);
-        absmean_partial_kernel<<<blocks, kRedThreads, 0, stream>>>(
-            reinterpret_cast<const float4 *>(W), n4, partial);
-        absmean_final_kernel<<<1, kRedThreads, 0, stream>>>(partial, blocks, (double)n,
-                                                             gamma_out);
+        launch_absmean(W, n, static_cast<double *>(workspace), gamma_out, stream);
         gptr = gamma_out;
     }
     const int64_t nwords = n / 16;
@@ -292,5 +335,38 @@ extern "C" int bitlinear_repack_base3(const uint32_t *packed, int64_t d_out, int
     if (blocks > 148 * 16) blocks = 148 * 16;
     repack_base3_kernel<<<(int)blocks, 256, 0, stream>>>(packed, d_out, d_in,
                                                           reinterpret_cast<uint32_t *>(packed3));
+    return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+extern "C" size_t bitlinear_w1_packed_bytes(int64_t d_out, int64_t d_in) {
+    if (bitlinear_packed_words(d_out, d_in) == 0) return 0;
+    return (size_t)(d_out * ((d_in + 511) / 512) * 64);
+}
+
+extern "C" int bitlinear_pack_weights_w1(const float *W, int64_t d_out, int64_t d_in,
+                                         const float *gamma_in, void *workspace,
+                                         size_t workspace_bytes, uint32_t *packed1,
+                                         float *gamma_out, cudaStream_t stream) {
+    if (!W || !packed1 || !gamma_out) return BITLINEAR_ERR_INVALID_ARG;
+    if (bitlinear_packed_words(d_out, d_in) == 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (!gamma_in) {
+        if (!workspace) return BITLINEAR_ERR_INVALID_ARG;
+        if (workspace_bytes < bitlinear_pack_workspace_bytes(d_out, d_in))
+            return BITLINEAR_ERR_INVALID_ARG;
+        if (!aligned(workspace, 8)) return BITLINEAR_ERR_MISALIGNED;
+    } else if (!aligned(gamma_in, 4)) {
+        return BITLINEAR_ERR_MISALIGNED;
+    }
+    if (!aligned(W, 16) || !aligned(packed1, 16) || !aligned(gamma_out, 4))
+        return BITLINEAR_ERR_MISALIGNED;
+    bitlinear_status st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    if (!gamma_in) launch_absmean(W, d_out * d_in, static_cast<double *>(workspace), gamma_out,
+                                  stream);
+    const int64_t nwords = (int64_t)(bitlinear_w1_packed_bytes(d_out, d_in) / 4);
+    int64_t blocks = (nwords + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    pack_w1_kernel<<<(int)blocks, 256, 0, stream>>>(W, d_out, d_in, packed1, gamma_in,
+                                                    gamma_out);
     return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }

@@ -15,6 +15,10 @@
 // reduction order is the one of quant_common.cuh, shared with the fused
 // decode kernel.
 //
+// 4-bit codes (BITLINEAR_ACT_4BIT, the A4 of the W1A4 regime): the same
+// section's Q_b = 2^(k-1) with k = 4, so the multiplier and the clip bound
+// are 7 instead of 127.
+//
 // Per-tensor scope (the same section prints beta as the max over all i, j):
 // three launches -- every token's statistics (beta[t] = its own absmax), one
 // CTA folding them into beta[0] = max_t beta[t], then every token's codes on
@@ -37,7 +41,7 @@ enum QuantMode : int {
 
 __global__ void __launch_bounds__(kQuantThreads)
 quant_act_kernel(const uint16_t *__restrict__ X, int d_in, const float *__restrict__ gain,
-                 int rmsnorm, float eps, float norm_eps, double inv_k,
+                 int rmsnorm, float eps, float norm_eps, double inv_k, float qmax,
                  const float *__restrict__ inv_rms_in,
                  int8_t *__restrict__ Xq, float *__restrict__ beta_out,
                  int32_t *__restrict__ rowsum, float *__restrict__ inv_rms_out, int mode) {
@@ -53,7 +57,7 @@ quant_act_kernel(const uint16_t *__restrict__ X, int d_in, const float *__restri
     pdl_wait_primary();
 
     const uint16_t *row = X + t * d_in;
-    token_stats<1>(row, 1, d_in, gain, rmsnorm != 0, eps, norm_eps, inv_k,
+    token_stats<1>(row, 1, d_in, gain, rmsnorm != 0, eps, norm_eps, inv_k, qmax,
                    inv_rms_in ? inv_rms_in + t : nullptr, qs);
     if (mode == kQuantStatsOnly) {
         if (threadIdx.x == 0) {
@@ -68,7 +72,7 @@ quant_act_kernel(const uint16_t *__restrict__ X, int d_in, const float *__restri
         if (threadIdx.x == 0) {
             const float b = beta_out[0];
             qs.beta[0] = b;
-            qs.scale[0] = __fdiv_rn(127.0f, __fadd_rn(b, eps));
+            qs.scale[0] = __fdiv_rn(qmax, __fadd_rn(b, eps));
         }
         quant_barrier();
     }
@@ -113,22 +117,24 @@ bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     const double inv_k = 1.0 / (double)d_in;
+    // Q_b - 1 for 8-bit codes (127) or, under BITLINEAR_ACT_4BIT, 4-bit (7).
+    const float qmax = (flags & BITLINEAR_ACT_4BIT) ? 7.0f : 127.0f;
     cudaError_t e;
     if (!per_tensor) {
         e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
-                               norm_eps, inv_k, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
+                               norm_eps, inv_k, qmax, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
                                (int)kQuantPerToken);
         return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
     }
     e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
-                           norm_eps, inv_k, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
+                           norm_eps, inv_k, qmax, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
                            (int)kQuantStatsOnly);
     if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
     beta_max_kernel<<<1, kBetaMaxThreads, 0, stream>>>(beta, T);
     if (cudaGetLastError() != cudaSuccess) return BITLINEAR_ERR_CUDA;
     cfg.numAttrs = 0;   // the codes need the folded beta: an ordinary stream-ordered launch
     e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
-                           norm_eps, inv_k, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
+                           norm_eps, inv_k, qmax, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
                            (int)kQuantSharedBeta);
     return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
@@ -144,7 +150,7 @@ extern "C" int bitlinear_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                                    cudaStream_t stream) {
     if (T < 0 || T > (1 << 20)) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     if (d_in <= 0 || d_in % 256 || d_in > 65536) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX))
+    if (flags & ~(BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX | BITLINEAR_ACT_4BIT))
         return BITLINEAR_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !std::isfinite(eps)) return BITLINEAR_ERR_INVALID_ARG;
     if (!(norm_eps >= 0.0f) || !std::isfinite(norm_eps)) return BITLINEAR_ERR_INVALID_ARG;

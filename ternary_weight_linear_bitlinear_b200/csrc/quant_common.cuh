@@ -51,7 +51,7 @@ struct QuantShared {
     int sum[kQuantWarps][TMAX];
     float inv_rms[TMAX];
     float beta[TMAX];
-    float scale[TMAX];   // 127 / (beta + eps)
+    float scale[TMAX];   // qmax / (beta + eps)
     int rowsum[TMAX];
 };
 
@@ -119,9 +119,10 @@ __device__ __forceinline__ int warp_sum_i32(int v) {
 // where the spacing is 1, exactly at 1.5 * 2^23 + floor(u).  The low byte is
 // then the code in two's complement, and the pattern minus kCodeBias is the
 // code itself.  Valid for |v| < 2^22; the quantiser's v never exceeds
-// 127.00001 in magnitude: |n| <= beta because beta is the absmax of the same
-// rounded products, and fl(127 / (beta + eps)) <= (127 / beta)(1 + 2^-24),
-// so floor(v + 0.5) already lies in [-127, 127] and the clip is a no-op.
+// qmax (1 + 2^-23) in magnitude (qmax = Q_b - 1 = 127 for 8-bit codes, 7 for
+// 4-bit): |n| <= beta because beta is the absmax of the same rounded
+// products, and fl(qmax / (beta + eps)) <= (qmax / beta)(1 + 2^-24), so
+// floor(v + 0.5) already lies in [-qmax, qmax] and the clip is a no-op.
 constexpr uint32_t kCodeBias = 0x4B400000u;   // bit pattern of 1.5 * 2^23
 __device__ __forceinline__ uint32_t code_bits(float v) {
     return __float_as_uint(__fadd_rd(__fadd_rd(v, 0.5f), 12582912.0f));
@@ -169,14 +170,14 @@ __device__ __forceinline__ void token_partials_smem(const uint16_t *X, int T, in
 struct TokenScale {
     float inv_rms;   // r (1 without RMSNorm)
     float beta;      // absmax of the normalised row
-    float scale;     // 127 / (beta + eps)
+    float scale;     // qmax / (beta + eps)
 };
 
 // Final statistics of token t from the warp partials (fixed warp order); any
 // thread may compute them and every thread gets the same bits.  No gain.
 template <int TMAX>
 __device__ __forceinline__ TokenScale token_finalize(int t, bool rmsnorm, float eps,
-                                                     float norm_eps, double inv_k,
+                                                     float norm_eps, double inv_k, float qmax,
                                                      const QuantShared<TMAX> &qs) {
     TokenScale ts;
     ts.inv_rms = 1.0f;
@@ -190,7 +191,7 @@ __device__ __forceinline__ TokenScale token_finalize(int t, bool rmsnorm, float 
     #pragma unroll
     for (int w = 1; w < kQuantWarps; ++w) m = fmaxf(m, qs.amax[w][t]);
     ts.beta = rmsnorm ? __fmul_rn(m, ts.inv_rms) : m;
-    ts.scale = __fdiv_rn(127.0f, __fadd_rn(ts.beta, eps));
+    ts.scale = __fdiv_rn(qmax, __fadd_rn(ts.beta, eps));
     return ts;
 }
 
@@ -223,7 +224,7 @@ __device__ __forceinline__ uint4 load_row_vec(const uint4 *row, int v) {
 template <int TMAX, bool kSmemSrc = false>
 __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int T, int K,
                                          const float *__restrict__ gain, bool rmsnorm,
-                                         float eps, float norm_eps, double inv_k,
+                                         float eps, float norm_eps, double inv_k, float qmax,
                                          const float *__restrict__ inv_rms_in,
                                          QuantShared<TMAX> &qs) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -271,7 +272,7 @@ __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int 
             qs.inv_rms[t] = r;
             qs.beta[t] = __fmul_rn(m, r);
         } else {
-            const TokenScale ts = token_finalize<TMAX>(t, rmsnorm, eps, norm_eps, inv_k, qs);
+            const TokenScale ts = token_finalize<TMAX>(t, rmsnorm, eps, norm_eps, inv_k, qmax, qs);
             qs.inv_rms[t] = ts.inv_rms;
             qs.beta[t] = ts.beta;                    // replaced below when a gain is set
         }
@@ -303,7 +304,7 @@ __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int 
         }
         quant_barrier();
     }
-    if (tid < T) qs.scale[tid] = __fdiv_rn(127.0f, __fadd_rn(qs.beta[tid], eps));
+    if (tid < T) qs.scale[tid] = __fdiv_rn(qmax, __fadd_rn(qs.beta[tid], eps));
     quant_barrier();
 }
 

@@ -125,6 +125,38 @@ def test_base3_sizes_and_validation(lib):
     assert rp(P(0x10000), 16, 256, P(0x20008), S0) == bl.ERR_MISALIGNED
 
 
+def test_w1_sizes_and_validation(lib):
+    """One bit per weight on rows padded to 512 columns; the W1 entry points
+    take 1 <= T <= 16, act_bits 4 or 8, and the 4-bit flag only with binary
+    weights."""
+    assert bl.w1_packed_bytes(6912, 2560) == 6912 * 2560 // 8
+    assert bl.w1_packed_bytes(4096, 11008) == 4096 * 11264 // 8
+    assert bl.w1_packed_bytes(16, 256) == 16 * 512 // 8
+    assert bl.w1_packed_bytes(15, 256) == 0
+    f = lib.bitlinear_forward_w1
+
+    def fwd(T=4, bits=4, d_in=256, packed=0x10000):
+        return f(P(packed), P(0x20000), 64, d_in, P(0x30000), P(0x40000), P(0x50000), T, bits,
+                 P(0x60000), 0, None, S0)
+
+    assert fwd(T=17) == bl.ERR_UNSUPPORTED_SHAPE
+    assert fwd(bits=5) == bl.ERR_INVALID_ARG
+    assert fwd(d_in=384) == bl.ERR_UNSUPPORTED_SHAPE
+    assert fwd(packed=0x10004) == bl.ERR_MISALIGNED
+    assert fwd(T=0) == bl.OK
+    args = (P(0x10000), P(0x20000), 64, 256, P(0x30000), 4, None)
+    tail = (1e-5, 1e-5, P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0)
+    assert lib.bitlinear_linear(*args, 1 | bl.ACT_4BIT, *tail) == bl.ERR_INVALID_ARG
+    assert lib.bitlinear_linear_w1(*args, 16, *tail) == bl.ERR_INVALID_ARG
+    pk = lib.bitlinear_pack_weights_w1
+    assert pk(P(0x10000), 16, 128, None, P(0x20000), 1 << 20, P(0x30000), P(0x40000),
+              S0) == bl.ERR_UNSUPPORTED_SHAPE
+    assert pk(P(0x10000), 16, 256, None, None, 0, P(0x30000), P(0x40000),
+              S0) == bl.ERR_INVALID_ARG
+    assert pk(P(0x10000), 16, 256, None, P(0x20000), 1 << 20, P(0x30008), P(0x40000),
+              S0) == bl.ERR_MISALIGNED
+
+
 def test_quant_act_validation(lib):
     q = lib.bitlinear_quant_act
     args = dict(X=0x10000, T=2, d_in=512, gain=None, flags=1, eps=1e-5, neps=1e-5, rms=None,
@@ -137,7 +169,8 @@ def test_quant_act_validation(lib):
                  P(a["beta"]), P(a["rs"]), P(a["rmso"]) if a["rmso"] else None, S0)
 
     assert call(X=0) == bl.ERR_INVALID_ARG
-    assert call(flags=8) == bl.ERR_INVALID_ARG                     # no such flag
+    assert call(flags=16) == bl.ERR_INVALID_ARG                    # no such flag
+    assert call(flags=1 | bl.ACT_4BIT) != bl.ERR_INVALID_ARG        # 4-bit codes
     assert call(flags=2) == bl.ERR_INVALID_ARG                     # bitlinear_linear's only
     assert call(flags=1 | bl.PER_TENSOR_ABSMAX) != bl.ERR_INVALID_ARG
     assert call(eps=float("nan")) == bl.ERR_INVALID_ARG
