@@ -196,15 +196,21 @@ def fused(p: Problem) -> bool:
     return p.tokens <= 8 and p.tokens * p.d_in <= FUSED_MAX_CODE_BYTES
 
 
-def decode_bytes(p: Problem, out_bytes: int = 2, base3: bool = False) -> dict:
+def decode_bytes(p: Problem, out_bytes: int = 2, fmt: str = "2bit") -> dict:
     """Algorithmic bytes of one decode BitLinear forward (quantise + product).
 
     Fused (one kernel): packed W + bf16 X read + codes, beta, row sums written
     once + gamma + Y.  Two kernels: the codes, beta and row sums are also read
-    back once by the product.  base3: five codes per byte on rows padded to
-    160 columns instead of four per byte."""
+    back once by the product.  fmt: "2bit" (four codes per byte), "base3" (five
+    codes per byte on rows padded to 160 columns) or "w1" (one bit per weight
+    on rows padded to 512 columns)."""
     T, K, N = p.tokens, p.d_in, p.d_out
-    w = N * ((K + 159) // 160 * 160) // 5 if base3 else N * K // 4
+    if fmt == "base3":
+        w = N * ((K + 159) // 160 * 160) // 5
+    elif fmt == "w1":
+        w = N * ((K + 511) // 512 * 512) // 8
+    else:
+        w = N * K // 4
     x = T * K * 2                    # bf16 activations
     inter = T * K + 8 * T            # codes, beta, row sums written
     y = T * N * out_bytes
@@ -273,10 +279,11 @@ def profile_traffic(summary_name: str, source):
 class DecodeRun:
     """`layers` forwards per step over distinct packed weight copies."""
 
-    def __init__(self, problems, layers, dev, out_dtype=torch.bfloat16, base3=False):
+    def __init__(self, problems, layers, dev, out_dtype=torch.bfloat16, fmt="2bit"):
         import ternary_weight_linear_bitlinear_b200 as bl
         self.bl = bl
-        self.base3 = base3
+        self.fmt = fmt
+        self.act_bits = 4 if fmt == "w1" else 8     # the W1A4 regime
         self.problems = problems
         self.dev = dev
         self.out_dtype = out_dtype
@@ -284,8 +291,11 @@ class DecodeRun:
         base = []
         for p in problems:
             W, X = draw(p)
-            w = bl.pack_weights(W.to(dev), EPS)
-            if base3:
+            if fmt == "w1":
+                w = bl.pack_weights_w1(W.to(dev))
+            else:
+                w = bl.pack_weights(W.to(dev), EPS)
+            if fmt == "base3":
                 w = bl.repack_base3(w)
             base.append((p, w, X.to(dev)))
             del W
@@ -305,7 +315,7 @@ class DecodeRun:
         torch.cuda.synchronize()
         # Pre-quantised activations for the product-only timing.
         for p, w, X, scratch, Y in self.layers:
-            xq, beta, rowsum, _ = bl.quant_act(X)
+            xq, beta, rowsum, _ = bl.quant_act(X, act_bits=self.act_bits)
             scratch[0].copy_(xq)
             scratch[1].copy_(beta)
             scratch[2].copy_(rowsum)
@@ -313,17 +323,18 @@ class DecodeRun:
 
     def step(self):
         for p, w, X, scratch, Y in self.layers:
-            self.bl.linear(w, X, out=Y, scratch=scratch, static_weights=True)
+            self.bl.linear(w, X, out=Y, scratch=scratch, static_weights=True,
+                           act_bits=self.act_bits)
 
     def product_only(self):
         for p, w, X, scratch, Y in self.layers:
-            self.bl.forward(w, scratch[0], scratch[1], scratch[2], out=Y)
+            self.bl.forward(w, scratch[0], scratch[1], scratch[2], out=Y, act_bits=self.act_bits)
 
     def bytes(self):
         ob = 2 if self.out_dtype == torch.bfloat16 else 4
         tot = dict(step=0, gemv=0, weights=0, weights_and_acts=0)
         for p, *_ in self.layers:
-            for k, v in decode_bytes(p, ob, self.base3).items():
+            for k, v in decode_bytes(p, ob, self.fmt).items():
                 tot[k] += v
         return tot
 
@@ -361,21 +372,22 @@ def measure_product_only(run, steps):
     return ms / launches, launches
 
 
-def measure_base3(dev, peaks, reps=5):
-    """The base-3 weight format (five codes per byte) against the 2-bit one on
-    the decode workloads, each over distinct weight copies of at least 4x the
-    L2: microseconds per forward of the whole fused forward and of the product
-    alone (codes precomputed), and the GB/s of each format's own bytes."""
+def measure_formats(dev, peaks, reps=5):
+    """The base-3 weight format (five codes per byte) and the W1A4 regime
+    (one bit per weight, 4-bit activation codes) against the 2-bit ternary
+    format on the decode workloads, each over distinct weight copies of at
+    least 4x the L2: microseconds per forward of the whole fused forward and of
+    the product alone (codes precomputed), and the GB/s of each format's own
+    bytes."""
     out = {}
     for name in ("decode_gemv_2560x6912_t1", "decode_block_4096_t1",
                  "large_gemv_8192x28672_t1", "large_gemv_8192x28672_t8"):
         wl = WORKLOADS[name]
         res = {}
-        for fmt in ("2bit", "base3"):
-            b3 = fmt == "base3"
-            per = sum(decode_bytes(p, base3=b3)["weights"] for p in wl.problems)
+        for fmt in ("2bit", "base3", "w1"):
+            per = sum(decode_bytes(p, fmt=fmt)["weights"] for p in wl.problems)
             layers = max(len(wl.problems), int(np.ceil(4 * L2_BYTES / per)) * len(wl.problems))
-            r = DecodeRun(wl.problems, layers, dev, base3=b3)
+            r = DecodeRun(wl.problems, layers, dev, fmt=fmt)
             g = capture(lambda: [r.step() for _ in range(reps)])
             time_graph(g)
             t = time_graph(g) / reps / len(r.layers)
@@ -393,10 +405,11 @@ def measure_base3(dev, peaks, reps=5):
                         "weight_bytes_per_forward": b["weights"] // n}
             del r, g, gp
             torch.cuda.empty_cache()
-        res["speedup_forward"] = round(res["2bit"]["us_per_forward"] /
-                                       res["base3"]["us_per_forward"], 3)
-        res["speedup_product_only"] = round(res["2bit"]["us_product_only"] /
-                                            res["base3"]["us_product_only"], 3)
+        for fmt in ("base3", "w1"):
+            res[fmt]["speedup_forward_vs_2bit"] = round(res["2bit"]["us_per_forward"] /
+                                                        res[fmt]["us_per_forward"], 3)
+            res[fmt]["speedup_product_vs_2bit"] = round(res["2bit"]["us_product_only"] /
+                                                        res[fmt]["us_product_only"], 3)
         out[name] = res
     return out
 
@@ -669,8 +682,8 @@ def main():
                     help="headline only (no prefill / other decode workloads)")
     ap.add_argument("--only-prefill", action="store_true",
                     help="time the prefill forward alone and print its JSON object")
-    ap.add_argument("--only-base3", action="store_true",
-                    help="time the base-3 and 2-bit decode formats alone, print their JSON")
+    ap.add_argument("--only-formats", action="store_true",
+                    help="time the 2-bit, base-3 and W1A4 decode formats alone, print their JSON")
     args = ap.parse_args()
     warmup = max(args.warmup, 3)
     rank, world, local = dist_init(args.gpus)
@@ -694,10 +707,10 @@ def main():
             barrier(world)
             dist.destroy_process_group()
         return
-    if args.only_base3:
-        res = measure_base3(dev, peaks)
+    if args.only_formats:
+        res = measure_formats(dev, peaks)
         if rank == 0:
-            print(json.dumps({"base3": res}), flush=True)
+            print(json.dumps({"weight_formats": res}), flush=True)
         if world > 1:
             import torch.distributed as dist
             barrier(world)
@@ -762,7 +775,7 @@ def main():
             torch.cuda.empty_cache()
         extras["decode_other"] = other
         sampler.mark(True)
-        extras["base3"] = measure_base3(dev, peaks)
+        extras["weight_formats"] = measure_formats(dev, peaks)
         sampler.mark(False)
         sampler.mark(True)
         extras["backward_ste"] = measure_backward(10, dev, peaks)
