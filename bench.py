@@ -480,9 +480,10 @@ def measure_prefill(steps, warmup, dev, peaks):
 
 def measure_backward(steps, dev, peaks):
     """The straight-through-estimator backward at the prefill shape (dX and
-    dW: two tcgen05 bf16 GEMMs plus the operand transposes), one call at a
-    time after an L2 flush; beside it the dense bf16 layer's two gradient
-    GEMMs with operands already transposed (its weights kept in bf16)."""
+    dW: the bf16 expansion of W~ and dequantisation of X^, then two tcgen05
+    bf16 GEMMs that read their operands in place), one call at a time after
+    an L2 flush; beside it the dense bf16 layer's two gradient GEMMs with
+    operands already in their K-major form (its weights kept in bf16)."""
     import ternary_weight_linear_bitlinear_b200 as bl
     p = WORKLOADS["prefill_2048x4096x11008"].problems[0]
     T, N, K = p.tokens, p.d_out, p.d_in
@@ -531,7 +532,7 @@ def measure_backward(steps, dev, peaks):
                          "peak_source": peaks["source"] + " bf16 burst"},
             "dense_bf16_gemms_ms": round(ms_dense, 4),
             "overhead_vs_dense": round(ms / ms_dense, 3),
-            "gpu_launches": 5 * steps}
+            "gpu_launches": 4 * steps}
 
 
 # ------------------------------------------------------- bf16 context ---

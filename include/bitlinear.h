@@ -393,8 +393,9 @@ int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, int64_t d_in,
  *   dX, dW          out: fp32 or bf16 (out_dtype), row-major, 16-byte aligned;
  *                   either may be NULL (not computed), not both.
  *   workspace       device scratch of bitlinear_backward_workspace_bytes()
- *                   bytes, 256-byte aligned, owned by the caller (the
- *                   transposed operands: W~^T, X^^T and dY^T in bf16).
+ *                   bytes, 256-byte aligned, owned by the caller (W~ and
+ *                   X^ in bf16; the tensor-core GEMMs read them and dY in
+ *                   their row-major layouts, without transposes).
  * X^ enters the dW product as bf16 of fl32(q * fl32(beta / 127)); products
  * and sums in fp32, gamma applied once to the fp32 sum.  Shapes: d_out a
  * multiple of 256 and at most 65536, d_in as above, 0 <= T <= 65536 (T = 0

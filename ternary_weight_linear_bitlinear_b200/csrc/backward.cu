@@ -11,14 +11,13 @@
 //                                          weights)
 //
 // Both are dense contractions, run on the tcgen05 bf16 GEMM of
-// dense_bf16.cu with gamma applied in its fp32 epilogue.  Three
-// memory-bound kernels put the operands in the K-major form it reads:
-//   * expand_ternary_t_kernel: the packed codes -> W~^T as bf16 {-1, 0, 1}
-//     (exact), [d_in][d_out];
-//   * dequant_t_kernel: X~ and beta -> X^^T as bf16 of fl32(q fl32(beta/127)),
-//     [d_in][Tp], zero for the padded tokens t >= T;
-//   * transpose_bf16_kernel: dY -> dY^T, [d_out][Tp], zero-padded likewise;
-// Tp = T rounded up to 256 (the GEMM's reduction granule).
+// dense_bf16.cu with gamma applied in its fp32 epilogue and the operands read
+// in their natural layouts (MN-major where the reduction index is the row):
+//   * dX: A = W~ [d_out][d_in] as bf16 {-1, 0, 1} (exact; expand_ternary_kernel
+//     writes it from the packed codes), read MN-major; B = dY [T][d_out];
+//   * dW: A = X^ [T][d_in] as bf16 of fl32(q fl32(beta / 127))
+//     (dequant_kernel), B = dY [T][d_out], both read MN-major; the copies
+//     zero-fill the token rows past T.
 #include <cstdint>
 
 #include <cuda_bf16.h>
@@ -33,114 +32,83 @@ bitlinear_status launch_dense_bf16(const uint16_t *W, int64_t d_out, int64_t d_i
                                    const uint16_t *X, int64_t T, void *Y, int out_dtype,
                                    const float *alpha, cudaStream_t stream);
 
-constexpr int kTrThreads = 256;
-constexpr int kTrTile = 64;          // 64 x 64 element tiles
-constexpr int kTrPad = 8;            // row padding of the shared tile (elements)
+bitlinear_status launch_dense_gemm_mn(const uint16_t *A, bool a_mn, const uint16_t *B, bool b_mn,
+                                      int64_t M, int64_t N, int64_t K, void *Y, int out_dtype,
+                                      const float *alpha, cudaStream_t stream);
 
-// W~^T: one CTA per 64 weight rows (four 16-row tiles) x one 256-column
-// k-block.  Thread i decodes row i mod 64's words kw = i / 64 (+ 4, 8, 12):
-// word kw holds columns 16 kw + 4 s + b in bits 8 b + 2 s as W~ + 1.
-__global__ void __launch_bounds__(kTrThreads)
-expand_ternary_t_kernel(const uint32_t *__restrict__ packed, int d_out, int kb_total,
-                        uint16_t *__restrict__ wt) {
-    __shared__ __align__(16) uint16_t tile[256][kTrTile + kTrPad];   // [column][row]
-    const int kb = blockIdx.y;
-    const int row0 = blockIdx.x * kTrTile;
-    const int row = threadIdx.x % kTrTile, kwq = threadIdx.x / kTrTile;
-    const int o = row0 + row;
-    const uint32_t *tile_words = packed + ((size_t)(o >> 4) * kb_total + kb) * 256 + (o & 15) * 16;
-    const uint16_t lut[3] = {0xBF80u, 0x0000u, 0x3F80u};   // bf16 of -1, 0, +1
-    #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int kw = kwq + 4 * i;
-        const uint32_t w = __ldg(tile_words + kw);
+constexpr int kBwThreads = 256;
+
+// W~ as bf16, [d_out][d_in]: one thread per packed word (16 weights of one
+// row); word kw of a tile row holds columns 16 kw + 4 s + b in bits 8 b + 2 s
+// as W~ + 1, so the 16 values are written as 32 contiguous bytes.
+__global__ void __launch_bounds__(kBwThreads)
+expand_ternary_kernel(const uint32_t *__restrict__ packed, int64_t d_out, int kb_total,
+                      uint16_t *__restrict__ wt) {
+    const int64_t nwords = d_out * kb_total * 16;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t d_in = (int64_t)kb_total * 256;
+    for (int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < nwords; wi += stride) {
+        const int64_t tile = wi >> 8;
+        const int within = (int)(wi & 255);
+        const int r = within >> 4, kw = within & 15;
+        const int64_t rb = tile / kb_total, kb = tile - rb * kb_total;
+        const uint32_t w = __ldg(packed + wi);
+        uint32_t v[8];   // bf16 pairs of columns 16 kw + 2 i, 2 i + 1
         #pragma unroll
-        for (int s = 0; s < 4; ++s)
+        for (int i = 0; i < 8; ++i) {
+            uint32_t h[2];
             #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const uint32_t c = (w >> (8 * b + 2 * s)) & 3u;
-                tile[16 * kw + 4 * s + b][row] = c < 3 ? lut[c] : (uint16_t)0x7FC0u;
+            for (int e = 0; e < 2; ++e) {
+                const int col = 2 * i + e, s = col >> 2, b = col & 3;
+                const uint32_t c = (w >> (8 * b + 2 * s)) & 3u;     // W~ + 1
+                h[e] = c == 1u ? 0u : (c == 0u ? 0xBF80u : 0x3F80u);  // bf16 -1, 0, +1
             }
-    }
-    __syncthreads();
-    // Each output row k holds 64 consecutive weight rows: 128 bytes.
-    #pragma unroll
-    for (int p = 0; p < 256 * kTrTile * 2 / (16 * kTrThreads); ++p) {
-        const int idx = p * kTrThreads + threadIdx.x;
-        const int col = idx >> 3, chunk = idx & 7;
-        const uint4 v = *reinterpret_cast<const uint4 *>(&tile[col][chunk * 8]);
-        *reinterpret_cast<uint4 *>(wt + (size_t)(kb * 256 + col) * d_out + row0 + chunk * 8) = v;
+            v[i] = h[0] | (h[1] << 16);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(wt + (rb * 16 + r) * d_in + kb * 256 + kw * 16);
+        dst[0] = make_uint4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_uint4(v[4], v[5], v[6], v[7]);
     }
 }
 
-// X^^T: one CTA per 64 tokens x 64 columns.
-__global__ void __launch_bounds__(kTrThreads)
-dequant_t_kernel(const int8_t *__restrict__ xq, const float *__restrict__ beta, int T, int K,
-                 int Tp, uint16_t *__restrict__ xt) {
-    __shared__ __align__(16) uint16_t tile[kTrTile][kTrTile + kTrPad];   // [k][t]
-    const int t0 = blockIdx.y * kTrTile, k0 = blockIdx.x * kTrTile;
-    const int tl = threadIdx.x / 4, kc = (threadIdx.x % 4) * 16;
-    const int t = t0 + tl;
-    uint4 q = make_uint4(0, 0, 0, 0);
-    float sc = 0.0f;
-    if (t < T) {
-        q = __ldg(reinterpret_cast<const uint4 *>(xq + (size_t)t * K + k0 + kc));
-        sc = __fdiv_rn(beta[t], 127.0f);
-    }
-    const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-    #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const int code = (int)(int8_t)((qw[j >> 2] >> (8 * (j & 3))) & 0xFFu);
-        const float v = __fmul_rn((float)code, sc);
-        tile[kc + j][tl] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-    }
-    __syncthreads();
-    #pragma unroll
-    for (int p = 0; p < kTrTile * kTrTile * 2 / (16 * kTrThreads); ++p) {
-        const int idx = p * kTrThreads + threadIdx.x;
-        const int k = idx >> 3, chunk = idx & 7;
-        const uint4 v = *reinterpret_cast<const uint4 *>(&tile[k][chunk * 8]);
-        *reinterpret_cast<uint4 *>(xt + (size_t)(k0 + k) * Tp + t0 + chunk * 8) = v;
-    }
-}
-
-// dY^T: one CTA per 64 tokens x 64 outputs.
-__global__ void __launch_bounds__(kTrThreads)
-transpose_bf16_kernel(const uint16_t *__restrict__ dy, int T, int N, int Tp,
-                      uint16_t *__restrict__ dyt) {
-    __shared__ __align__(16) uint16_t tile[kTrTile][kTrTile + kTrPad];   // [n][t]
-    const int t0 = blockIdx.y * kTrTile, n0 = blockIdx.x * kTrTile;
-    const int tl = threadIdx.x / 8, nc = (threadIdx.x % 8) * 8;
-    #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int tt = tl + 32 * h, t = t0 + tt;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (t < T) v = __ldg(reinterpret_cast<const uint4 *>(dy + (size_t)t * N + n0 + nc));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// X^ as bf16, [T][d_in]: one thread per 16 codes of one token.
+__global__ void __launch_bounds__(kBwThreads)
+dequant_kernel(const int8_t *__restrict__ xq, const float *__restrict__ beta, int64_t T, int K,
+               uint16_t *__restrict__ xh) {
+    const int64_t nvec = T * (K / 16);
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t vi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; vi < nvec; vi += stride) {
+        const int64_t t = vi / (K / 16);
+        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(xq) + vi);
+        const float sc = __fdiv_rn(beta[t], 127.0f);
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+        uint32_t v[8];
         #pragma unroll
-        for (int j = 0; j < 8; ++j) tile[nc + j][tt] = (uint16_t)(w[j >> 1] >> (16 * (j & 1)));
-    }
-    __syncthreads();
-    #pragma unroll
-    for (int p = 0; p < kTrTile * kTrTile * 2 / (16 * kTrThreads); ++p) {
-        const int idx = p * kTrThreads + threadIdx.x;
-        const int n = idx >> 3, chunk = idx & 7;
-        const uint4 v = *reinterpret_cast<const uint4 *>(&tile[n][chunk * 8]);
-        *reinterpret_cast<uint4 *>(dyt + (size_t)(n0 + n) * Tp + t0 + chunk * 8) = v;
+        for (int i = 0; i < 8; ++i) {
+            uint32_t h[2];
+            #pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int j = 2 * i + e;
+                const int code = (int)(int8_t)((qw[j >> 2] >> (8 * (j & 3))) & 0xFFu);
+                h[e] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)code, sc)));
+            }
+            v[i] = h[0] | (h[1] << 16);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(xh) + vi * 2;
+        dst[0] = make_uint4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_uint4(v[4], v[5], v[6], v[7]);
     }
 }
 
 static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 struct BackwardLayout {
-    size_t wt, xt, dyt, total;   // byte offsets of the three operands, total bytes
-    int64_t tp;
+    size_t wt, xh, total;   // byte offsets of the two bf16 operands, total bytes
 };
 
 static BackwardLayout backward_layout(int64_t d_out, int64_t d_in, int64_t T, bool want_dx,
                                       bool want_dw) {
     BackwardLayout l = {};
-    l.tp = round_up(T > 0 ? T : 1, 256);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t at = off;
@@ -148,8 +116,7 @@ static BackwardLayout backward_layout(int64_t d_out, int64_t d_in, int64_t T, bo
         return at;
     };
     l.wt = want_dx ? take((size_t)d_in * d_out * 2) : 0;
-    l.xt = want_dw ? take((size_t)d_in * l.tp * 2) : 0;
-    l.dyt = want_dw ? take((size_t)d_out * l.tp * 2) : 0;
+    l.xh = want_dw ? take((size_t)d_in * (T > 0 ? T : 1) * 2) : 0;
     l.total = off;
     return l;
 }
@@ -197,26 +164,28 @@ extern "C" int bitlinear_backward(const uint32_t *packed, const float *gamma, in
     }
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const int kb_total = (int)(d_in / 256);
+    auto grid_for = [](int64_t items) {
+        int64_t b = (items + kBwThreads - 1) / kBwThreads;
+        return (unsigned)(b > 148 * 16 ? 148 * 16 : b);
+    };
     if (want_dx) {
         uint16_t *wt = reinterpret_cast<uint16_t *>(ws + lay.wt);
-        expand_ternary_t_kernel<<<dim3((unsigned)(d_out / kTrTile), (unsigned)kb_total), kTrThreads,
-                                  0, stream>>>(packed, (int)d_out, kb_total, wt);
+        expand_ternary_kernel<<<grid_for(d_out * d_in / 16), kBwThreads, 0, stream>>>(
+            packed, d_out, kb_total, wt);
         if (cudaGetLastError() != cudaSuccess) return BITLINEAR_ERR_CUDA;
-        // dX[t][k] = gamma sum_o dY[t][o] W~^T[k][o]
-        st = launch_dense_bf16(wt, d_in, d_out, dY, T, dX, out_dtype, gamma, stream);
+        // dX[t][k] = gamma sum_o dY[t][o] W~[o][k]: A = W~ read MN-major (M = d_in).
+        st = launch_dense_gemm_mn(wt, true, dY, false, d_in, T, d_out, dX, out_dtype, gamma,
+                                  stream);
         if (st != BITLINEAR_OK) return st;
     }
     if (want_dw) {
-        uint16_t *xt = reinterpret_cast<uint16_t *>(ws + lay.xt);
-        uint16_t *dyt = reinterpret_cast<uint16_t *>(ws + lay.dyt);
-        const unsigned tb = (unsigned)(lay.tp / kTrTile);
-        dequant_t_kernel<<<dim3((unsigned)(d_in / kTrTile), tb), kTrThreads, 0, stream>>>(
-            Xq, beta, (int)T, (int)d_in, (int)lay.tp, xt);
-        transpose_bf16_kernel<<<dim3((unsigned)(d_out / kTrTile), tb), kTrThreads, 0, stream>>>(
-            dY, (int)T, (int)d_out, (int)lay.tp, dyt);
+        uint16_t *xh = reinterpret_cast<uint16_t *>(ws + lay.xh);
+        dequant_kernel<<<grid_for(T * d_in / 16), kBwThreads, 0, stream>>>(Xq, beta, T, (int)d_in,
+                                                                           xh);
         if (cudaGetLastError() != cudaSuccess) return BITLINEAR_ERR_CUDA;
-        // dW[o][k] = gamma sum_t dY^T[o][t] X^^T[k][t]
-        st = launch_dense_bf16(xt, d_in, lay.tp, dyt, d_out, dW, out_dtype, gamma, stream);
+        // dW[o][k] = gamma sum_t dY[t][o] X^[t][k]: both read MN-major (M = d_in, N = d_out).
+        st = launch_dense_gemm_mn(xh, true, dY, true, d_in, d_out, T, dW, out_dtype, gamma,
+                                  stream);
         if (st != BITLINEAR_OK) return st;
     }
     return BITLINEAR_OK;

@@ -20,6 +20,7 @@
 //     finished accumulator, round it and write it with TMA tensor stores
 //     while the next tile accumulates.  Every mbarrier wait is bounded.
 #include <cstdint>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -139,8 +140,13 @@ struct __align__(8) DenseBarriers {
     int abort_flag;
 };
 constexpr int kDSmemBytes = kDStages * kDStageBytes + kDOutBytes + 1024 + 1024;
+constexpr int kDPanel = 64;                   // MN-elements of one MN-major panel (128 bytes)
+constexpr int kDPanelBytes = kDPanel * 128;   // 64 K-rows of 128 bytes per stage and panel
 
-template <bool OUT_BF16>
+// D[m][n] = sum_k A[m][k] B[n][k] (A: M = d_out rows, B: N = T rows, K = d_in),
+// stored as Y[n][m].  A_MN / B_MN: the operand is stored MN-major, i.e. as
+// [k][m] / [k][n] in memory, loaded as 64-element panels (no transpose pass).
+template <bool OUT_BF16, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kDThreads, 1)
 dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
                   const __grid_constant__ CUtensorMap map_y, int d_out, int d_in, int T,
@@ -157,7 +163,7 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = (d_out + kDM - 1) / kDM;
     const int num_tiles = m_tiles * ((T + kDN - 1) / kDN);
-    const int num_k = d_in / kDKE;
+    const int num_k = (d_in + kDKE - 1) / kDKE;   // MN-major K edges are zero-filled by the copy
     volatile int *abort_flag = &bars->abort_flag;
 
     if (threadIdx.x == 0) {
@@ -198,8 +204,22 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
                     }
                     const uint32_t fb = smem_u32(&bars->full[s]);
                     mbar_arrive_expect_tx(fb, kDStageBytes);
-                    tma_load_2d(stage_a(s), &map_w, kt * kDKE, m0, fb);
-                    tma_load_2d(stage_b(s), &map_x, kt * kDKE, n0, fb);
+                    if constexpr (A_MN) {
+                        #pragma unroll
+                        for (int p = 0; p < kDM / kDPanel; ++p)
+                            tma_load_2d(stage_a(s) + p * kDPanelBytes, &map_w, m0 + p * kDPanel,
+                                        kt * kDKE, fb);
+                    } else {
+                        tma_load_2d(stage_a(s), &map_w, kt * kDKE, m0, fb);
+                    }
+                    if constexpr (B_MN) {
+                        #pragma unroll
+                        for (int p = 0; p < kDN / kDPanel; ++p)
+                            tma_load_2d(stage_b(s) + p * kDPanelBytes, &map_x, n0 + p * kDPanel,
+                                        kt * kDKE, fb);
+                    } else {
+                        tma_load_2d(stage_b(s), &map_x, kt * kDKE, n0, fb);
+                    }
                     ++step;
                     if (++s == kDStages) { s = 0; ph ^= 1u; }
                 }
@@ -212,7 +232,7 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ---
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(kDM, kDN);
+            constexpr uint32_t idesc = idesc_bf16(kDM, kDN, A_MN, B_MN);
             int s = 0, i = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -230,10 +250,17 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
                     }
                     tc_fence_after();
                     #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)   // K = 16 bf16 (32 bytes) per MMA
-                        tc_mma_f16_ss(tmem_acc, smem_desc_sw128(stage_a(s) + kk * 32),
-                                      smem_desc_sw128(stage_b(s) + kk * 32), idesc,
-                                      (kt > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {   // K = 16 bf16 per MMA
+                        // K-major: 32 bytes along each 128-byte row; MN-major:
+                        // 16 K-rows of every panel (two 1024-byte atoms).
+                        const uint64_t da =
+                            A_MN ? smem_desc_sw128_mn(stage_a(s) + kk * 2048, kDPanelBytes)
+                                 : smem_desc_sw128(stage_a(s) + kk * 32);
+                        const uint64_t db =
+                            B_MN ? smem_desc_sw128_mn(stage_b(s) + kk * 2048, kDPanelBytes)
+                                 : smem_desc_sw128(stage_b(s) + kk * 32);
+                        tc_mma_f16_ss(tmem_acc, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                    }
                     tc_commit(smem_u32(&bars->empty[s]));
                     if (++s == kDStages) { s = 0; ph ^= 1u; }
                 }
@@ -316,9 +343,12 @@ static cudaError_t launch_dense_gemv_t(const uint16_t *W, int64_t d_out, int64_t
     return cudaGetLastError();
 }
 
+// A: [d_out][d_in] (K-major) or [d_in][d_out] (a_mn); B: [T][d_in] or
+// [d_in][T] (b_mn).  Y[T][d_out].
 static bitlinear_status launch_dense_gemm(const uint16_t *W, int64_t d_out, int64_t d_in,
                                           const uint16_t *X, int64_t T, void *Y, bool bf,
-                                          const float *alpha, cudaStream_t stream) {
+                                          const float *alpha, cudaStream_t stream,
+                                          bool a_mn = false, bool b_mn = false) {
     PFN_encodeTiled encode = get_encode_fn();
     if (!encode) return BITLINEAR_ERR_CUDA;
     DeviceCtx ctx;
@@ -327,9 +357,10 @@ static bitlinear_status launch_dense_gemm(const uint16_t *W, int64_t d_out, int6
     CUtensorMap map_w, map_x, map_y;
     const cuuint32_t estr[2] = {1, 1};
     {
-        const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)d_out};
-        const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
-        const cuuint32_t box[2] = {kDKE, kDM};
+        const cuuint64_t dims[2] = {(cuuint64_t)(a_mn ? d_out : d_in), (cuuint64_t)(a_mn ? d_in : d_out)};
+        const cuuint64_t strides[1] = {(cuuint64_t)(a_mn ? d_out : d_in) * 2};
+        const cuuint32_t box[2] = {a_mn ? (cuuint32_t)kDPanel : (cuuint32_t)kDKE,
+                                   a_mn ? (cuuint32_t)kDKE : (cuuint32_t)kDM};
         if (encode(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(W), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -337,9 +368,10 @@ static bitlinear_status launch_dense_gemm(const uint16_t *W, int64_t d_out, int6
             return BITLINEAR_ERR_CUDA;
     }
     {
-        const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)T};
-        const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
-        const cuuint32_t box[2] = {kDKE, kDN};
+        const cuuint64_t dims[2] = {(cuuint64_t)(b_mn ? T : d_in), (cuuint64_t)(b_mn ? d_in : T)};
+        const cuuint64_t strides[1] = {(cuuint64_t)(b_mn ? T : d_in) * 2};
+        const cuuint32_t box[2] = {b_mn ? (cuuint32_t)kDPanel : (cuuint32_t)kDKE,
+                                   b_mn ? (cuuint32_t)kDKE : (cuuint32_t)kDN};
         if (encode(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(X), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -357,7 +389,14 @@ static bitlinear_status launch_dense_gemm(const uint16_t *W, int64_t d_out, int6
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BITLINEAR_ERR_CUDA;
     }
-    auto kern = bf ? dense_gemm_kernel<true> : dense_gemm_kernel<false>;
+    auto pick = [&](auto bf_tag) {
+        constexpr bool B = decltype(bf_tag)::value;
+        if (a_mn && b_mn) return dense_gemm_kernel<B, true, true>;
+        if (a_mn) return dense_gemm_kernel<B, true, false>;
+        if (b_mn) return dense_gemm_kernel<B, false, true>;
+        return dense_gemm_kernel<B, false, false>;
+    };
+    auto kern = bf ? pick(std::true_type{}) : pick(std::false_type{});
     if (ensure_dynamic_smem((const void *)kern, kDSmemBytes) != cudaSuccess)
         return BITLINEAR_ERR_CUDA;
     int dev = 0, sms = 148;
@@ -368,6 +407,15 @@ static bitlinear_status launch_dense_gemm(const uint16_t *W, int64_t d_out, int6
     kern<<<grid, kDThreads, kDSmemBytes, stream>>>(map_w, map_x, map_y, (int)d_out, (int)d_in,
                                                    (int)T, alpha, ctx);
     return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+// The tcgen05 GEMM with MN-major operands (see launch_dense_gemm): used by the
+// backward pass so that dY, X^ and W~ are read in their natural layouts.
+bitlinear_status launch_dense_gemm_mn(const uint16_t *A, bool a_mn, const uint16_t *B, bool b_mn,
+                                      int64_t M, int64_t N, int64_t K, void *Y, int out_dtype,
+                                      const float *alpha, cudaStream_t stream) {
+    return launch_dense_gemm(A, M, K, B, N, Y, out_dtype == BITLINEAR_OUT_BF16, alpha, stream,
+                             a_mn, b_mn);
 }
 
 // alpha: optional device scalar multiplying every output (in fp32, once).

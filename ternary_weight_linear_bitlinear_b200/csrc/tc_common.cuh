@@ -215,13 +215,32 @@ __device__ __forceinline__ void tc_mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, 
         : "memory");
 }
 
-// Instruction descriptor, kind::f16: D f32, A and B bf16, both K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+// Instruction descriptor, kind::f16: D f32, A and B bf16; a_mn / b_mn mark
+// an operand stored MN-major (its M or N index contiguous) instead of K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool a_mn = false,
+                                                  bool b_mn = false) {
     return (1u << 4)                       // D format f32
            | (1u << 7)                     // A bf16
            | (1u << 10)                    // B bf16
+           | ((a_mn ? 1u : 0u) << 15)      // A major: 0 K, 1 MN
+           | ((b_mn ? 1u : 0u) << 16)      // B major: 0 K, 1 MN
            | ((uint32_t)(n >> 3) << 17)    // N / 8
            | ((uint32_t)(m >> 4) << 24);   // M / 16
+}
+
+// Shared-memory matrix descriptor, MN-major operand with 128-byte swizzle:
+// panels of 64 16-bit MN-elements (128-byte rows, one row per K index, as a
+// TMA box {64, k} with 128-byte swizzle writes them), 1024-byte atoms of 8
+// K-rows (stride byte offset) and panels `panel_bytes` apart (leading byte
+// offset).  addr is the atom-aligned first K-row of the slice.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t addr, uint32_t panel_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((panel_bytes >> 4) & 0x3FFFu) << 16;   // leading byte offset: next panel
+    d |= (uint64_t)(1024u >> 4) << 32;                      // stride byte offset: next 8 K-rows
+    d |= (uint64_t)1u << 46;                                // version
+    d |= (uint64_t)2u << 61;                                // layout: 128-byte swizzle
+    return d;
 }
 
 // ------------------------------------------------------------------ host ---
