@@ -593,9 +593,10 @@ def measure_context_bf16(dev, peaks, decode_us: dict, prefill_ms: float):
 def measure_e2e(run, steps):
     """Through the public API with host buffers: every step copies its
     activations (all layers' X, one pinned host buffer) host -> device and
-    reads all its outputs back device -> host, inside the timed region; the
-    forwards are eager bitlinear_linear calls through the binding's
-    LinearPlan (arguments bound once per layer)."""
+    reads all its outputs back device -> host, inside the timed region.  The
+    step is a LinearPlan call per layer (arguments bound once), run as a
+    StepGraph (the step captured once as a CUDA graph, copies included, and
+    replayed) and, for comparison, eagerly."""
     bl = run.bl
     dev = run.dev
     xs = [X for _, _, X, _, _ in run.layers]
@@ -614,8 +615,8 @@ def measure_e2e(run, steps):
         oy += ny
     h2d = host_x.numel() * host_x.element_size()
     d2h = host_y.numel() * host_y.element_size()
-    s = torch.cuda.current_stream()
-    plans = [bl.LinearPlan(w, X.shape[0], out=Y, scratch=scratch, static_weights=True)
+    cs = torch.cuda.Stream()
+    plans = [bl.LinearPlan(w, X.shape[0], out=Y, scratch=scratch, static_weights=True, stream=cs)
              for (_, w, _, scratch, _), X, Y in zip(run.layers, x_views, y_views)]
 
     def one():
@@ -624,15 +625,25 @@ def measure_e2e(run, steps):
             plan(X)
         host_y.copy_(dev_y, non_blocking=True)
 
-    one()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(s)
-    for _ in range(steps):
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(cs)
+        for _ in range(steps):
+            fn()
+        b.record(cs)
+        b.synchronize()
+        return a.elapsed_time(b) / steps
+
+    with torch.cuda.stream(cs):
         one()
-    b.record(s)
-    b.synchronize()
-    return a.elapsed_time(b) / steps, h2d, d2h
+        torch.cuda.synchronize()
+        ms_eager = timed(one)
+        step = bl.StepGraph(one, stream=cs)
+        step()
+        ms_graph = timed(step)
+    return ms_graph, ms_eager, h2d, d2h
+
 
 
 # -------------------------------------------------------- CPU oracle ---
@@ -788,8 +799,9 @@ def main():
             extras["prefill"]["ms_gemm"])
         sampler.mark(False)
 
-    e2e_ms, h2d, d2h = measure_e2e(run, max(3, min(args.steps, 20)))
+    e2e_ms, e2e_eager_ms, h2d, d2h = measure_e2e(run, max(3, min(args.steps, 20)))
     e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_eager_ms = max_over_ranks(e2e_eager_ms, world)
     sampler.stop()
     status = run.bl.device_error(clear=True)
 
@@ -837,9 +849,12 @@ def main():
             "e2e": {"value": round(replica_value(nb["step"], world, e2e_ms), 3),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 4),
-                    "how": "public Python API (LinearPlan per layer: eager bitlinear_linear "
-                           "calls), every step one copy of all its X in from pinned host memory "
-                           "and one of all its Y out"},
+                    "eager": {"value": round(replica_value(nb["step"], world, e2e_eager_ms), 3),
+                              "ms_per_step": round(e2e_eager_ms, 4)},
+                    "how": "public Python API: a LinearPlan per layer (bitlinear_linear with "
+                           "bound arguments), the step replayed as a StepGraph (CUDA graph of "
+                           "the copies and the calls); every step one copy of all its X in "
+                           "from pinned host memory and one of all its Y out"},
             "gpu_launches": (1 if one_kernel else 2) * len(run.layers) * args.steps,
             "clocks": clocks,
             "device_error": run.bl.status_string(status),

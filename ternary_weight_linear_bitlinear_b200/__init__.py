@@ -345,14 +345,15 @@ def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
 class LinearPlan:
     """bitlinear_linear with everything but X bound once: the weights, the
     scratch (Xq, beta, rowsum), the output, the flags and the CUDA stream
-    current at construction.  Each call passes X's address to the same
+    (`stream`, default: the one current at construction).  Each call passes X's address to the same
     entry point and returns the bound output tensor (overwritten by the next
     call).  For a serving loop that calls the same layer shape repeatedly."""
 
     def __init__(self, w, T: int, gain: torch.Tensor = None, rmsnorm: bool = True,
                  eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.bfloat16,
                  out: torch.Tensor = None, scratch=None, static_weights: bool = False,
-                 per_tensor: bool = False, device=None, act_bits: int = 8):
+                 per_tensor: bool = False, device=None, act_bits: int = 8,
+                 stream: torch.cuda.Stream = None):
         dev = device if device is not None else w.packed.device
         if scratch is None:
             scratch = (torch.empty((T, w.d_in), dtype=torch.int8, device=dev),
@@ -371,8 +372,9 @@ class LinearPlan:
         self._shape = (T, w.d_in)
         self._fn, self._name = _entry(w, "bitlinear_linear")
         self._pre = (w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in)
+        sh = stream.cuda_stream if stream is not None else _stream()
         self._post = (T, _ptr(gain), flags, eps, norm_eps, Xq.data_ptr(), beta.data_ptr(),
-                      rowsum.data_ptr(), out.data_ptr(), od, _stream())
+                      rowsum.data_ptr(), out.data_ptr(), od, sh)
 
     def __call__(self, X: torch.Tensor) -> torch.Tensor:
         if X.dtype != torch.bfloat16 or tuple(X.shape) != self._shape or not X.is_contiguous():
@@ -381,6 +383,33 @@ class LinearPlan:
         if st != OK:
             raise BitLinearError(st, self._name)
         return self.out
+
+
+class StepGraph:
+    """A serving step captured once as a CUDA graph and replayed per call.
+
+    fn() enqueues the step's work on the current stream: typically a copy of
+    the step's inputs from pinned host memory into fixed device buffers, the
+    LinearPlan calls of the layers, and a copy of the outputs back to pinned
+    host memory.  Every address it uses must stay valid and fixed; a replay
+    re-runs the same kernels and copies (the host buffers' current contents
+    go in, the new outputs come out).  fn is captured on `stream` (default:
+    a new stream), so LinearPlans called inside it must be bound to that
+    stream; it runs once eagerly on the same stream before the capture."""
+
+    def __init__(self, fn, stream: torch.cuda.Stream = None):
+        self.stream = stream if stream is not None else torch.cuda.Stream()
+        self.stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.stream):
+            fn()
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            fn()
+        torch.cuda.synchronize()
+
+    def __call__(self):
+        self.graph.replay()
 
 
 def backward(w: PackedTernary, Xq: torch.Tensor, beta: torch.Tensor, dY: torch.Tensor,

@@ -407,3 +407,35 @@ def test_linear_plan_matches_linear():
     assert torch.equal(got, ref)
     with pytest.raises(TypeError):
         plan(Xd.float())
+
+
+def test_step_graph_replays_copies_and_calls():
+    """A StepGraph of (pinned host X -> device, LinearPlan, device Y -> pinned
+    host) gives, for new host contents on every replay, the same bits as an
+    eager bl.linear of those contents."""
+    d_out, d_in = 2560, 1024
+    W, X = draw(Problem("sg", d_in, d_out, 2, 0.02, 0.01, 50.0, 14))
+    w = bl.pack_weights(W.to(dev()), EPS)
+    cs = torch.cuda.Stream()
+    host_x = torch.empty((2, d_in), dtype=torch.bfloat16).pin_memory()
+    host_y = torch.empty((2, d_out), dtype=torch.bfloat16).pin_memory()
+    dev_x = torch.empty((2, d_in), dtype=torch.bfloat16, device=dev())
+    plan = bl.LinearPlan(w, 2, out_dtype=torch.bfloat16, static_weights=True, stream=cs)
+
+    def step():
+        dev_x.copy_(host_x, non_blocking=True)
+        plan(dev_x)
+        host_y.copy_(plan.out, non_blocking=True)
+
+    host_x.copy_(X)
+    g = bl.StepGraph(step, stream=cs)
+    gen = torch.Generator().manual_seed(5)
+    for _ in range(3):
+        xnew = (torch.randn(2, d_in, generator=gen) * 3).to(torch.bfloat16)
+        host_x.copy_(xnew)
+        with torch.cuda.stream(cs):
+            g()
+        cs.synchronize()
+        ref = bl.linear(w, xnew.to(dev()), out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert torch.equal(host_y, ref.cpu())
