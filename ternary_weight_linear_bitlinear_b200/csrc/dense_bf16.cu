@@ -15,7 +15,10 @@
 //   * dense_gemm_kernel (T > 16): a persistent tcgen05 kind::f16 GEMM.  One
 //     CTA per SM walks 128 x 256 output tiles; warp 0 TMA-loads 64-column
 //     stages of W (A operand, 128 rows) and X (B operand, 256 tokens), both
-//     128-byte swizzled K-major; warp 1 issues four MMAs per stage into one
+//     128-byte swizzled, K-major -- or, for the backward pass's GEMMs,
+//     either operand MN-major (stored with the reduction index as the row,
+//     loaded as 64-element panels, no transpose pass); warp 1 issues four
+//     MMAs per stage into one
 //     of two TMEM fp32 accumulators (2 x 256 columns); warps 2..5 read a
 //     finished accumulator, round it and write it with TMA tensor stores
 //     while the next tile accumulates.  Every mbarrier wait is bounded.
