@@ -263,11 +263,13 @@ def test_gemm_bf16_out(T):
     forward_case(256, 1024, T, torch.bfloat16)
 
 
-# Many tiles per CTA (the persistent tile loop and both accumulators in turn).
+# Many tiles per CTA (the persistent tile loop and both accumulators in turn);
+# with at least one 256 x 256 tile per SM pair these run on the CTA-pair kernel.
 LARGE_GEMM_CASES = [
     (4096, 512, 1201, torch.float32),    # ragged tokens in the last tile
     (4112, 256, 1100, torch.bfloat16),   # 4112 rows: the last row tile holds 16
     (9472, 256, 512, torch.float32),
+    (8192, 256, 1800, torch.float32),    # 256 pair tiles: up to four per CTA pair
 ]
 
 
