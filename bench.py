@@ -246,7 +246,7 @@ def capture(fn):
 
 
 DECODE_SOURCES = ("gemv.cu", "quant_common.cuh", "common.cuh")
-GEMM_SOURCES = ("gemm_tc.cu", "common.cuh")
+GEMM_SOURCES = ("gemm_tc2.cu", "common.cuh", "tc_common.cuh")
 
 
 def source_sha(names):
@@ -454,7 +454,17 @@ def measure_prefill(steps, warmup, dev, peaks):
                            steps, flush)
     ms_mm = time_each(lambda: bl.forward(w, scratch[0], scratch[1], scratch[2], out=Y), steps,
                       flush)
-    del flush
+    # Context, not this library's path: the vendor int8 GEMM (cuBLASLt, through
+    # torch._int_mm) on the same shape, int8 x int8 -> int32 with the weights
+    # stored unpacked -- what this GPU's tensor cores reach on the contraction
+    # alone under the same timing.
+    g = torch.Generator().manual_seed(5)
+    w8 = torch.randint(-1, 2, (p.d_out, p.d_in), dtype=torch.int8, generator=g).to(dev)
+    for _ in range(max(warmup, 3)):   # the library picks and sets up its kernel on first use
+        torch._int_mm(scratch[0], w8.t())
+    torch.cuda.synchronize()
+    ms_lib = time_each(lambda: torch._int_mm(scratch[0], w8.t()), steps, flush)
+    del flush, w8
     ops = 2.0 * T * p.d_in * p.d_out
     tops = ops / (ms_mm * 1e-3) / 1e12
     peak = peaks["bf16"] * INT8_OVER_BF16
@@ -466,11 +476,15 @@ def measure_prefill(steps, warmup, dev, peaks):
         "ms_step_per_tensor_absmax": round(ms_step_pt, 4),
         "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(peak, 1),
                      "unit": "TFLOP/s", "frac": round(tops / peak, 4),
-                     "traffic": profile_traffic("gemm_tc_prefill_2048x4096x11008.md",
+                     "traffic": profile_traffic("gemm_tc_pair_prefill_2048x4096x11008.md",
                                                 GEMM_SOURCES),
                      "peak_source": "%s bf16 burst x %.0f (nominal int8/bf16 dense ratio)"
                                     % (peaks["source"], INT8_OVER_BF16)},
         "frac_of_datasheet_4500": round(tops / 4500.0, 4),
+        "vendor_int8_gemm_same_shape": {
+            "impl": "cuBLASLt via torch._int_mm (int8 x int8 -> int32, unpacked weights)",
+            "ms": round(ms_lib, 4), "tops": round(ops / (ms_lib * 1e-3) / 1e12, 1),
+            "ours_over_vendor": round(ms_lib / ms_mm, 3)},
         "l2": "L2 overwritten before every timed call; each call timed alone",
         "gpu_launches": 7 * steps,
     }
