@@ -246,7 +246,7 @@ def capture(fn):
 
 
 DECODE_SOURCES = ("gemv.cu", "quant_common.cuh", "common.cuh")
-GEMM_SOURCES = ("gemm_tc2.cu", "common.cuh", "tc_common.cuh")
+GEMM_SOURCES = ("gemm_tc.cu", "common.cuh", "tc_common.cuh")
 
 
 def source_sha(names):

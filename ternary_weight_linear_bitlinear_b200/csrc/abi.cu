@@ -26,10 +26,6 @@ bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int
                                      int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
                                      int out_dtype, bool static_weights, int fmt, float qmax,
                                      cudaStream_t stream);
-bitlinear_status launch_gemm_tc(const uint32_t *packed, const float *gamma, int64_t d_out,
-                                int64_t d_in, const int8_t *Xq, const float *beta,
-                                const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                                int32_t *acc_out, cudaStream_t stream);
 bitlinear_status launch_gemm_tc_pair(const uint32_t *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const int8_t *Xq, const float *beta,
                                      const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
@@ -138,14 +134,8 @@ static bitlinear_status dispatch_forward(const void *packed, const float *gamma,
     if (T <= 16 || fmt != kFmt2Bit)
         return launch_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
                            acc_out, static_weights, fmt, qmax, stream);
-    // Enough 256 x 256 tiles to give every SM pair one: the CTA-pair kernel;
-    // otherwise the single-CTA kernel, whose 128 x 256 tiles spread further.
-    const bitlinear_status st =
-        launch_gemm_tc_pair(static_cast<const uint32_t *>(packed), gamma, d_out, d_in, Xq, beta,
-                            rowsum, T, Y, out_dtype, acc_out, stream);
-    if (st != BITLINEAR_ERR_UNSUPPORTED_SHAPE) return st;
-    return launch_gemm_tc(static_cast<const uint32_t *>(packed), gamma, d_out, d_in, Xq, beta,
-                          rowsum, T, Y, out_dtype, acc_out, stream);
+    return launch_gemm_tc_pair(static_cast<const uint32_t *>(packed), gamma, d_out, d_in, Xq,
+                               beta, rowsum, T, Y, out_dtype, acc_out, stream);
 }
 
 static bitlinear_status forward_common(const void *packed, const float *gamma, int64_t d_out,

@@ -263,8 +263,8 @@ def test_gemm_bf16_out(T):
     forward_case(256, 1024, T, torch.bfloat16)
 
 
-# Many tiles per CTA (the persistent tile loop and both accumulators in turn);
-# with at least one 256 x 256 tile per SM pair these run on the CTA-pair kernel.
+# Many tiles per CTA pair (the persistent tile loop and both accumulators in
+# turn), ragged rows and tokens in the last pair tile.
 LARGE_GEMM_CASES = [
     (4096, 512, 1201, torch.float32),    # ragged tokens in the last tile
     (4112, 256, 1100, torch.bfloat16),   # 4112 rows: the last row tile holds 16
