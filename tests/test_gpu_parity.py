@@ -249,7 +249,9 @@ def test_gemv_bf16_out(T):
     forward_case(512, 512, T, torch.bfloat16)
 
 
-GEMM_SHAPES = [(128, 256), (144, 512), (272, 768), (512, 512), (384, 2560)]
+# 16 and 48 rows: the pair tile's first CTA is itself mostly past the last
+# row; 144 and 272: the second CTA's rows are partly or wholly past it.
+GEMM_SHAPES = [(16, 256), (48, 768), (128, 256), (144, 512), (272, 768), (512, 512), (384, 2560)]
 
 
 @pytest.mark.parametrize("d_out,d_in", GEMM_SHAPES)
