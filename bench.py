@@ -372,7 +372,7 @@ def measure_product_only(run, steps):
     return ms / launches, launches
 
 
-def measure_formats(dev, peaks, reps=5):
+def measure_formats(dev, peaks, reps=5, workloads=None):
     """The base-3 weight format (five codes per byte) and the W1A4 regime
     (one bit per weight, 4-bit activation codes) against the 2-bit ternary
     format on the decode workloads, each over distinct weight copies of at
@@ -380,8 +380,8 @@ def measure_formats(dev, peaks, reps=5):
     the product alone (codes precomputed), and the GB/s of each format's own
     bytes."""
     out = {}
-    for name in ("decode_gemv_2560x6912_t1", "decode_block_4096_t1",
-                 "large_gemv_8192x28672_t1", "large_gemv_8192x28672_t8"):
+    for name in workloads or ("decode_gemv_2560x6912_t1", "decode_block_4096_t1",
+                              "large_gemv_8192x28672_t1", "large_gemv_8192x28672_t8"):
         wl = WORKLOADS[name]
         res = {}
         for fmt in ("2bit", "base3", "w1"):
@@ -710,6 +710,12 @@ def main():
                     help="time the prefill forward alone and print its JSON object")
     ap.add_argument("--only-formats", action="store_true",
                     help="time the 2-bit, base-3 and W1A4 decode formats alone, print their JSON")
+    ap.add_argument("--formats-workload", default=None,
+                    choices=["decode_gemv_2560x6912_t1", "decode_block_4096_t1",
+                             "large_gemv_8192x28672_t1", "large_gemv_8192x28672_t8"],
+                    help="with --only-formats: that one decode workload")
+    ap.add_argument("--only-backward", action="store_true",
+                    help="time the straight-through-estimator backward alone, print its JSON")
     args = ap.parse_args()
     warmup = max(args.warmup, 3)
     rank, world, local = dist_init(args.gpus)
@@ -734,9 +740,19 @@ def main():
             dist.destroy_process_group()
         return
     if args.only_formats:
-        res = measure_formats(dev, peaks)
+        res = measure_formats(dev, peaks, workloads=[args.formats_workload]
+                              if args.formats_workload else None)
         if rank == 0:
             print(json.dumps({"weight_formats": res}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            barrier(world)
+            dist.destroy_process_group()
+        return
+    if args.only_backward:
+        res = measure_backward(max(3, args.steps), dev, peaks)
+        if rank == 0:
+            print(json.dumps({"backward_ste": res}), flush=True)
         if world > 1:
             import torch.distributed as dist
             barrier(world)
