@@ -218,7 +218,9 @@ int bitlinear_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
  *   acc_out    out: int32 [T][d_out] raw accumulators, or NULL.
  * T <= 16 runs the decode GEMV (register-decoded ternary weights, warp-level
  * int8 tensor-core MMA); T > 16 runs the prefill GEMM (TMA-staged packed
- * tiles expanded into tensor memory, tcgen05 int8 MMA, TMEM accumulator).
+ * tiles expanded in shared memory, tcgen05 int8 MMA on clusters of two CTAs,
+ * TMEM accumulators).  The prefill GEMM launches clusters of two CTAs of
+ * about 215 KiB of shared memory each, one pair per two SMs.
  */
 int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
                       int64_t d_in, const int8_t *Xq, const float *beta,
