@@ -458,15 +458,25 @@ def measure_prefill(steps, warmup, dev, peaks):
     # torch._int_mm) on the same shape, int8 x int8 -> int32 with the weights
     # stored unpacked -- what this GPU's tensor cores reach on the contraction
     # alone under the same timing.
-    g = torch.Generator().manual_seed(5)
-    w8 = torch.randint(-1, 2, (p.d_out, p.d_in), dtype=torch.int8, generator=g).to(dev)
-    for _ in range(max(warmup, 3)):   # the library picks and sets up its kernel on first use
-        torch._int_mm(scratch[0], w8.t())
-    torch.cuda.synchronize()
-    ms_lib = time_each(lambda: torch._int_mm(scratch[0], w8.t()), steps, flush)
-    del flush, w8
+    vendor = None
+    try:
+        g = torch.Generator().manual_seed(5)
+        w8 = torch.randint(-1, 2, (p.d_out, p.d_in), dtype=torch.int8, generator=g).to(dev)
+        for _ in range(max(warmup, 3)):   # the library picks and sets up its kernel on first use
+            torch._int_mm(scratch[0], w8.t())
+        torch.cuda.synchronize()
+        ms_lib = time_each(lambda: torch._int_mm(scratch[0], w8.t()), steps, flush)
+        del w8
+        vendor = {"impl": "cuBLASLt via torch._int_mm (int8 x int8 -> int32, unpacked weights)",
+                  "ms": round(ms_lib, 4), "tops": None, "ours_over_vendor": None}
+    except Exception as e:   # context only: its absence must not cost the measurement
+        vendor = {"impl": "cuBLASLt via torch._int_mm", "unavailable": repr(e)[:200]}
+    del flush
     ops = 2.0 * T * p.d_in * p.d_out
     tops = ops / (ms_mm * 1e-3) / 1e12
+    if vendor.get("ms"):
+        vendor["tops"] = round(ops / (vendor["ms"] * 1e-3) / 1e12, 1)
+        vendor["ours_over_vendor"] = round(vendor["ms"] / ms_mm, 3)
     peak = peaks["bf16"] * INT8_OVER_BF16
     return {
         "workload": WORKLOADS["prefill_2048x4096x11008"].name,
@@ -481,10 +491,7 @@ def measure_prefill(steps, warmup, dev, peaks):
                      "peak_source": "%s bf16 burst x %.0f (nominal int8/bf16 dense ratio)"
                                     % (peaks["source"], INT8_OVER_BF16)},
         "frac_of_datasheet_4500": round(tops / 4500.0, 4),
-        "vendor_int8_gemm_same_shape": {
-            "impl": "cuBLASLt via torch._int_mm (int8 x int8 -> int32, unpacked weights)",
-            "ms": round(ms_lib, 4), "tops": round(ops / (ms_lib * 1e-3) / 1e12, 1),
-            "ours_over_vendor": round(ms_lib / ms_mm, 3)},
+        "vendor_int8_gemm_same_shape": vendor,
         "l2": "L2 overwritten before every timed call; each call timed alone",
         "gpu_launches": 7 * steps,
     }
