@@ -64,12 +64,12 @@ namespace bl {
 
 namespace pair {
 
-constexpr int kBM = 128;          // weight rows per CTA (256 per pair)
-constexpr int kBN = 256;          // tokens per tile (MMA N), 128 loaded by each CTA
+constexpr int kBM = 128;          // weight rows per CTA (MMA N = 256 per pair)
+constexpr int kBN = 256;          // tokens per pair tile (MMA M), 128 loaded by each CTA
 constexpr int kBNHalf = kBN / 2;
 constexpr int kBK = 128;          // reduction columns per step (bytes)
 // A stage holds both operands of one 128-column step: this CTA's 16 KiB token
-// half (B) and its 16 KiB of expanded weight codes (A).  One barrier per
+// half (A) and its 16 KiB of expanded weight codes (B).  One barrier per
 // stage says both CTAs' operands are in place and one multicast commit frees
 // it, so the MMA issuer makes a single check and a single commit per step.
 constexpr int kStages = 5;
