@@ -149,13 +149,16 @@ int bitlinear_pack_weights(const float *W, int64_t d_out, int64_t d_in, float ep
  * NULL, workspace, ..., packed, gamma_out, stream); gamma is bit-identical.
  * The partial sums live instead in one fixed array inside the library of
  * 1184 doubles (9,472 bytes), held in the memory of every GPU that loads
- * the library until the process exits.  Shapes whose reduction would need
- * more partials than that are rejected with BITLINEAR_ERR_UNSUPPORTED_SHAPE
- * (the reduction grid is capped at 1184 blocks, so every shape the other
- * rules accept fits).  Calls no allocator (no cudaMalloc, cudaFree or
- * allocating library routine).  The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  All calls share the one
+ * the library until the process exits.  The reduction grid is capped at
+ * 1184 blocks, so every shape the rules above accept fits; shapes they
+ * reject return BITLINEAR_ERR_UNSUPPORTED_SHAPE as in bitlinear_pack_weights.
+ * Calls no allocator (no cudaMalloc, cudaFree or allocating library
+ * routine).  Every call made outside stream capture looks up the array's
+ * device address (cudaGetSymbolAddress) with the current device, so a
+ * device reset between calls is harmless; a call made during a capture uses
+ * the address found by the last such call on that device, and fails with
+ * BITLINEAR_ERR_CUDA if there was none: make one call on each device before
+ * capturing, and again after any device reset.  All calls share the one
  * array, which keeps the last call's contents (every partial read is first
  * written by the same call, so nothing needs clearing): calls that overlap
  * on the GPU -- on different streams, or on different host threads -- race

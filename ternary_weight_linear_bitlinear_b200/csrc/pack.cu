@@ -269,15 +269,25 @@ std::mutex g_noalloc_mu;
 double *g_noalloc_ptr[64];
 }  // namespace
 
-static bitlinear_status noalloc_scratch(double **out) {
+// The address is looked up again on every call made outside stream capture,
+// so a device reset (after which the array may sit at a new address) never
+// leaves a stale pointer in use; during a capture the address remembered
+// from the last such call on this device is used.
+static bitlinear_status noalloc_scratch(cudaStream_t stream, double **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BITLINEAR_ERR_DEVICE;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return BITLINEAR_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_pack_partials) != cudaSuccess || !p)
             return BITLINEAR_ERR_CUDA;
         g_noalloc_ptr[dev] = static_cast<double *>(p);
+    } else if (!g_noalloc_ptr[dev]) {
+        // First use on this device inside a capture: the lookup may have to
+        // load the module, which is not allowed while capturing.
+        return BITLINEAR_ERR_CUDA;
     }
     *out = g_noalloc_ptr[dev];
     return BITLINEAR_OK;
@@ -299,11 +309,12 @@ extern "C" int bitlinear_pack_weights_noalloc(const float *W, int64_t d_out, int
     int64_t blocks = (n4 + kRedThreads * 8 - 1) / (kRedThreads * 8);
     if (blocks > kRedMaxBlocks) blocks = kRedMaxBlocks;
     if (blocks < 1) blocks = 1;
-    if (blocks > kNoallocPartials) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    // The grid cap above is the array's size, so every accepted shape fits.
+    static_assert(kNoallocPartials >= kRedMaxBlocks, "noalloc partials hold the largest grid");
     bitlinear_status st = check_device();
     if (st != BITLINEAR_OK) return st;
     double *partial = nullptr;
-    st = noalloc_scratch(&partial);
+    st = noalloc_scratch(stream, &partial);
     if (st != BITLINEAR_OK) return st;
     // Every partial the final kernel reads is written by this call first, so
     // nothing in the shared array has to start at zero.

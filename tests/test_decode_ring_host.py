@@ -21,6 +21,16 @@ import pytest
 DEC_WARPS = 4
 
 
+def test_model_constants_match_kernel_source():
+    """The model's warp count is the kernel's (csrc/gemv.cu)."""
+    import os
+    import re
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "ternary_weight_linear_bitlinear_b200", "csrc", "gemv.cu")
+    m = re.search(r"constexpr int kDecWarps = (\d+);", open(path).read())
+    assert m and int(m.group(1)) == DEC_WARPS
+
+
 class Protocol(AssertionError):
     pass
 

@@ -28,6 +28,34 @@ EXP_WARPS = 4                  # warps per expander group
 EPI_WARPS = 4
 
 
+def _source_constants(fname):
+    """constexpr int values of a kernel source, by name."""
+    import os
+    import re
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "ternary_weight_linear_bitlinear_b200", "csrc", fname)
+    text = open(path).read()
+    out = {}
+    for name, expr in re.findall(r"constexpr int (k\w+) = ([^;]+);", text):
+        try:
+            out[name] = eval(expr, {}, dict(out))
+        except Exception:
+            pass
+    return out
+
+
+def test_model_constants_match_kernel_source():
+    """The model runs on the kernel's own ring constants: a change in the
+    kernel that the model does not follow fails here."""
+    c = _source_constants("gemm_tc.cu")
+    assert c["kStages"] == K_STAGES
+    assert c["kPSlots"] == K_PSLOTS
+    assert c["kPAhead"] == K_PAHEAD
+    assert c["kAccBufs"] == K_ACC_BUFS
+    assert c["kReadyCount"] == K_READY_COUNT
+    assert c["kEpiWarps"] == EPI_WARPS
+
+
 class Protocol(AssertionError):
     pass
 
