@@ -669,36 +669,87 @@ def measure_e2e(run, steps):
 
 # -------------------------------------------------------- CPU oracle ---
 
-def oracle_layer_step(p, wq, gamma, xb):
+def oracle_layer_step(p, wq, gamma, xb, parallel=False):
     import oracle
     xq, beta, rowsum, _ = oracle.quant_act(xb, eps=EPS)
-    acc = oracle.int_matmul(wq, xq)
+    acc = oracle.int_matmul(wq, xq, parallel=parallel)
     return oracle.rescale(acc, gamma, beta)
 
 
-def cpu_oracle_rate(name, seconds, max_layers=None):
-    """Time the oracle on bounded samples of the workload; returns
-    (GB/s of algorithmic bytes, layers done, seconds, description)."""
+def _oracle_prepared(name):
     import oracle
     oracle.build()
-    wl = WORKLOADS[name]
     prepared = []
-    for p in wl.problems:
+    for p in WORKLOADS[name].problems:
         W, X = draw(p)
         Wn = W.numpy()
         g = oracle.absmean_gamma(Wn)
         prepared.append((p, oracle.ternarize(Wn, g, EPS), g, bf16_bits(X)))
         del W, Wn
+    return prepared
+
+
+def cpu_oracle_rate(name, seconds, parallel=False, max_layers=None):
+    """Time the oracle on bounded samples of a decode workload: whole
+    forwards (quantise, int32 product, rescale) for about `seconds`.  Returns
+    (GB/s of algorithmic bytes, forwards done, seconds)."""
+    prepared = _oracle_prepared(name)
     done, nbytes, t0 = 0, 0, time.perf_counter()
     while True:
         p, wq, g, xb = prepared[done % len(prepared)]
-        oracle_layer_step(p, wq, g, xb)
+        oracle_layer_step(p, wq, g, xb, parallel)
         done += 1
         nbytes += decode_bytes(p)["step"]
         el = time.perf_counter() - t0
         if el >= seconds or (max_layers and done >= max_layers):
             break
     return nbytes / el / 1e9, done, el
+
+
+def cpu_oracle_prefill(seconds):
+    """The prefill product on the host's cores: the oracle's int32 product of
+    the first tokens of the 2048-token workload (quantised once), growing the
+    token count until a call takes about `seconds`.  Returns (TOPS, tokens,
+    seconds of the last call)."""
+    import oracle
+    (p, wq, g, xb), = _oracle_prepared("prefill_2048x4096x11008")
+    xq, _, _, _ = oracle.quant_act(xb, eps=EPS)
+    T = 8
+    while True:
+        t0 = time.perf_counter()
+        oracle.int_matmul(wq, xq[:T], parallel=True)
+        el = time.perf_counter() - t0
+        if el >= seconds / 4 or T >= p.tokens:
+            break
+        T = min(p.tokens, T * 4)
+    return 2.0 * T * p.d_in * p.d_out / el / 1e12, T, el
+
+
+def cpu_baseline_line(workload, seconds):
+    """The CPU oracle on this host: every core (the OpenMP build of the same
+    C source) on the headline, the large GEMV and a prefill sample, plus the
+    single-thread rate on the headline."""
+    import oracle
+    threads = oracle.threads(parallel=True)
+    rate, done, el = cpu_oracle_rate(workload, seconds / 3, parallel=True)
+    rate1, done1, el1 = cpu_oracle_rate(workload, seconds / 3)
+    rl, donel, ell = cpu_oracle_rate("large_gemv_8192x28672_t1", seconds / 6, parallel=True)
+    tops, tp, elp = cpu_oracle_prefill(seconds / 6)
+    shape = "x".join(workload.split("_")[2:3])
+    return {
+        "value": round(rate, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+        "host_cpus": len(os.sched_getaffinity(0)),
+        "sample": "%d single-token %s BitLinear forwards (quantise + int32 product + rescale) "
+                  "by the plain C oracle, its product split over %d OpenMP threads, %.1f s"
+                  % (done, shape, threads, el),
+        "single_thread": {"value": round(rate1, 4), "unit": "GB/s", "cores": 1,
+                          "sample": "%d forwards, one thread, %.1f s" % (done1, el1)},
+        "large_gemv_8192x28672_t1": {"value": round(rl, 4), "unit": "GB/s", "cores": threads,
+                                     "sample": "%d forwards, %.1f s" % (donel, ell)},
+        "prefill_2048x4096x11008": {"value": round(tops, 5), "unit": "TOPS", "cores": threads,
+                                    "sample": "int32 product of the first %d of 2048 quantised "
+                                              "tokens, %.2f s" % (tp, elp)},
+    }
 
 
 # -------------------------------------------------------------- main ---
@@ -844,11 +895,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1:
-        rate, done, el = cpu_oracle_rate(args.workload, args.cpu_seconds)
-        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": "%d single-token %s BitLinear forwards (quantise + int32 product + "
-                         "rescale) by the plain C oracle, single thread, %.1f s"
-                         % (done, "x".join(args.workload.split("_")[2:3]), el)}
+        cpu = cpu_baseline_line(args.workload, args.cpu_seconds)
 
     if rank == 0:
         clocks = sampler.summary()
@@ -908,22 +955,17 @@ def reference_arm(args, warmup):
     """The CPU oracle timed on this host: each step is a bounded sample
     (one BitLinear forward of the workload's shape), same metric and unit."""
     import oracle
-    oracle.build()
     wl = WORKLOADS[args.workload]
-    prepared = []
-    for p in wl.problems:
-        W, X = draw(p)
-        Wn = W.numpy()
-        g = oracle.absmean_gamma(Wn)
-        prepared.append((p, oracle.ternarize(Wn, g, EPS), g, bf16_bits(X)))
+    prepared = _oracle_prepared(args.workload)
+    threads = oracle.threads(parallel=True)
     for i in range(warmup):
         p, wq, g, xb = prepared[i % len(prepared)]
-        oracle_layer_step(p, wq, g, xb)
+        oracle_layer_step(p, wq, g, xb, parallel=True)
     nbytes = 0
     t0 = time.perf_counter()
     for i in range(args.steps):
         p, wq, g, xb = prepared[i % len(prepared)]
-        oracle_layer_step(p, wq, g, xb)
+        oracle_layer_step(p, wq, g, xb, parallel=True)
         nbytes += decode_bytes(p)["step"]
     el = time.perf_counter() - t0
     value = nbytes / el / 1e9
@@ -935,9 +977,11 @@ def reference_arm(args, warmup):
         "config": {"workload": args.workload, "forwards_per_step": 1,
                    "tokens": wl.problems[0].tokens, "d_in": wl.problems[0].d_in,
                    "d_out": wl.problems[0].d_out},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "host_cpus": len(os.sched_getaffinity(0)),
                          "sample": "each step one BitLinear forward of the workload by the "
-                                   "plain C oracle, single thread"},
+                                   "plain C oracle, its product split over %d OpenMP threads"
+                                   % threads},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

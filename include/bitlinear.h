@@ -94,7 +94,7 @@ typedef enum {
  * Q_b - 1 = 7, codes in [-7, 7] (still stored one per int8). */
 #define BITLINEAR_ACT_4BIT 8u
 
-/* Library ABI version (this header: 1). */
+/* Library ABI version (this header: 2). */
 int bitlinear_version(void);
 
 /* Static description of a status code.  Never NULL. */
@@ -232,23 +232,26 @@ int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
 
 /*
  * bitlinear_linear -- the whole BitLinear forward from bf16 activations:
- * bitlinear_quant_act (with r computed, inv_rms_in = NULL) followed by
- * bitlinear_forward, with the same arguments, meaning and results (bit for
- * bit) as those two calls made back to back ([MF] section 2, all three
- * parts).  flags: BITLINEAR_RMSNORM, BITLINEAR_STATIC_WEIGHTS.  Xq, beta and
- * rowsum are caller-owned intermediates of T*d_in, T and T elements, written
- * with the codes, absmax and row sums.  For T <= 8 with T*d_in <= 32768 one
- * kernel quantises (in shared memory, per CTA) and multiplies; otherwise the
- * quantiser runs first and the product kernel is its programmatic dependent.
- * Kernels are launched as programmatic dependents of the work before them
- * and read nothing earlier work produces before their dependency wait,
- * except the weights under BITLINEAR_STATIC_WEIGHTS.
+ * bitlinear_quant_act followed by bitlinear_forward, with the same arguments,
+ * meaning and results (bit for bit) as those two calls made back to back
+ * ([MF] section 2, all three parts).  flags: BITLINEAR_RMSNORM,
+ * BITLINEAR_STATIC_WEIGHTS, BITLINEAR_PER_TENSOR_ABSMAX.  inv_rms_in: fp32
+ * [T] per-token reciprocal RMS to use instead of computing it, or NULL (as in
+ * bitlinear_quant_act).  Xq, beta and rowsum are caller-owned intermediates
+ * of T*d_in, T and T elements, written with the codes, absmax and row sums.
+ * For T <= 8 with T*d_in <= 32768 one kernel quantises (in shared memory,
+ * per CTA) and multiplies; otherwise the quantiser runs first and the
+ * product kernel is its programmatic dependent.  Kernels are launched as
+ * programmatic dependents of the work before them and read nothing earlier
+ * work produces before their dependency wait, except the weights under
+ * BITLINEAR_STATIC_WEIGHTS.
  */
 int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
                      int64_t d_in, const uint16_t *X, int64_t T,
                      const float *norm_gain, uint32_t flags, float eps,
-                     float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
-                     void *Y, int out_dtype, cudaStream_t stream);
+                     float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                     float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                     cudaStream_t stream);
 
 /*
  * Base-3 weight format ([MF] section 4, "Memory Bandwidth and Latency
@@ -300,8 +303,9 @@ int bitlinear_forward_base3(const uint8_t *packed3, const float *gamma, int64_t 
 int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
                            int64_t d_in, const uint16_t *X, int64_t T,
                            const float *norm_gain, uint32_t flags, float eps,
-                           float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
-                           void *Y, int out_dtype, cudaStream_t stream);
+                           float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                           float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                           cudaStream_t stream);
 
 /*
  * W1A4: binary weights with 4-bit activations, the regime "The End of Matrix
@@ -359,8 +363,9 @@ int bitlinear_forward_w1(const uint32_t *packed1, const float *gamma, int64_t d_
  */
 int bitlinear_linear_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
                         int64_t d_in, const uint16_t *X, int64_t T, const float *norm_gain,
-                        uint32_t flags, float eps, float norm_eps, int8_t *Xq, float *beta,
-                        int32_t *rowsum, void *Y, int out_dtype, cudaStream_t stream);
+                        uint32_t flags, float eps, float norm_eps, const float *inv_rms_in,
+                        int8_t *Xq, float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                        cudaStream_t stream);
 
 /*
  * bitlinear_dense_bf16_forward -- the dense bf16 linear layer Y = X W^T that

@@ -29,89 +29,118 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "bitlinear_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+# The same source built with OpenMP: int_matmul's independent outputs are
+# split over the host's cores.  Only the benchmark's CPU baseline uses it.
+_LIB_OMP = os.path.join(_HERE, "liboracle_omp.so")
 
 QB_MINUS_1 = 127  # [MF] §2: Q_b - 1, multiplier and clip bound of the activation codes
 
 
-def build(force: bool = False) -> str:
-    """Compile the oracle with gcc; returns the path of the shared object."""
-    if (not force and os.path.exists(_LIB)
-            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
-        return _LIB
-    tmp = _LIB + ".tmp.%d" % os.getpid()
+def _compile(out: str, extra, force: bool) -> str:
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(_SRC)):
+        return out
+    tmp = out + ".tmp.%d" % os.getpid()
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
            "-fno-fast-math", "-fno-unsafe-math-optimizations", "-Wall", "-Wextra",
-           _SRC, "-o", tmp, "-lm"]
+           "-Wno-unknown-pragmas", *extra, _SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, _LIB)
-    return _LIB
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain, and the OpenMP build of the same
+    source); returns the path of the plain shared object."""
+    _compile(_LIB_OMP, ["-fopenmp"], force)
+    return _compile(_LIB, [], force)
 
 
 _lib = None
+_lib_omp = None
 
 
-def _load():
-    global _lib
+def _load(parallel: bool = False):
+    global _lib, _lib_omp
+    if parallel:
+        if _lib_omp is None:
+            build()
+            lib = ctypes.CDLL(_LIB_OMP)
+            _declare(lib)
+            _lib_omp = lib
+        return _lib_omp
     if _lib is None:
         lib = ctypes.CDLL(build())
-        i64, f32, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_int
-        vp = ctypes.c_void_p
-        lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
-        lib.oracle_bf16_to_f32.restype = f32
-        lib.oracle_f32_to_bf16.argtypes = [f32]
-        lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
-        lib.oracle_abs_sum.argtypes = [vp, i64, i64]
-        lib.oracle_abs_sum.restype = ctypes.c_double
-        lib.oracle_absmean_gamma.argtypes = [vp, i64, i64]
-        lib.oracle_absmean_gamma.restype = f32
-        lib.oracle_ternarize.argtypes = [vp, i64, f32, f32, vp]
-        lib.oracle_ternarize.restype = None
-        lib.oracle_pack.argtypes = [vp, i64, i64, vp]
-        lib.oracle_pack.restype = i32
-        lib.oracle_unpack.argtypes = [vp, i64, i64, vp]
-        lib.oracle_unpack.restype = i32
-        lib.oracle_unpack_row.argtypes = [vp, i64, i64, i64, vp]
-        lib.oracle_unpack_row.restype = i32
-        lib.oracle_base3_cols.argtypes = [i64]
-        lib.oracle_base3_cols.restype = i64
-        lib.oracle_pack_base3.argtypes = [vp, i64, i64, vp]
-        lib.oracle_pack_base3.restype = i32
-        lib.oracle_unpack_base3.argtypes = [vp, i64, i64, vp]
-        lib.oracle_unpack_base3.restype = i32
-        lib.oracle_binarize.argtypes = [vp, i64, vp]
-        lib.oracle_binarize.restype = None
-        lib.oracle_w1_cols.argtypes = [i64]
-        lib.oracle_w1_cols.restype = i64
-        lib.oracle_pack_w1.argtypes = [vp, i64, i64, vp]
-        lib.oracle_pack_w1.restype = i32
-        lib.oracle_unpack_w1.argtypes = [vp, i64, i64, vp]
-        lib.oracle_unpack_w1.restype = i32
-        lib.oracle_quant_act_bits.argtypes = [vp, i64, i64, vp, i32, i32, i32, f32, f32, vp,
-                                              vp, vp, vp, vp]
-        lib.oracle_quant_act_bits.restype = None
-        lib.oracle_rescale_bits.argtypes = [vp, i64, i64, f32, vp, i32, vp]
-        lib.oracle_rescale_bits.restype = None
-        lib.oracle_inv_rms.argtypes = [vp, i64, f32]
-        lib.oracle_inv_rms.restype = f32
-        lib.oracle_quant_act.argtypes = [vp, i64, i64, vp, i32, i32, f32, f32, vp,
-                                         vp, vp, vp, vp]
-        lib.oracle_quant_act.restype = None
-        lib.oracle_int_matmul.argtypes = [vp, vp, i64, i64, i64, vp]
-        lib.oracle_int_matmul.restype = None
-        lib.oracle_dot_masked_add.argtypes = [vp, vp, i64]
-        lib.oracle_dot_masked_add.restype = ctypes.c_int32
-        lib.oracle_rescale.argtypes = [vp, i64, i64, f32, vp, vp]
-        lib.oracle_rescale.restype = None
-        lib.oracle_dequant_act_bf16.argtypes = [ctypes.c_int8, f32]
-        lib.oracle_dequant_act_bf16.restype = ctypes.c_uint16
-        lib.oracle_backward.argtypes = [vp, f32, vp, vp, vp, i64, i64, i64, vp, vp]
-        lib.oracle_backward.restype = None
-        lib.oracle_dense_bf16_dot.argtypes = [vp, vp, i64]
-        lib.oracle_dense_bf16_dot.restype = ctypes.c_double
-        lib.oracle_dense_bf16.argtypes = [vp, vp, i64, i64, i64, vp]
-        lib.oracle_dense_bf16.restype = None
+        _declare(lib)
         _lib = lib
     return _lib
+
+
+def threads(parallel: bool = True) -> int:
+    """Threads the oracle's parallel loops use (1 for the plain build)."""
+    return int(_load(parallel).oracle_threads())
+
+
+def _declare(lib):
+    """Argument and result types of every exported oracle function."""
+    i64, f32, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_int
+    vp = ctypes.c_void_p
+    lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.oracle_bf16_to_f32.restype = f32
+    lib.oracle_f32_to_bf16.argtypes = [f32]
+    lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+    lib.oracle_abs_sum.argtypes = [vp, i64, i64]
+    lib.oracle_abs_sum.restype = ctypes.c_double
+    lib.oracle_absmean_gamma.argtypes = [vp, i64, i64]
+    lib.oracle_absmean_gamma.restype = f32
+    lib.oracle_ternarize.argtypes = [vp, i64, f32, f32, vp]
+    lib.oracle_ternarize.restype = None
+    lib.oracle_pack.argtypes = [vp, i64, i64, vp]
+    lib.oracle_pack.restype = i32
+    lib.oracle_unpack.argtypes = [vp, i64, i64, vp]
+    lib.oracle_unpack.restype = i32
+    lib.oracle_unpack_row.argtypes = [vp, i64, i64, i64, vp]
+    lib.oracle_unpack_row.restype = i32
+    lib.oracle_base3_cols.argtypes = [i64]
+    lib.oracle_base3_cols.restype = i64
+    lib.oracle_pack_base3.argtypes = [vp, i64, i64, vp]
+    lib.oracle_pack_base3.restype = i32
+    lib.oracle_unpack_base3.argtypes = [vp, i64, i64, vp]
+    lib.oracle_unpack_base3.restype = i32
+    lib.oracle_binarize.argtypes = [vp, i64, vp]
+    lib.oracle_binarize.restype = None
+    lib.oracle_w1_cols.argtypes = [i64]
+    lib.oracle_w1_cols.restype = i64
+    lib.oracle_pack_w1.argtypes = [vp, i64, i64, vp]
+    lib.oracle_pack_w1.restype = i32
+    lib.oracle_unpack_w1.argtypes = [vp, i64, i64, vp]
+    lib.oracle_unpack_w1.restype = i32
+    lib.oracle_quant_act_bits.argtypes = [vp, i64, i64, vp, i32, i32, i32, f32, f32, vp,
+                                          vp, vp, vp, vp]
+    lib.oracle_quant_act_bits.restype = None
+    lib.oracle_rescale_bits.argtypes = [vp, i64, i64, f32, vp, i32, vp]
+    lib.oracle_rescale_bits.restype = None
+    lib.oracle_inv_rms.argtypes = [vp, i64, f32]
+    lib.oracle_inv_rms.restype = f32
+    lib.oracle_quant_act.argtypes = [vp, i64, i64, vp, i32, i32, f32, f32, vp,
+                                     vp, vp, vp, vp]
+    lib.oracle_quant_act.restype = None
+    lib.oracle_int_matmul.argtypes = [vp, vp, i64, i64, i64, vp]
+    lib.oracle_int_matmul.restype = None
+    lib.oracle_dot_masked_add.argtypes = [vp, vp, i64]
+    lib.oracle_dot_masked_add.restype = ctypes.c_int32
+    lib.oracle_rescale.argtypes = [vp, i64, i64, f32, vp, vp]
+    lib.oracle_rescale.restype = None
+    lib.oracle_dequant_act_bf16.argtypes = [ctypes.c_int8, f32]
+    lib.oracle_dequant_act_bf16.restype = ctypes.c_uint16
+    lib.oracle_backward.argtypes = [vp, f32, vp, vp, vp, i64, i64, i64, vp, vp]
+    lib.oracle_backward.restype = None
+    lib.oracle_dense_bf16_dot.argtypes = [vp, vp, i64]
+    lib.oracle_dense_bf16_dot.restype = ctypes.c_double
+    lib.oracle_dense_bf16.argtypes = [vp, vp, i64, i64, i64, vp]
+    lib.oracle_dense_bf16.restype = None
+    lib.oracle_threads.argtypes = []
+    lib.oracle_threads.restype = ctypes.c_int
 
 
 def _ptr(a):
@@ -293,14 +322,15 @@ def quant_act(X_bf16_bits, gain=None, rmsnorm: bool = True, eps: float = 1e-5,
 
 # ----------------------------------------------------- product / rescale ---
 
-def int_matmul(wq, xq) -> np.ndarray:
-    """acc[t][o] = sum_k W~[o][k] X~[t][k] in int32 ([MF] §2)."""
+def int_matmul(wq, xq, parallel: bool = False) -> np.ndarray:
+    """acc[t][o] = sum_k W~[o][k] X~[t][k] in int32 ([MF] §2).  parallel: the
+    OpenMP build (same arithmetic, outputs split over the host's cores)."""
     wq = _c(wq, np.int8)
     xq = _c(xq, np.int8)
     N, K = wq.shape
     T = xq.shape[0]
     acc = np.empty((T, N), dtype=np.int32)
-    _load().oracle_int_matmul(_ptr(wq), _ptr(xq), T, N, K, _ptr(acc))
+    _load(parallel).oracle_int_matmul(_ptr(wq), _ptr(xq), T, N, K, _ptr(acc))
     return acc
 
 

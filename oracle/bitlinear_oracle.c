@@ -337,6 +337,14 @@ int oracle_unpack_w1(const uint32_t *packed, int64_t n_out, int64_t n_in, int8_t
     return 0;
 }
 
+/* Threads the OpenMP build runs its parallel loops on (1 in the plain build). */
+#ifdef _OPENMP
+#include <omp.h>
+int oracle_threads(void) { return omp_get_max_threads(); }
+#else
+int oracle_threads(void) { return 1; }
+#endif
+
 /* ---------------------------------------- activation quantisation ([MF] §2) */
 
 /* Reciprocal RMS of one token: 1 / sqrt(mean(x^2) + norm_eps), carried in
@@ -442,6 +450,11 @@ void oracle_quant_act(const uint16_t *X, int64_t T, int64_t K, const float *gain
 void oracle_int_matmul(const int8_t *wq, const int8_t *xq, int64_t T, int64_t N,
                        int64_t K, int32_t *acc)
 {
+    /* The outputs are independent: the OpenMP build of this file (used only
+     * to time the oracle on every host core) splits them over threads; the
+     * plain build ignores the pragma.  Each output is the same sum either
+     * way. */
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t t = 0; t < T; ++t)
         for (int64_t o = 0; o < N; ++o) {
             int32_t s = 0;

@@ -54,20 +54,20 @@ SIGNATURES = {
                                    _vp, _vp, _vp]),
     "bitlinear_forward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int,
                                  _vp, _vp]),
-    "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
+    "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32, _vp,
                                 _vp, _vp, _vp, _vp, _int, _vp]),
     "bitlinear_base3_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bitlinear_repack_base3": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "bitlinear_forward_base3": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int,
                                        _vp, _vp]),
-    "bitlinear_linear_base3": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
+    "bitlinear_linear_base3": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32, _vp,
                                       _vp, _vp, _vp, _vp, _int, _vp]),
     "bitlinear_w1_packed_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bitlinear_pack_weights_w1": (_int, [_vp, _i64, _i64, _vp, _vp, ctypes.c_size_t, _vp, _vp,
                                          _vp]),
     "bitlinear_forward_w1": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _int,
                                     _vp, _vp]),
-    "bitlinear_linear_w1": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32,
+    "bitlinear_linear_w1": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32, _vp,
                                    _vp, _vp, _vp, _vp, _int, _vp]),
     "bitlinear_dense_bf16_forward": (_int, [_vp, _i64, _i64, _vp, _i64, _vp, _int, _vp]),
     "bitlinear_backward_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _int, _int]),
@@ -253,20 +253,28 @@ def pack_weights(W: torch.Tensor, eps: float = 1e-5, gamma: torch.Tensor = None,
 
 def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
               eps: float = 1e-5, norm_eps: float = 1e-5, inv_rms: torch.Tensor = None,
-              per_tensor: bool = False, act_bits: int = 8):
+              per_tensor: bool = False, act_bits: int = 8, outs=None):
     """Fused RMSNorm + absmax int8 codes of bf16 X [T][d_in], with one beta
     per token (default) or one for the whole tensor (per_tensor).
 
     Returns (Xq int8 [T][d_in], beta f32 [T], rowsum int32 [T], inv_rms f32 [T]),
-    inv_rms being the per-token reciprocal RMS used (or given).
+    inv_rms being the per-token reciprocal RMS used (or given).  ``outs``, if
+    given, is that tuple of caller-owned tensors to write instead.
     """
     _need(X, torch.bfloat16, "X")
     T, d_in = X.shape
     dev = X.device
-    Xq = torch.empty((T, d_in), dtype=torch.int8, device=dev)
-    beta = torch.empty(T, dtype=torch.float32, device=dev)
-    rowsum = torch.empty(T, dtype=torch.int32, device=dev)
-    rms_out = torch.empty(T, dtype=torch.float32, device=dev)
+    if outs is not None:
+        Xq, beta, rowsum, rms_out = outs
+        _need(Xq, torch.int8, "Xq")
+        _need(beta, torch.float32, "beta")
+        _need(rowsum, torch.int32, "rowsum")
+        _need(rms_out, torch.float32, "inv_rms_out")
+    else:
+        Xq = torch.empty((T, d_in), dtype=torch.int8, device=dev)
+        beta = torch.empty(T, dtype=torch.float32, device=dev)
+        rowsum = torch.empty(T, dtype=torch.int32, device=dev)
+        rms_out = torch.empty(T, dtype=torch.float32, device=dev)
     if gain is not None:
         _need(gain, torch.float32, "gain")
     if inv_rms is not None:
@@ -282,17 +290,22 @@ def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
 
 def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
             out_dtype=torch.float32, want_acc: bool = False, out: torch.Tensor = None,
-            act_bits: int = 8):
+            act_bits: int = 8, acc: torch.Tensor = None):
     """Y = (X~ W~^T) gamma beta / (Q_b - 1); returns Y (and the int32 acc if
-    asked).  w is a PackedTernary, PackedTernaryBase3 or PackedBinary; act_bits
-    (4 or 8, the width the codes were made with) applies to PackedBinary."""
+    asked, written to ``acc`` when that tensor is given).  w is a
+    PackedTernary, PackedTernaryBase3 or PackedBinary; act_bits (4 or 8, the
+    width the codes were made with) applies to PackedBinary."""
     _need(Xq, torch.int8, "Xq")
     T = Xq.shape[0]
     dev = Xq.device
     if out is None:
         out = torch.empty((T, w.d_out), dtype=out_dtype, device=dev)
     od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
-    acc = torch.empty((T, w.d_out), dtype=torch.int32, device=dev) if want_acc else None
+    if acc is not None:
+        _need(acc, torch.int32, "acc")
+        want_acc = True
+    elif want_acc:
+        acc = torch.empty((T, w.d_out), dtype=torch.int32, device=dev)
     fn, name = _entry(w, "bitlinear_forward")
     if isinstance(w, PackedBinary):
         st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq), _ptr(beta),
@@ -309,7 +322,7 @@ def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
 def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
            eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.float32,
            out: torch.Tensor = None, scratch=None, static_weights: bool = False,
-           per_tensor: bool = False, act_bits: int = 8):
+           per_tensor: bool = False, act_bits: int = 8, inv_rms: torch.Tensor = None):
     """The whole BitLinear forward from bf16 X: quantise, then product.
     w is a PackedTernary, PackedTernaryBase3 or PackedBinary; act_bits = 4
     (PackedBinary only) makes it the W1A4 forward.
@@ -318,7 +331,8 @@ def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
     writes w.packed or w.gamma (the product may then stream the weights
     before earlier work has finished).  per_tensor: one activation absmax for
     the whole X instead of one per token.  ``scratch`` = (Xq, beta, rowsum)
-    receives the intermediates.
+    receives the intermediates.  inv_rms: f32 [T] reciprocal RMS to use
+    instead of computing it.
     """
     _need(X, torch.bfloat16, "X")
     T = X.shape[0]
@@ -333,11 +347,14 @@ def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
     od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
     if gain is not None:
         _need(gain, torch.float32, "gain")
+    if inv_rms is not None:
+        _need(inv_rms, torch.float32, "inv_rms")
     flags = ((RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
              | (PER_TENSOR_ABSMAX if per_tensor else 0) | (ACT_4BIT if act_bits == 4 else 0))
     fn, name = _entry(w, "bitlinear_linear")
     st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(X), T, _ptr(gain), flags, eps,
-            norm_eps, _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od, _stream())
+            norm_eps, _ptr(inv_rms), _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od,
+            _stream())
     _check(st, name)
     return out
 
@@ -373,8 +390,8 @@ class LinearPlan:
         self._fn, self._name = _entry(w, "bitlinear_linear")
         self._pre = (w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in)
         sh = stream.cuda_stream if stream is not None else _stream()
-        self._post = (T, _ptr(gain), flags, eps, norm_eps, Xq.data_ptr(), beta.data_ptr(),
-                      rowsum.data_ptr(), out.data_ptr(), od, sh)
+        self._post = (T, _ptr(gain), flags, eps, norm_eps, None, Xq.data_ptr(),
+                      beta.data_ptr(), rowsum.data_ptr(), out.data_ptr(), od, sh)
 
     def __call__(self, X: torch.Tensor) -> torch.Tensor:
         if X.dtype != torch.bfloat16 or tuple(X.shape) != self._shape or not X.is_contiguous():

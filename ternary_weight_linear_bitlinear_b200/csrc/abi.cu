@@ -23,8 +23,9 @@ bool decode_can_fuse(int64_t T, int64_t d_in);
 bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const uint16_t *X, int64_t T,
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
-                                     int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
-                                     int out_dtype, bool static_weights, int fmt, float qmax,
+                                     const float *inv_rms_in, int8_t *Xq, float *beta,
+                                     int32_t *rowsum, void *Y, int out_dtype,
+                                     bool static_weights, int fmt, float qmax,
                                      cudaStream_t stream);
 bitlinear_status launch_gemm_tc_pair(const uint32_t *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const int8_t *Xq, const float *beta,
@@ -159,8 +160,9 @@ static bitlinear_status forward_common(const void *packed, const float *gamma, i
 static bitlinear_status linear_common(const void *packed, const float *gamma, int64_t d_out,
                                       int64_t d_in, const uint16_t *X, int64_t T,
                                       const float *norm_gain, uint32_t flags, float eps,
-                                      float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
-                                      void *Y, int out_dtype, int fmt, cudaStream_t stream) {
+                                      float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                      float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                      int fmt, cudaStream_t stream) {
     bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, nullptr);
     if (st != BITLINEAR_OK) return st;
     if (fmt != kFmt2Bit && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
@@ -173,7 +175,7 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
     if (T == 0) return BITLINEAR_OK;
     if (!X || !Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
     if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4) ||
-        (norm_gain && !aligned(norm_gain, 4)))
+        (norm_gain && !aligned(norm_gain, 4)) || (inv_rms_in && !aligned(inv_rms_in, 4)))
         return BITLINEAR_ERR_MISALIGNED;
     st = check_device();
     if (st != BITLINEAR_OK) return st;
@@ -182,14 +184,14 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
     const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
     if (!per_tensor && decode_can_fuse(T, d_in))
         return launch_linear_fused(packed, gamma, d_out, d_in, X, T, norm_gain, rmsnorm, eps,
-                                   norm_eps, Xq, beta, rowsum, Y, out_dtype, static_weights,
-                                   fmt, qmax, stream);
+                                   norm_eps, inv_rms_in, Xq, beta, rowsum, Y, out_dtype,
+                                   static_weights, fmt, qmax, stream);
     // Quantiser, then the product as its programmatic dependent: with static
     // weights the product streams them while the codes are still being made.
     st = launch_quant_act(X, T, d_in, norm_gain,
                           flags & (BITLINEAR_RMSNORM | BITLINEAR_PER_TENSOR_ABSMAX |
                                    BITLINEAR_ACT_4BIT),
-                          eps, norm_eps, nullptr, Xq, beta, rowsum, nullptr, true, stream);
+                          eps, norm_eps, inv_rms_in, Xq, beta, rowsum, nullptr, true, stream);
     if (st != BITLINEAR_OK) return st;
     return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
                             nullptr, static_weights, fmt, qmax, stream);
@@ -199,7 +201,7 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
 
 using namespace bl;
 
-extern "C" int bitlinear_version(void) { return 1; }
+extern "C" int bitlinear_version(void) { return 2; }
 
 extern "C" const char *bitlinear_status_string(int status) {
     switch (status) {
@@ -242,28 +244,30 @@ extern "C" int bitlinear_forward_w1(const uint32_t *packed1, const float *gamma,
 extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
                                 int64_t d_in, const uint16_t *X, int64_t T,
                                 const float *norm_gain, uint32_t flags, float eps, float norm_eps,
-                                int8_t *Xq, float *beta, int32_t *rowsum, void *Y, int out_dtype,
-                                cudaStream_t stream) {
-    return linear_common(packed, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps, Xq,
-                         beta, rowsum, Y, out_dtype, kFmt2Bit, stream);
+                                const float *inv_rms_in, int8_t *Xq, float *beta,
+                                int32_t *rowsum, void *Y, int out_dtype, cudaStream_t stream) {
+    return linear_common(packed, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps,
+                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmt2Bit, stream);
 }
 
 extern "C" int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
                                       int64_t d_in, const uint16_t *X, int64_t T,
                                       const float *norm_gain, uint32_t flags, float eps,
-                                      float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
-                                      void *Y, int out_dtype, cudaStream_t stream) {
-    return linear_common(packed3, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps, Xq,
-                         beta, rowsum, Y, out_dtype, kFmtBase3, stream);
+                                      float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                      float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                      cudaStream_t stream) {
+    return linear_common(packed3, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps,
+                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmtBase3, stream);
 }
 
 extern "C" int bitlinear_linear_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
                                    int64_t d_in, const uint16_t *X, int64_t T,
                                    const float *norm_gain, uint32_t flags, float eps,
-                                   float norm_eps, int8_t *Xq, float *beta, int32_t *rowsum,
-                                   void *Y, int out_dtype, cudaStream_t stream) {
-    return linear_common(packed1, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps, Xq,
-                         beta, rowsum, Y, out_dtype, kFmt1Bit, stream);
+                                   float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                   float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                   cudaStream_t stream) {
+    return linear_common(packed1, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps,
+                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmt1Bit, stream);
 }
 
 extern "C" int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, int64_t d_in,

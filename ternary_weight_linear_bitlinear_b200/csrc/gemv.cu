@@ -78,6 +78,7 @@
 
 #include "bitlinear.h"
 #include "common.cuh"
+#include "decode_common.cuh"
 #include "quant_common.cuh"
 
 namespace bl {
@@ -102,6 +103,7 @@ struct DecodeArgs {
     // fused inputs and the intermediates CTA 0 writes back
     const uint16_t *X;
     const float *gain;
+    const float *inv_rms_in; // supplied per-token reciprocal RMS, or null
     int rmsnorm;
     float eps;
     float norm_eps;
@@ -122,24 +124,6 @@ struct DecodePlan {
     int stage_bytes;   // R * ks KiB of weights + T * ks * 256 B of codes (unfused)
     int xs_bytes;      // fused: T * K codes, rounded up to 128
 };
-
-__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mma_s8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ __half2 h2_bits(uint32_t u) {
     return *reinterpret_cast<const __half2 *>(&u);
@@ -170,34 +154,8 @@ __device__ __forceinline__ void base3_neg_codes(uint32_t w, uint32_t *d) {
     d[4] = __byte_perm(h2_u32(__hadd2(ve, m3072)), h2_u32(__hadd2(vo, m3072)), 0x6240);
 }
 
-// Bulk (TMA-engine) copy of `bytes` contiguous bytes global -> shared,
-// completing on an mbarrier.  Both addresses 16-byte aligned, bytes % 16 == 0.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
-                                         uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
 __device__ __forceinline__ void consumer_barrier() {
     asm volatile("bar.sync 2, %0;" ::"n"(kDecWarps * 32) : "memory");
-}
-
-// Bounded wait that also gives up once another role has aborted.
-__device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, const DeviceCtx &ctx,
-                                         volatile int *abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > ctx.wait_ns) {
-            atomicOr(ctx.err, kErrTimeout);
-            *abort_flag = 1;
-            return false;
-        }
-    }
 }
 
 template <int NT, int R, bool FUSED, bool OUT_BF16, int FMT>
@@ -347,7 +305,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             // between the codes and the MMAs.
             fast_quant = true;
             const bool rmsnorm = a.rmsnorm != 0;
-            token_partials_smem<TMAX>(xb, T, K, rmsnorm, qs);
+            token_partials_smem<TMAX>(xb, T, K, rmsnorm && !a.inv_rms_in, qs);
             consumer_barrier();
             int sums[TMAX];
             #pragma unroll
@@ -355,7 +313,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 sums[t] = 0;
                 if (t < T) {
                     const TokenScale ts =
-                        token_finalize<TMAX>(t, rmsnorm, a.eps, a.norm_eps, a.inv_k, a.qmax, qs);
+                        token_finalize<TMAX>(t, rmsnorm, a.eps, a.norm_eps, a.inv_k, a.qmax,
+                                             a.inv_rms_in, qs);
                     if (threadIdx.x == 0) {
                         s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, ts.beta), a.qmax);
                         if (blockIdx.x == 0 && a.beta_out) a.beta_out[t] = ts.beta;
@@ -381,7 +340,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             if constexpr (FMT != kFmt2Bit) consumer_barrier();
         } else {
             token_stats<TMAX, true>(xb, T, K, a.gain, a.rmsnorm != 0, a.eps, a.norm_eps,
-                                    a.inv_k, a.qmax, nullptr, qs);
+                                    a.inv_k, a.qmax, a.inv_rms_in, qs);
             token_codes<TMAX, true>(xb, T, K, a.gain, a.rmsnorm != 0, xs, qs);
             if (threadIdx.x < T) {
                 const int t = threadIdx.x;
@@ -806,10 +765,12 @@ bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_o
 bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const uint16_t *X, int64_t T,
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
-                                     int8_t *Xq, float *beta, int32_t *rowsum, void *Y,
-                                     int out_dtype, bool static_weights, int fmt, float qmax,
+                                     const float *inv_rms_in, int8_t *Xq, float *beta,
+                                     int32_t *rowsum, void *Y, int out_dtype,
+                                     bool static_weights, int fmt, float qmax,
                                      cudaStream_t stream) {
     DecodeArgs a = {};
+    a.inv_rms_in = inv_rms_in;
     a.packed = static_cast<const uint8_t *>(packed);
     a.gamma = gamma;
     a.d_out = (int)d_out;

@@ -175,13 +175,17 @@ struct TokenScale {
 
 // Final statistics of token t from the warp partials (fixed warp order); any
 // thread may compute them and every thread gets the same bits.  No gain.
+// inv_rms_in, when given, supplies r.
 template <int TMAX>
 __device__ __forceinline__ TokenScale token_finalize(int t, bool rmsnorm, float eps,
                                                      float norm_eps, double inv_k, float qmax,
+                                                     const float *inv_rms_in,
                                                      const QuantShared<TMAX> &qs) {
     TokenScale ts;
     ts.inv_rms = 1.0f;
-    if (rmsnorm) {
+    if (rmsnorm && inv_rms_in) {
+        ts.inv_rms = __ldg(inv_rms_in + t);
+    } else if (rmsnorm) {
         double s = qs.ss[0][t];
         #pragma unroll
         for (int w = 1; w < kQuantWarps; ++w) s += qs.ss[w][t];
@@ -272,7 +276,8 @@ __device__ __forceinline__ void token_stats(const uint16_t *__restrict__ X, int 
             qs.inv_rms[t] = r;
             qs.beta[t] = __fmul_rn(m, r);
         } else {
-            const TokenScale ts = token_finalize<TMAX>(t, rmsnorm, eps, norm_eps, inv_k, qmax, qs);
+            const TokenScale ts =
+                token_finalize<TMAX>(t, rmsnorm, eps, norm_eps, inv_k, qmax, nullptr, qs);
             qs.inv_rms[t] = ts.inv_rms;
             qs.beta[t] = ts.beta;                    // replaced below when a gain is set
         }

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.bitlinear_version() == 1
+    assert lib.bitlinear_version() == 2
     for code in range(0, 7):
         s = bl.status_string(code)
         assert s and s != "unknown status"
@@ -115,9 +115,9 @@ def test_base3_sizes_and_validation(lib):
     assert fwd(packed=0x10008) == bl.ERR_MISALIGNED
     assert fwd(T=0, xq=0) == bl.OK
     lin = lib.bitlinear_linear_base3
-    assert lin(P(0x10000), P(0x20000), 64, 256, P(0x30000), 17, None, 1, 1e-5, 1e-5,
+    assert lin(P(0x10000), P(0x20000), 64, 256, P(0x30000), 17, None, 1, 1e-5, 1e-5, None,
                P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0) == bl.ERR_UNSUPPORTED_SHAPE
-    assert lin(P(0x10000), P(0x20000), 64, 256, P(0x30000), 4, None, 8, 1e-5, 1e-5,
+    assert lin(P(0x10000), P(0x20000), 64, 256, P(0x30000), 4, None, 8, 1e-5, 1e-5, None,
                P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0) == bl.ERR_INVALID_ARG
     rp = lib.bitlinear_repack_base3
     assert rp(P(0x10000), 16, 128, P(0x20000), S0) == bl.ERR_UNSUPPORTED_SHAPE
@@ -145,9 +145,12 @@ def test_w1_sizes_and_validation(lib):
     assert fwd(packed=0x10004) == bl.ERR_MISALIGNED
     assert fwd(T=0) == bl.OK
     args = (P(0x10000), P(0x20000), 64, 256, P(0x30000), 4, None)
-    tail = (1e-5, 1e-5, P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0)
+    tail = (1e-5, 1e-5, None, P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0)
     assert lib.bitlinear_linear(*args, 1 | bl.ACT_4BIT, *tail) == bl.ERR_INVALID_ARG
     assert lib.bitlinear_linear_w1(*args, 16, *tail) == bl.ERR_INVALID_ARG
+    # A supplied reciprocal RMS must be 4-byte aligned.
+    tail_r = (1e-5, 1e-5, P(0x80002), P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0)
+    assert lib.bitlinear_linear(*args, 1, *tail_r) == bl.ERR_MISALIGNED
     pk = lib.bitlinear_pack_weights_w1
     assert pk(P(0x10000), 16, 128, None, P(0x20000), 1 << 20, P(0x30000), P(0x40000),
               S0) == bl.ERR_UNSUPPORTED_SHAPE

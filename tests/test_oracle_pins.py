@@ -480,6 +480,9 @@ def test_int_matmul_brute_force(T, N, K):
     xq = RNG.integers(-127, 128, size=(T, K)).astype(np.int8)
     acc = oracle.int_matmul(wq, xq)
     np.testing.assert_array_equal(acc, xq.astype(np.int64) @ wq.astype(np.int64).T)
+    # The OpenMP build (every host core, used for the timed CPU baseline)
+    # computes the same exact sums.
+    np.testing.assert_array_equal(oracle.int_matmul(wq, xq, parallel=True), acc)
 
 
 def test_masked_add_identity_exhaustive():
