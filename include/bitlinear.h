@@ -254,6 +254,42 @@ int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
                      cudaStream_t stream);
 
 /*
+ * Plans: a bitlinear_linear call bound once.  For a serving loop that calls
+ * the same layer again and again with new activations ([MF] section 6: the
+ * per-call work -- here argument checks, kernel selection, launch shapes and,
+ * for T > 16, the prefill GEMM's tensor-map descriptors -- is done once).
+ *
+ * bitlinear_linear_plan_create validates the arguments (every argument of
+ * bitlinear_linear except X, inv_rms_in, which a plan does not take, and the
+ * stream; same rules and errors), checks the device, prepares the launches
+ * and returns a plan in *plan (NULL on error).  The plan is a small host
+ * object owned by the caller; it holds no device memory and keeps the
+ * pointers it was given, which must stay valid while it is used.
+ * flags: BITLINEAR_RMSNORM, BITLINEAR_STATIC_WEIGHTS,
+ * BITLINEAR_PER_TENSOR_ABSMAX (2-bit weights only, as bitlinear_linear).
+ *
+ * bitlinear_linear_plan_run enqueues on `stream` exactly what
+ * bitlinear_linear(..., X, ...) with the bound arguments would (the same
+ * kernels and results, bit for bit).  X: bf16 [T][d_in], 16-byte aligned.
+ * The device current at creation must be current; otherwise
+ * BITLINEAR_ERR_DEVICE.  Runs of one plan may be enqueued on any streams;
+ * runs that overlap on the GPU share the plan's output buffers, as two
+ * bitlinear_linear calls on the same buffers would.  A run may be captured
+ * into a CUDA graph.
+ *
+ * bitlinear_plan_destroy frees the plan (NULL is allowed).
+ */
+typedef struct bitlinear_plan bitlinear_plan;
+int bitlinear_linear_plan_create(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                 int64_t d_in, int64_t T, const float *norm_gain,
+                                 uint32_t flags, float eps, float norm_eps, int8_t *Xq,
+                                 float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                 bitlinear_plan **plan);
+int bitlinear_linear_plan_run(const bitlinear_plan *plan, const uint16_t *X,
+                              cudaStream_t stream);
+void bitlinear_plan_destroy(bitlinear_plan *plan);
+
+/*
  * Base-3 weight format ([MF] section 4, "Memory Bandwidth and Latency
  * Bounds": five ternary values fit in one byte, 3^5 = 243 < 256, so a weight
  * costs 1.6 bits instead of 2).  This library's own order: each row is padded

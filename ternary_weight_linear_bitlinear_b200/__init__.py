@@ -73,6 +73,11 @@ SIGNATURES = {
     "bitlinear_backward_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _int, _int]),
     "bitlinear_backward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _int, _vp,
                                   ctypes.c_size_t, _vp]),
+    "bitlinear_linear_plan_create": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _u32, _f32, _f32,
+                                            _vp, _vp, _vp, _vp, _int,
+                                            ctypes.POINTER(ctypes.c_void_p)]),
+    "bitlinear_linear_plan_run": (_int, [_vp, _vp, _vp]),
+    "bitlinear_plan_destroy": (None, [_vp]),
     "bitlinear_device_error": (_int, [_vp, _int]),
     "bitlinear_get_last_device_error": (_int, [_vp]),
     "bitlinear_set_wait_limit_ns": (_int, [ctypes.c_uint64]),
@@ -360,11 +365,15 @@ def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
 
 
 class LinearPlan:
-    """bitlinear_linear with everything but X bound once: the weights, the
-    scratch (Xq, beta, rowsum), the output, the flags and the CUDA stream
-    (`stream`, default: the one current at construction).  Each call passes X's address to the same
-    entry point and returns the bound output tensor (overwritten by the next
-    call).  For a serving loop that calls the same layer shape repeatedly."""
+    """A bitlinear_linear call bound once (bitlinear_linear_plan_create): the
+    weights, the scratch (Xq, beta, rowsum), the output, the flags and the
+    CUDA stream (`stream`, default: the one current at construction).  The
+    library validates the arguments and prepares the kernel launches at
+    construction; each call passes X's address to bitlinear_linear_plan_run
+    and returns the bound output tensor (overwritten by the next call).
+    2-bit weights (PackedTernary); other formats bind bitlinear_linear_base3
+    or bitlinear_linear_w1 each call.  For a serving loop that calls the same
+    layer shape repeatedly."""
 
     def __init__(self, w, T: int, gain: torch.Tensor = None, rmsnorm: bool = True,
                  eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.bfloat16,
@@ -387,19 +396,39 @@ class LinearPlan:
         od = OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32
         self.w, self.scratch, self.out, self.gain = w, scratch, out, gain   # keep alive
         self._shape = (T, w.d_in)
-        self._fn, self._name = _entry(w, "bitlinear_linear")
-        self._pre = (w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in)
-        sh = stream.cuda_stream if stream is not None else _stream()
-        self._post = (T, _ptr(gain), flags, eps, norm_eps, None, Xq.data_ptr(),
-                      beta.data_ptr(), rowsum.data_ptr(), out.data_ptr(), od, sh)
+        self._stream = stream.cuda_stream if stream is not None else _stream()
+        self._handle = None
+        if isinstance(w, PackedTernary):
+            h = ctypes.c_void_p()
+            _check(lib().bitlinear_linear_plan_create(
+                w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in, T, _ptr(gain), flags,
+                eps, norm_eps, Xq.data_ptr(), beta.data_ptr(), rowsum.data_ptr(), out.data_ptr(),
+                od, ctypes.byref(h)), "bitlinear_linear_plan_create")
+            self._handle = h
+            self._run = lib().bitlinear_linear_plan_run
+            self._name = "bitlinear_linear_plan_run"
+        else:
+            self._fn, self._name = _entry(w, "bitlinear_linear")
+            self._pre = (w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in)
+            self._post = (T, _ptr(gain), flags, eps, norm_eps, None, Xq.data_ptr(),
+                          beta.data_ptr(), rowsum.data_ptr(), out.data_ptr(), od, self._stream)
 
     def __call__(self, X: torch.Tensor) -> torch.Tensor:
         if X.dtype != torch.bfloat16 or tuple(X.shape) != self._shape or not X.is_contiguous():
             raise TypeError("X must be a contiguous bf16 tensor of shape %s" % (self._shape,))
-        st = self._fn(*self._pre, X.data_ptr(), *self._post)
+        if self._handle is not None:
+            st = self._run(self._handle, X.data_ptr(), self._stream)
+        else:
+            st = self._fn(*self._pre, X.data_ptr(), *self._post)
         if st != OK:
             raise BitLinearError(st, self._name)
         return self.out
+
+    def __del__(self):
+        h = getattr(self, "_handle", None)
+        if h is not None and _lib is not None:
+            _lib.bitlinear_plan_destroy(h)
+            self._handle = None
 
 
 class StepGraph:

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <new>
 
 #include "bitlinear.h"
 #include "common.cuh"
@@ -27,6 +28,27 @@ bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int
                                      int32_t *rowsum, void *Y, int out_dtype,
                                      bool static_weights, int fmt, float qmax,
                                      cudaStream_t stream);
+bitlinear_status prepare_gemv(const void *packed, const float *gamma, int64_t d_out,
+                              int64_t d_in, const int8_t *Xq, const float *beta,
+                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                              int32_t *acc_out, bool static_weights, int fmt, float qmax,
+                              LaunchRec *rec);
+bitlinear_status prepare_linear_fused(const void *packed, const float *gamma, int64_t d_out,
+                                      int64_t d_in, const uint16_t *X, int64_t T,
+                                      const float *gain, bool rmsnorm, float eps,
+                                      float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                      float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                      bool static_weights, int fmt, float qmax, LaunchRec *rec);
+size_t decode_x_offset();
+bitlinear_status prepare_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
+                                   const float *norm_gain, uint32_t flags, float eps,
+                                   float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                   float *beta, int32_t *rowsum, float *inv_rms_out, bool pdl,
+                                   LaunchRec *rec);
+bitlinear_status prepare_gemm_tc_pair(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                      int64_t d_in, const int8_t *Xq, const float *beta,
+                                      const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                                      int32_t *acc_out, LaunchRec *rec);
 bitlinear_status launch_gemm_tc_pair(const uint32_t *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const int8_t *Xq, const float *beta,
                                      const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
@@ -157,26 +179,42 @@ static bitlinear_status forward_common(const void *packed, const float *gamma, i
                             acc_out, false, fmt, qmax, stream);
 }
 
-static bitlinear_status linear_common(const void *packed, const float *gamma, int64_t d_out,
-                                      int64_t d_in, const uint16_t *X, int64_t T,
-                                      const float *norm_gain, uint32_t flags, float eps,
-                                      float norm_eps, const float *inv_rms_in, int8_t *Xq,
-                                      float *beta, int32_t *rowsum, void *Y, int out_dtype,
-                                      int fmt, cudaStream_t stream) {
+// Argument checks of bitlinear_linear (and of a plan for it), X excluded:
+// everything but the device.
+static bitlinear_status validate_linear(const void *packed, const float *gamma, int64_t d_out,
+                                        int64_t d_in, int64_t T, const float *norm_gain,
+                                        uint32_t flags, float eps, float norm_eps,
+                                        const float *inv_rms_in, int8_t *Xq, float *beta,
+                                        int32_t *rowsum, void *Y, int out_dtype, int fmt) {
     bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, nullptr);
     if (st != BITLINEAR_OK) return st;
     if (fmt != kFmt2Bit && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     uint32_t allowed = BITLINEAR_RMSNORM | BITLINEAR_STATIC_WEIGHTS | BITLINEAR_PER_TENSOR_ABSMAX;
     if (fmt == kFmt1Bit) allowed |= BITLINEAR_ACT_4BIT;   // the A4 of W1A4
     if (flags & ~allowed) return BITLINEAR_ERR_INVALID_ARG;
-    const float qmax = (flags & BITLINEAR_ACT_4BIT) ? 7.0f : 127.0f;
     if (!(eps >= 0.0f) || !std::isfinite(eps) || !(norm_eps >= 0.0f) || !std::isfinite(norm_eps))
         return BITLINEAR_ERR_INVALID_ARG;
     if (T == 0) return BITLINEAR_OK;
-    if (!X || !Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
-    if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4) ||
+    if (!Xq || !beta || !rowsum) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(Xq, 16) || !aligned(beta, 4) || !aligned(rowsum, 4) ||
         (norm_gain && !aligned(norm_gain, 4)) || (inv_rms_in && !aligned(inv_rms_in, 4)))
         return BITLINEAR_ERR_MISALIGNED;
+    return BITLINEAR_OK;
+}
+
+static bitlinear_status linear_common(const void *packed, const float *gamma, int64_t d_out,
+                                      int64_t d_in, const uint16_t *X, int64_t T,
+                                      const float *norm_gain, uint32_t flags, float eps,
+                                      float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                      float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                      int fmt, cudaStream_t stream) {
+    bitlinear_status st = validate_linear(packed, gamma, d_out, d_in, T, norm_gain, flags, eps,
+                                          norm_eps, inv_rms_in, Xq, beta, rowsum, Y, out_dtype,
+                                          fmt);
+    if (st != BITLINEAR_OK || T == 0) return st;
+    if (!X) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(X, 16)) return BITLINEAR_ERR_MISALIGNED;
+    const float qmax = (flags & BITLINEAR_ACT_4BIT) ? 7.0f : 127.0f;
     st = check_device();
     if (st != BITLINEAR_OK) return st;
     const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
@@ -198,6 +236,28 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
 }
 
 }  // namespace bl
+
+// A bound bitlinear_linear call: the validated arguments and the prepared
+// launches, with the activations left to fill in at each run.
+struct bitlinear_plan {
+    int device = -1;
+    int64_t T = 0;
+    int steps = 0;            // 0: nothing to run (T = 0); -1: no prepared launches
+    bl::LaunchRec rec[2];     // rec[0] takes X
+    size_t x_field = 0;       // byte offset of X inside rec[0]'s parameter 0
+    // the call's arguments, for plans run through bitlinear_linear itself
+    const uint32_t *packed = nullptr;
+    const float *gamma = nullptr;
+    int64_t d_out = 0, d_in = 0;
+    const float *norm_gain = nullptr;
+    uint32_t flags = 0;
+    float eps = 0.0f, norm_eps = 0.0f;
+    int8_t *Xq = nullptr;
+    float *beta = nullptr;
+    int32_t *rowsum = nullptr;
+    void *Y = nullptr;
+    int out_dtype = 0;
+};
 
 using namespace bl;
 
@@ -327,3 +387,92 @@ extern "C" int bitlinear_wait_probe(uint64_t limit_ns, cudaStream_t stream) {
     wait_probe_kernel<<<1, 32, 0, stream>>>(ctx);
     return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
+
+extern "C" int bitlinear_linear_plan_create(const uint32_t *packed, const float *gamma,
+                                            int64_t d_out, int64_t d_in, int64_t T,
+                                            const float *norm_gain, uint32_t flags, float eps,
+                                            float norm_eps, int8_t *Xq, float *beta,
+                                            int32_t *rowsum, void *Y, int out_dtype,
+                                            bitlinear_plan **plan) {
+    if (!plan) return BITLINEAR_ERR_INVALID_ARG;
+    *plan = nullptr;
+    bitlinear_status st = validate_linear(packed, gamma, d_out, d_in, T, norm_gain, flags, eps,
+                                          norm_eps, nullptr, Xq, beta, rowsum, Y, out_dtype,
+                                          kFmt2Bit);
+    if (st != BITLINEAR_OK) return st;
+    st = check_device();
+    if (st != BITLINEAR_OK) return st;
+    bitlinear_plan *p = new (std::nothrow) bitlinear_plan();
+    if (!p) return BITLINEAR_ERR_INVALID_ARG;
+    if (cudaGetDevice(&p->device) != cudaSuccess) {
+        delete p;
+        return BITLINEAR_ERR_DEVICE;
+    }
+    p->T = T;
+    p->packed = packed;
+    p->gamma = gamma;
+    p->d_out = d_out;
+    p->d_in = d_in;
+    p->norm_gain = norm_gain;
+    p->flags = flags;
+    p->eps = eps;
+    p->norm_eps = norm_eps;
+    p->Xq = Xq;
+    p->beta = beta;
+    p->rowsum = rowsum;
+    p->Y = Y;
+    p->out_dtype = out_dtype;
+    const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
+    const bool rmsnorm = (flags & BITLINEAR_RMSNORM) != 0;
+    const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
+    if (T == 0) {
+        p->steps = 0;
+    } else if (per_tensor) {
+        p->steps = -1;   // three launches with a folded beta: run as bitlinear_linear
+    } else if (decode_can_fuse(T, d_in)) {
+        st = prepare_linear_fused(packed, gamma, d_out, d_in, nullptr, T, norm_gain, rmsnorm, eps,
+                                  norm_eps, nullptr, Xq, beta, rowsum, Y, out_dtype,
+                                  static_weights, kFmt2Bit, 127.0f, &p->rec[0]);
+        p->x_field = decode_x_offset();
+        p->steps = 1;
+    } else {
+        st = prepare_quant_act(nullptr, T, d_in, norm_gain, flags & BITLINEAR_RMSNORM, eps,
+                               norm_eps, nullptr, Xq, beta, rowsum, nullptr, true, &p->rec[0]);
+        p->x_field = 0;
+        if (st == BITLINEAR_OK)
+            st = T <= 16 ? prepare_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y,
+                                        out_dtype, nullptr, static_weights, kFmt2Bit, 127.0f,
+                                        &p->rec[1])
+                         : prepare_gemm_tc_pair(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y,
+                                                out_dtype, nullptr, &p->rec[1]);
+        p->steps = 2;
+    }
+    if (st != BITLINEAR_OK) {
+        delete p;
+        return st;
+    }
+    *plan = p;
+    return BITLINEAR_OK;
+}
+
+extern "C" int bitlinear_linear_plan_run(const bitlinear_plan *plan, const uint16_t *X,
+                                         cudaStream_t stream) {
+    if (!plan) return BITLINEAR_ERR_INVALID_ARG;
+    if (plan->steps == 0) return BITLINEAR_OK;
+    if (!X) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(X, 16)) return BITLINEAR_ERR_MISALIGNED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) return BITLINEAR_ERR_DEVICE;
+    if (plan->steps < 0)
+        return linear_common(plan->packed, plan->gamma, plan->d_out, plan->d_in, X, plan->T,
+                             plan->norm_gain, plan->flags, plan->eps, plan->norm_eps, nullptr,
+                             plan->Xq, plan->beta, plan->rowsum, plan->Y, plan->out_dtype,
+                             kFmt2Bit, stream);
+    LaunchRec first = plan->rec[0];
+    first.patch_ptr(0, plan->x_field, X);
+    if (first.launch(stream) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+    if (plan->steps == 2 && plan->rec[1].launch(stream) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+    return BITLINEAR_OK;
+}
+
+extern "C" void bitlinear_plan_destroy(bitlinear_plan *plan) { delete plan; }

@@ -1,7 +1,9 @@
 // common.cuh -- device helpers shared by the library's kernels (sm_100a).
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
+#include <cstring>
 #include <cuda_runtime.h>
 
 #include "bitlinear.h"
@@ -34,6 +36,62 @@ bitlinear_status check_device();
 inline bool aligned(const void *p, uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
+
+// A prepared kernel launch: the kernel, its launch shape and copies of its
+// parameters, so that a launch can be repeated with one pointer patched
+// (the activations of a plan, see bitlinear_linear_plan_run) without
+// recomputing anything.  Every entry point launches through one of these,
+// so a plan and a direct call run the same launch.
+struct LaunchRec {
+    const void *func = nullptr;
+    dim3 grid{1, 1, 1}, block{1, 1, 1};
+    size_t smem = 0;
+    unsigned cluster_x = 0;   // 0: no cluster attribute
+    bool pdl = false;         // programmatic dependent launch
+    int nargs = 0;
+    size_t off[16] = {};
+    size_t used = 0;
+    alignas(128) unsigned char buf[1024];
+
+    template <class V>
+    void push(const V &v) {
+        const size_t a = alignof(V);
+        used = (used + a - 1) & ~(a - 1);
+        std::memcpy(buf + used, &v, sizeof(V));
+        off[nargs++] = used;
+        used += sizeof(V);
+    }
+    // Overwrite the pointer at byte `field` of parameter `arg`.
+    void patch_ptr(int arg, size_t field, const void *p) {
+        std::memcpy(buf + off[arg] + field, &p, sizeof p);
+    }
+    cudaError_t launch(cudaStream_t stream) const {
+        void *argv[16];
+        for (int i = 0; i < nargs; ++i) argv[i] = const_cast<unsigned char *>(buf + off[i]);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        int na = 0;
+        if (cluster_x) {
+            attr[na].id = cudaLaunchAttributeClusterDimension;
+            attr[na].val.clusterDim.x = cluster_x;
+            attr[na].val.clusterDim.y = 1;
+            attr[na].val.clusterDim.z = 1;
+            ++na;
+        }
+        if (pdl) {
+            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        return cudaLaunchKernelExC(&cfg, func, argv);
+    }
+};
 
 // ------------------------------------------------------------- rounding --
 // RoundClip's floor(z + 0.5), evaluated exactly on a binary32 z: with

@@ -533,10 +533,11 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
 // Launches the CTA-pair kernel: 2 x min(pair tiles, SMs / 2) CTAs in clusters
 // of two, one pair per two SMs.  A pair tile spans as many SMs as two 128-row
 // single-CTA tiles would, so every problem uses the pair form.
-bitlinear_status launch_gemm_tc_pair(const uint32_t *packed, const float *gamma, int64_t d_out,
-                                     int64_t d_in, const int8_t *Xq, const float *beta,
-                                     const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                                     int32_t *acc_out, cudaStream_t stream) {
+// The prefill GEMM's launch (both tensor maps encoded) as a launch record.
+bitlinear_status prepare_gemm_tc_pair(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                      int64_t d_in, const int8_t *Xq, const float *beta,
+                                      const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                                      int32_t *acc_out, LaunchRec *rec) {
     using namespace pair;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -581,23 +582,36 @@ bitlinear_status launch_gemm_tc_pair(const uint32_t *packed, const float *gamma,
     const int64_t max_pairs = sms / 2 > 0 ? sms / 2 : 1;
     const int64_t pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
 
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * pairs));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map_x, map_w, gamma, (int)d_out, (int)d_in,
-                                       beta, rowsum, (int)T, Y, acc_out, ctx);
-    return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+    *rec = LaunchRec();
+    rec->func = (const void *)kern;
+    rec->grid = dim3((unsigned)(2 * pairs));
+    rec->block = dim3(kThreads);
+    rec->smem = kSmemBytes;
+    rec->cluster_x = 2;
+    rec->pdl = true;
+    rec->push(map_x);
+    rec->push(map_w);
+    rec->push(gamma);
+    rec->push((int)d_out);
+    rec->push((int)d_in);
+    rec->push(beta);
+    rec->push(rowsum);
+    rec->push((int)T);
+    rec->push(Y);
+    rec->push(acc_out);
+    rec->push(ctx);
+    return BITLINEAR_OK;
+}
+
+bitlinear_status launch_gemm_tc_pair(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                     int64_t d_in, const int8_t *Xq, const float *beta,
+                                     const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                                     int32_t *acc_out, cudaStream_t stream) {
+    LaunchRec rec;
+    bitlinear_status st = prepare_gemm_tc_pair(packed, gamma, d_out, d_in, Xq, beta, rowsum, T,
+                                               Y, out_dtype, acc_out, &rec);
+    if (st != BITLINEAR_OK) return st;
+    return rec.launch(stream) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
 }  // namespace bl

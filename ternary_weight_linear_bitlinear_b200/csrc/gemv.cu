@@ -71,6 +71,7 @@
 // Every mbarrier wait is bounded; on expiry the CTA stops consuming, the
 // producer waits (bounded) for the copies it issued, and the error word is
 // set.
+#include <cstddef>
 #include <cstdint>
 
 #include <cuda_bf16.h>
@@ -636,8 +637,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
 constexpr int kFusedMaxCodeBytes = BL_FUSED_MAX_CODE_BYTES;
 
 template <int NT, int R, bool FUSED, bool OUT_BF16, int FMT>
-static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
-                                   cudaStream_t stream) {
+static cudaError_t prepare_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
+                                    LaunchRec *rec) {
     constexpr int kTileBytes = FMT == kFmtBase3 ? 512 : 1024;
     constexpr int kTileCols = FMT == kFmtBase3 ? 160 : (FMT == kFmt1Bit ? 512 : 256);
     const int n_rt = args.d_out / 16;
@@ -679,32 +680,31 @@ static cudaError_t launch_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
     if (max_ctas < sms) max_ctas = sms;
     const int grid = n_groups < max_ctas ? n_groups : max_ctas;
 
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args, plan, ctx);
+    *rec = LaunchRec();
+    rec->func = (const void *)kern;
+    rec->grid = dim3((unsigned)grid);
+    rec->block = dim3(kDecThreads);
+    rec->smem = smem;
+    rec->pdl = true;
+    rec->push(args);
+    rec->push(plan);
+    rec->push(ctx);
+    return cudaSuccess;
 }
 
 template <bool FUSED, bool OUT_BF16, int FMT>
-static cudaError_t launch_decode_r(const DecodeArgs &args, const DeviceCtx &ctx,
-                                   cudaStream_t stream) {
+static cudaError_t prepare_decode_r(const DecodeArgs &args, const DeviceCtx &ctx,
+                                    LaunchRec *rec) {
     // One row tile per group while that still leaves a few CTAs per SM;
     // larger matrices share each activation fragment over two row tiles.
     const int n_rt = args.d_out / 16;
     const bool wide = n_rt >= BL_DEC_WIDE_ROW_TILES;
     if (args.T <= 8)
-        return wide ? launch_decode_t<1, 2, FUSED, OUT_BF16, FMT>(args, ctx, stream)
-                    : launch_decode_t<1, 1, FUSED, OUT_BF16, FMT>(args, ctx, stream);
+        return wide ? prepare_decode_t<1, 2, FUSED, OUT_BF16, FMT>(args, ctx, rec)
+                    : prepare_decode_t<1, 1, FUSED, OUT_BF16, FMT>(args, ctx, rec);
     if constexpr (FUSED) return cudaErrorInvalidValue;   // fused path is T <= 8 only
-    return wide ? launch_decode_t<2, 2, false, OUT_BF16, FMT>(args, ctx, stream)
-                : launch_decode_t<2, 1, false, OUT_BF16, FMT>(args, ctx, stream);
+    return wide ? prepare_decode_t<2, 2, false, OUT_BF16, FMT>(args, ctx, rec)
+                : prepare_decode_t<2, 1, false, OUT_BF16, FMT>(args, ctx, rec);
 }
 
 bool decode_can_fuse(int64_t T, int64_t d_in) {
@@ -712,17 +712,20 @@ bool decode_can_fuse(int64_t T, int64_t d_in) {
 }
 
 template <int FMT>
-static cudaError_t launch_decode_f(const DecodeArgs &args, bool fused, bool bf,
-                                   const DeviceCtx &ctx, cudaStream_t stream) {
+static cudaError_t prepare_decode_f(const DecodeArgs &args, bool fused, bool bf,
+                                    const DeviceCtx &ctx, LaunchRec *rec) {
     if (fused)
-        return bf ? launch_decode_r<true, true, FMT>(args, ctx, stream)
-                  : launch_decode_r<true, false, FMT>(args, ctx, stream);
-    return bf ? launch_decode_r<false, true, FMT>(args, ctx, stream)
-              : launch_decode_r<false, false, FMT>(args, ctx, stream);
+        return bf ? prepare_decode_r<true, true, FMT>(args, ctx, rec)
+                  : prepare_decode_r<true, false, FMT>(args, ctx, rec);
+    return bf ? prepare_decode_r<false, true, FMT>(args, ctx, rec)
+              : prepare_decode_r<false, false, FMT>(args, ctx, rec);
 }
 
-bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, int fmt,
-                               cudaStream_t stream) {
+// The decode kernel's launch for `args` (kernel choice, shared-memory plan,
+// grid) as a launch record; its parameter 0 is the DecodeArgs, whose X field
+// sits at decode_x_offset().
+static bitlinear_status prepare_decode(DecodeArgs args, bool fused, int out_dtype, int fmt,
+                                       LaunchRec *rec) {
     DeviceCtx ctx;
     bitlinear_status st = get_ctx(&ctx);
     if (st != BITLINEAR_OK) return st;
@@ -730,22 +733,31 @@ bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, int f
     cudaError_t e;
     if (fmt == kFmtBase3) {
         args.kb_total = (args.d_in + 159) / 160;
-        e = launch_decode_f<kFmtBase3>(args, fused, bf, ctx, stream);
+        e = prepare_decode_f<kFmtBase3>(args, fused, bf, ctx, rec);
     } else if (fmt == kFmt1Bit) {
         args.kb_total = (args.d_in + 511) / 512;
-        e = launch_decode_f<kFmt1Bit>(args, fused, bf, ctx, stream);
+        e = prepare_decode_f<kFmt1Bit>(args, fused, bf, ctx, rec);
     } else {
         args.kb_total = args.d_in / 256;
-        e = launch_decode_f<kFmt2Bit>(args, fused, bf, ctx, stream);
+        e = prepare_decode_f<kFmt2Bit>(args, fused, bf, ctx, rec);
     }
     return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
-bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_out,
-                             int64_t d_in, const int8_t *Xq, const float *beta,
-                             const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                             int32_t *acc_out, bool static_weights, int fmt, float qmax,
-                             cudaStream_t stream) {
+size_t decode_x_offset() { return offsetof(DecodeArgs, X); }
+
+bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, int fmt,
+                               cudaStream_t stream) {
+    LaunchRec rec;
+    bitlinear_status st = prepare_decode(args, fused, out_dtype, fmt, &rec);
+    if (st != BITLINEAR_OK) return st;
+    return rec.launch(stream) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+static DecodeArgs gemv_args(const void *packed, const float *gamma, int64_t d_out,
+                            int64_t d_in, const int8_t *Xq, const float *beta,
+                            const int32_t *rowsum, int64_t T, void *Y, int32_t *acc_out,
+                            bool static_weights, float qmax) {
     DecodeArgs a = {};
     a.packed = static_cast<const uint8_t *>(packed);
     a.gamma = gamma;
@@ -759,16 +771,35 @@ bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_o
     a.acc_out = acc_out;
     a.static_weights = static_weights ? 1 : 0;
     a.qmax = qmax;
-    return launch_decode(a, false, out_dtype, fmt, stream);
+    return a;
 }
 
-bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
-                                     int64_t d_in, const uint16_t *X, int64_t T,
-                                     const float *gain, bool rmsnorm, float eps, float norm_eps,
-                                     const float *inv_rms_in, int8_t *Xq, float *beta,
-                                     int32_t *rowsum, void *Y, int out_dtype,
-                                     bool static_weights, int fmt, float qmax,
-                                     cudaStream_t stream) {
+bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_out,
+                             int64_t d_in, const int8_t *Xq, const float *beta,
+                             const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                             int32_t *acc_out, bool static_weights, int fmt, float qmax,
+                             cudaStream_t stream) {
+    return launch_decode(gemv_args(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, acc_out,
+                                   static_weights, qmax),
+                         false, out_dtype, fmt, stream);
+}
+
+bitlinear_status prepare_gemv(const void *packed, const float *gamma, int64_t d_out,
+                              int64_t d_in, const int8_t *Xq, const float *beta,
+                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                              int32_t *acc_out, bool static_weights, int fmt, float qmax,
+                              LaunchRec *rec) {
+    return prepare_decode(gemv_args(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, acc_out,
+                                    static_weights, qmax),
+                          false, out_dtype, fmt, rec);
+}
+
+bitlinear_status prepare_linear_fused(const void *packed, const float *gamma, int64_t d_out,
+                                      int64_t d_in, const uint16_t *X, int64_t T,
+                                      const float *gain, bool rmsnorm, float eps,
+                                      float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                      float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                      bool static_weights, int fmt, float qmax, LaunchRec *rec) {
     DecodeArgs a = {};
     a.inv_rms_in = inv_rms_in;
     a.packed = static_cast<const uint8_t *>(packed);
@@ -788,7 +819,22 @@ bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int
     a.Y = Y;
     a.static_weights = static_weights ? 1 : 0;
     a.qmax = qmax;
-    return launch_decode(a, true, out_dtype, fmt, stream);
+    return prepare_decode(a, true, out_dtype, fmt, rec);
+}
+
+bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
+                                     int64_t d_in, const uint16_t *X, int64_t T,
+                                     const float *gain, bool rmsnorm, float eps, float norm_eps,
+                                     const float *inv_rms_in, int8_t *Xq, float *beta,
+                                     int32_t *rowsum, void *Y, int out_dtype,
+                                     bool static_weights, int fmt, float qmax,
+                                     cudaStream_t stream) {
+    LaunchRec rec;
+    bitlinear_status st = prepare_linear_fused(packed, gamma, d_out, d_in, X, T, gain, rmsnorm,
+                                               eps, norm_eps, inv_rms_in, Xq, beta, rowsum, Y,
+                                               out_dtype, static_weights, fmt, qmax, &rec);
+    if (st != BITLINEAR_OK) return st;
+    return rec.launch(stream) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
 }  // namespace bl

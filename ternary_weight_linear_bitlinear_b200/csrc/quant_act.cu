@@ -100,6 +100,34 @@ __global__ void __launch_bounds__(kBetaMaxThreads) beta_max_kernel(float *beta, 
     }
 }
 
+// The per-token quantiser's launch as a launch record (parameter 0 is X).
+bitlinear_status prepare_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
+                                   const float *norm_gain, uint32_t flags, float eps,
+                                   float norm_eps, const float *inv_rms_in, int8_t *Xq,
+                                   float *beta, int32_t *rowsum, float *inv_rms_out, bool pdl,
+                                   LaunchRec *rec) {
+    *rec = LaunchRec();
+    rec->func = (const void *)quant_act_kernel;
+    rec->grid = dim3((unsigned)T);
+    rec->block = dim3(kQuantThreads);
+    rec->pdl = pdl;
+    rec->push(X);
+    rec->push((int)d_in);
+    rec->push(norm_gain);
+    rec->push((flags & BITLINEAR_RMSNORM) ? 1 : 0);
+    rec->push(eps);
+    rec->push(norm_eps);
+    rec->push(1.0 / (double)d_in);
+    rec->push((flags & BITLINEAR_ACT_4BIT) ? 7.0f : 127.0f);
+    rec->push(inv_rms_in);
+    rec->push(Xq);
+    rec->push(beta);
+    rec->push(rowsum);
+    rec->push(inv_rms_out);
+    rec->push((int)kQuantPerToken);
+    return BITLINEAR_OK;
+}
+
 bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                                   const float *norm_gain, uint32_t flags, float eps,
                                   float norm_eps, const float *inv_rms_in, int8_t *Xq,
@@ -107,6 +135,12 @@ bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                                   cudaStream_t stream) {
     const int rmsnorm = (flags & BITLINEAR_RMSNORM) ? 1 : 0;
     const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
+    if (!per_tensor) {
+        LaunchRec rec;
+        prepare_quant_act(X, T, d_in, norm_gain, flags, eps, norm_eps, inv_rms_in, Xq, beta,
+                          rowsum, inv_rms_out, pdl, &rec);
+        return rec.launch(stream) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)T);
     cfg.blockDim = dim3(kQuantThreads);
@@ -119,14 +153,7 @@ bitlinear_status launch_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
     const double inv_k = 1.0 / (double)d_in;
     // Q_b - 1 for 8-bit codes (127) or, under BITLINEAR_ACT_4BIT, 4-bit (7).
     const float qmax = (flags & BITLINEAR_ACT_4BIT) ? 7.0f : 127.0f;
-    cudaError_t e;
-    if (!per_tensor) {
-        e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
-                               norm_eps, inv_k, qmax, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
-                               (int)kQuantPerToken);
-        return e == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
-    }
-    e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
+    cudaError_t e = cudaLaunchKernelEx(&cfg, quant_act_kernel, X, (int)d_in, norm_gain, rmsnorm, eps,
                            norm_eps, inv_k, qmax, inv_rms_in, Xq, beta, rowsum, inv_rms_out,
                            (int)kQuantStatsOnly);
     if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;

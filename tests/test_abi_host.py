@@ -208,3 +208,25 @@ def test_no_device_fails_loudly(lib):
     assert _fwd(lib) == bl.ERR_DEVICE
     with pytest.raises((RuntimeError, TypeError)):
         bl.quant_act(torch.zeros(2, 256, dtype=torch.bfloat16))
+
+
+def test_plan_validation(lib):
+    """bitlinear_linear_plan_create checks the bound arguments like
+    bitlinear_linear, before it looks at the device."""
+    import ctypes as C
+    h = C.c_void_p()
+    mk = lib.bitlinear_linear_plan_create
+
+    def create(d_in=256, T=4, flags=1, xq=0x30000, plan=True):
+        return mk(P(0x10000), P(0x20000), 64, d_in, T, None, flags, 1e-5, 1e-5, P(xq),
+                  P(0x40000), P(0x50000), P(0x60000), 0, C.byref(h) if plan else None)
+
+    assert create(plan=False) == bl.ERR_INVALID_ARG
+    assert create(d_in=300) == bl.ERR_UNSUPPORTED_SHAPE
+    assert create(flags=bl.ACT_4BIT | 1) == bl.ERR_INVALID_ARG      # 2-bit weights only
+    assert create(xq=0x30001) == bl.ERR_MISALIGNED
+    assert lib.bitlinear_linear_plan_run(None, P(0x1000), S0) == bl.ERR_INVALID_ARG
+    lib.bitlinear_plan_destroy(None)
+    if not torch.cuda.is_available():
+        assert create() == bl.ERR_DEVICE
+        assert h.value is None

@@ -487,6 +487,52 @@ def test_linear_plan_matches_linear():
         plan(Xd.float())
 
 
+PLAN_CASES = [
+    # (d_out, d_in, T, flags)   the path each bound call takes
+    (6912, 2560, 1, bl.RMSNORM | bl.STATIC_WEIGHTS),     # fused quantiser + GEMV
+    (272, 4096, 12, bl.RMSNORM),                           # quantiser, then GEMV
+    (512, 1024, 300, bl.RMSNORM | bl.STATIC_WEIGHTS),     # quantiser, then prefill GEMM
+    (272, 1024, 5, bl.RMSNORM | bl.PER_TENSOR_ABSMAX),     # run as bitlinear_linear
+    (144, 512, 3, 0),                                      # no RMSNorm
+]
+
+
+@pytest.mark.parametrize("d_out,d_in,T,flags", PLAN_CASES)
+def test_plan_runs_equal_linear(d_out, d_in, T, flags):
+    """bitlinear_linear_plan_run gives the bits of bitlinear_linear with the
+    same arguments, on every path, run after run with new activations."""
+    import ctypes as C
+    W = draw(Problem("pl", d_in, d_out, T, 0.02, 0.01, 50.0, 31))[0]
+    w = bl.pack_weights(W.to(dev()), EPS)
+    sc = guarded_scratch(T, d_in)
+    gy = Guarded((T, d_out), torch.bfloat16)
+    h = C.c_void_p()
+    L = bl.lib()
+    assert L.bitlinear_linear_plan_create(
+        w.packed.data_ptr(), w.gamma.data_ptr(), d_out, d_in, T, None, flags, EPS, NORM_EPS,
+        sc[0].t.data_ptr(), sc[1].t.data_ptr(), sc[2].t.data_ptr(), gy.t.data_ptr(),
+        bl.OUT_BF16, C.byref(h)) == bl.OK
+    try:
+        gen = torch.Generator().manual_seed(9)
+        for _ in range(3):
+            X = (torch.randn(T, d_in, generator=gen) * 2).to(torch.bfloat16).to(dev())
+            assert L.bitlinear_linear_plan_run(h, X.data_ptr(),
+                                               torch.cuda.current_stream().cuda_stream) == bl.OK
+            ref = bl.linear(w, X, rmsnorm=bool(flags & bl.RMSNORM), out_dtype=torch.bfloat16,
+                            static_weights=bool(flags & bl.STATIC_WEIGHTS),
+                            per_tensor=bool(flags & bl.PER_TENSOR_ABSMAX))
+            check_all(gy, *sc)
+            assert torch.equal(gy.t, ref)
+    finally:
+        L.bitlinear_plan_destroy(h)
+    # T = 0: a plan that enqueues nothing.
+    assert L.bitlinear_linear_plan_create(
+        w.packed.data_ptr(), w.gamma.data_ptr(), d_out, d_in, 0, None, flags, EPS, NORM_EPS,
+        None, None, None, None, bl.OUT_BF16, C.byref(h)) == bl.OK
+    assert L.bitlinear_linear_plan_run(h, None, None) == bl.OK
+    L.bitlinear_plan_destroy(h)
+
+
 def test_step_graph_replays_copies_and_calls():
     """A StepGraph of (pinned host X -> device, LinearPlan, device Y -> pinned
     host) gives, for new host contents on every replay, the same bits as an
