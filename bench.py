@@ -287,7 +287,7 @@ class DecodeRun:
         self.problems = problems
         self.dev = dev
         self.out_dtype = out_dtype
-        self.layers = []      # (problem, PackedTernary, X, scratch, Y, Xq-state)
+        self.layers = []      # (problem, PackedTernary, X, scratch, Y, split workspace)
         base = []
         for p in problems:
             W, X = draw(p)
@@ -311,10 +311,11 @@ class DecodeRun:
                            torch.empty(T, dtype=torch.float32, device=dev),
                            torch.empty(T, dtype=torch.int32, device=dev))
                 Y = torch.empty((T, p.d_out), dtype=out_dtype, device=dev)
-                self.layers.append((p, w, X, scratch, Y))
+                ws = bl.decode_workspace(p.d_out, T, dev)
+                self.layers.append((p, w, X, scratch, Y, ws))
         torch.cuda.synchronize()
         # Pre-quantised activations for the product-only timing.
-        for p, w, X, scratch, Y in self.layers:
+        for p, w, X, scratch, Y, _ in self.layers:
             xq, beta, rowsum, _ = bl.quant_act(X, act_bits=self.act_bits)
             scratch[0].copy_(xq)
             scratch[1].copy_(beta)
@@ -322,13 +323,14 @@ class DecodeRun:
         torch.cuda.synchronize()
 
     def step(self):
-        for p, w, X, scratch, Y in self.layers:
+        for p, w, X, scratch, Y, ws in self.layers:
             self.bl.linear(w, X, out=Y, scratch=scratch, static_weights=True,
-                           act_bits=self.act_bits)
+                           act_bits=self.act_bits, workspace=ws)
 
     def product_only(self):
-        for p, w, X, scratch, Y in self.layers:
-            self.bl.forward(w, scratch[0], scratch[1], scratch[2], out=Y, act_bits=self.act_bits)
+        for p, w, X, scratch, Y, ws in self.layers:
+            self.bl.forward(w, scratch[0], scratch[1], scratch[2], out=Y, act_bits=self.act_bits,
+                            workspace=ws)
 
     def bytes(self):
         ob = 2 if self.out_dtype == torch.bfloat16 else 4
@@ -620,8 +622,8 @@ def measure_e2e(run, steps):
     replayed) and, for comparison, eagerly."""
     bl = run.bl
     dev = run.dev
-    xs = [X for _, _, X, _, _ in run.layers]
-    ys = [Y for *_, Y in run.layers]
+    xs = [X for _, _, X, _, _, _ in run.layers]
+    ys = [Y for _, _, _, _, Y, _ in run.layers]
     x_elems = [x.numel() for x in xs]
     y_elems = [y.numel() for y in ys]
     host_x = torch.cat([x.reshape(-1) for x in xs]).cpu().pin_memory()
@@ -638,7 +640,7 @@ def measure_e2e(run, steps):
     d2h = host_y.numel() * host_y.element_size()
     cs = torch.cuda.Stream()
     plans = [bl.LinearPlan(w, X.shape[0], out=Y, scratch=scratch, static_weights=True, stream=cs)
-             for (_, w, _, scratch, _), X, Y in zip(run.layers, x_views, y_views)]
+             for (_, w, _, scratch, _, _), X, Y in zip(run.layers, x_views, y_views)]
 
     def one():
         dev_x.copy_(host_x, non_blocking=True)

@@ -18,7 +18,8 @@
  * Conventions for every entry point
  *   - All array arguments are DEVICE pointers on the current CUDA device,
  *     owned by the caller; the library allocates nothing and keeps no
- *     pointer after the call returns.
+ *     pointer after the call returns (plans, below, are the exception: they
+ *     keep the pointers they were given and own a small workspace).
  *   - All work is enqueued on `stream` (0 = legacy default stream); no entry
  *     point synchronises except bitlinear_device_error and
  *     bitlinear_get_last_device_error.
@@ -94,7 +95,7 @@ typedef enum {
  * Q_b - 1 = 7, codes in [-7, 7] (still stored one per int8). */
 #define BITLINEAR_ACT_4BIT 8u
 
-/* Library ABI version (this header: 2). */
+/* Library ABI version (this header: 3). */
 int bitlinear_version(void);
 
 /* Static description of a status code.  Never NULL. */
@@ -224,11 +225,41 @@ int bitlinear_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
  * tiles expanded in shared memory, tcgen05 int8 MMA on clusters of two CTAs,
  * TMEM accumulators).  The prefill GEMM launches clusters of two CTAs of
  * about 215 KiB of shared memory each, one pair per two SMs.
+ *
+ * workspace, workspace_bytes: optional (NULL, 0) split workspace of the
+ * decode product (T <= 16), caller-owned: at least
+ * bitlinear_decode_workspace_bytes(d_out, T) bytes (else
+ * BITLINEAR_ERR_INVALID_ARG), 16-byte aligned, zero-filled before its first
+ * use.  Every call that runs to completion leaves it zero again, so one
+ * workspace serves any sequence of calls on one stream; calls that may
+ * overlap on the GPU need workspaces of their own.  With it, a matrix whose
+ * 16-row tiles do not divide evenly over the resident CTAs has its
+ * (rows, k-tile) units split evenly instead, the CTAs sharing a row tile
+ * adding exact int32 partial sums (the results are the same integers).
+ * Ignored for T > 16.
  */
 int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
                       int64_t d_in, const int8_t *Xq, const float *beta,
                       const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                      int32_t *acc_out, cudaStream_t stream);
+                      int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                      cudaStream_t stream);
+
+/* Bytes of the split workspace of a decode product with d_out outputs and T
+ * tokens (1 <= T <= 16), or 0 for other T or an unsupported d_out:
+ * 8 * 16 * (d_out / 16 + 1) * T rounded up to a multiple of 256. */
+size_t bitlinear_decode_workspace_bytes(int64_t d_out, int64_t T);
+
+/* When decode calls given a split workspace split their units (process-wide;
+ * calls and plans made afterwards follow it): BITLINEAR_SPLIT_AUTO (default:
+ * when the 16-row tiles do not divide evenly over the resident CTAs and each
+ * CTA gets at least two tiles' worth), BITLINEAR_SPLIT_ALWAYS (every decode
+ * call with a workspace, whatever its size: for tests), BITLINEAR_SPLIT_NEVER.
+ * The results are the same integers in every mode.  Returns
+ * BITLINEAR_ERR_INVALID_ARG for another value. */
+#define BITLINEAR_SPLIT_AUTO 0
+#define BITLINEAR_SPLIT_ALWAYS 1
+#define BITLINEAR_SPLIT_NEVER 2
+int bitlinear_set_decode_split(int mode);
 
 /*
  * bitlinear_linear -- the whole BitLinear forward from bf16 activations:
@@ -244,14 +275,15 @@ int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
  * product kernel is its programmatic dependent.  Kernels are launched as
  * programmatic dependents of the work before them and read nothing earlier
  * work produces before their dependency wait, except the weights under
- * BITLINEAR_STATIC_WEIGHTS.
+ * BITLINEAR_STATIC_WEIGHTS.  workspace, workspace_bytes: the optional split
+ * workspace, as in bitlinear_forward.
  */
 int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
                      int64_t d_in, const uint16_t *X, int64_t T,
                      const float *norm_gain, uint32_t flags, float eps,
                      float norm_eps, const float *inv_rms_in, int8_t *Xq,
                      float *beta, int32_t *rowsum, void *Y, int out_dtype,
-                     cudaStream_t stream);
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Plans: a bitlinear_linear call bound once.  For a serving loop that calls
@@ -263,8 +295,11 @@ int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
  * bitlinear_linear except X, inv_rms_in, which a plan does not take, and the
  * stream; same rules and errors), checks the device, prepares the launches
  * and returns a plan in *plan (NULL on error).  The plan is a small host
- * object owned by the caller; it holds no device memory and keeps the
- * pointers it was given, which must stay valid while it is used.
+ * object owned by the caller; it keeps the pointers it was given, which must
+ * stay valid while it is used, and, when its decode product splits its
+ * units (see bitlinear_forward), owns a split workspace in device memory
+ * (bitlinear_decode_workspace_bytes(d_out, T) bytes; BITLINEAR_ERR_CUDA if
+ * it cannot be allocated).
  * flags: BITLINEAR_RMSNORM, BITLINEAR_STATIC_WEIGHTS,
  * BITLINEAR_PER_TENSOR_ABSMAX (2-bit weights only, as bitlinear_linear).
  *
@@ -273,11 +308,12 @@ int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
  * kernels and results, bit for bit).  X: bf16 [T][d_in], 16-byte aligned.
  * The device current at creation must be current; otherwise
  * BITLINEAR_ERR_DEVICE.  Runs of one plan may be enqueued on any streams;
- * runs that overlap on the GPU share the plan's output buffers, as two
- * bitlinear_linear calls on the same buffers would.  A run may be captured
- * into a CUDA graph.
+ * runs that overlap on the GPU share the plan's output buffers and its
+ * workspace, as two bitlinear_linear calls on the same buffers would, and
+ * must not.  A run may be captured into a CUDA graph.
  *
- * bitlinear_plan_destroy frees the plan (NULL is allowed).
+ * bitlinear_plan_destroy frees the plan and its workspace (NULL is allowed);
+ * no run of it may still be in flight.
  */
 typedef struct bitlinear_plan bitlinear_plan;
 int bitlinear_linear_plan_create(const uint32_t *packed, const float *gamma, int64_t d_out,
@@ -329,7 +365,8 @@ int bitlinear_repack_base3(const uint32_t *packed, int64_t d_out, int64_t d_in,
 int bitlinear_forward_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
                             int64_t d_in, const int8_t *Xq, const float *beta,
                             const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                            int32_t *acc_out, cudaStream_t stream);
+                            int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
 
 /*
  * bitlinear_linear_base3 -- bitlinear_linear on base-3 weights (same
@@ -341,7 +378,7 @@ int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma, int64_t d
                            const float *norm_gain, uint32_t flags, float eps,
                            float norm_eps, const float *inv_rms_in, int8_t *Xq,
                            float *beta, int32_t *rowsum, void *Y, int out_dtype,
-                           cudaStream_t stream);
+                           void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * W1A4: binary weights with 4-bit activations, the regime "The End of Matrix
@@ -388,7 +425,8 @@ int bitlinear_pack_weights_w1(const float *W, int64_t d_out, int64_t d_in,
 int bitlinear_forward_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
                          int64_t d_in, const int8_t *Xq, const float *beta,
                          const int32_t *rowsum, int64_t T, int act_bits, void *Y, int out_dtype,
-                         int32_t *acc_out, cudaStream_t stream);
+                         int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
 
 /*
  * bitlinear_linear_w1 -- bitlinear_linear on 1-bit weights: quantise (with
@@ -401,7 +439,7 @@ int bitlinear_linear_w1(const uint32_t *packed1, const float *gamma, int64_t d_o
                         int64_t d_in, const uint16_t *X, int64_t T, const float *norm_gain,
                         uint32_t flags, float eps, float norm_eps, const float *inv_rms_in,
                         int8_t *Xq, float *beta, int32_t *rowsum, void *Y, int out_dtype,
-                        cudaStream_t stream);
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * bitlinear_dense_bf16_forward -- the dense bf16 linear layer Y = X W^T that

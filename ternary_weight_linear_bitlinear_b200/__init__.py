@@ -53,22 +53,24 @@ SIGNATURES = {
     "bitlinear_quant_act": (_int, [_vp, _i64, _i64, _vp, _u32, _f32, _f32, _vp, _vp, _vp,
                                    _vp, _vp, _vp]),
     "bitlinear_forward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int,
-                                 _vp, _vp]),
+                                 _vp, _vp, ctypes.c_size_t, _vp]),
+    "bitlinear_decode_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "bitlinear_set_decode_split": (_int, [_int]),
     "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32, _vp,
-                                _vp, _vp, _vp, _vp, _int, _vp]),
+                                _vp, _vp, _vp, _vp, _int, _vp, ctypes.c_size_t, _vp]),
     "bitlinear_base3_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bitlinear_repack_base3": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "bitlinear_forward_base3": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int,
-                                       _vp, _vp]),
+                                       _vp, _vp, ctypes.c_size_t, _vp]),
     "bitlinear_linear_base3": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32, _vp,
-                                      _vp, _vp, _vp, _vp, _int, _vp]),
+                                      _vp, _vp, _vp, _vp, _int, _vp, ctypes.c_size_t, _vp]),
     "bitlinear_w1_packed_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bitlinear_pack_weights_w1": (_int, [_vp, _i64, _i64, _vp, _vp, ctypes.c_size_t, _vp, _vp,
                                          _vp]),
     "bitlinear_forward_w1": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _int, _vp, _int,
-                                    _vp, _vp]),
+                                    _vp, _vp, ctypes.c_size_t, _vp]),
     "bitlinear_linear_w1": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32, _vp,
-                                   _vp, _vp, _vp, _vp, _int, _vp]),
+                                   _vp, _vp, _vp, _vp, _int, _vp, ctypes.c_size_t, _vp]),
     "bitlinear_dense_bf16_forward": (_int, [_vp, _i64, _i64, _vp, _i64, _vp, _int, _vp]),
     "bitlinear_backward_workspace_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _int, _int]),
     "bitlinear_backward": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _int, _vp,
@@ -293,13 +295,47 @@ def quant_act(X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
     return Xq, beta, rowsum, rms_out
 
 
+SPLIT_AUTO, SPLIT_ALWAYS, SPLIT_NEVER = 0, 1, 2
+
+
+def set_decode_split(mode: int) -> None:
+    """When decode calls with a split workspace split their units:
+    SPLIT_AUTO (default), SPLIT_ALWAYS (tests) or SPLIT_NEVER; process-wide."""
+    _check(lib().bitlinear_set_decode_split(mode), "bitlinear_set_decode_split")
+
+
+def decode_workspace_bytes(d_out: int, T: int) -> int:
+    """Bytes of the split workspace of a decode product (0 unless 1 <= T <= 16)."""
+    return int(lib().bitlinear_decode_workspace_bytes(d_out, T))
+
+
+def decode_workspace(d_out: int, T: int, device=None):
+    """A zero-filled split workspace for decode products with d_out outputs
+    and up to T tokens (None when T > 16).  The kernels leave it zero, so one
+    workspace serves every call on one stream; calls that may overlap on the
+    GPU need their own."""
+    n = decode_workspace_bytes(d_out, min(max(T, 1), 16)) if T <= 16 else 0
+    if n == 0:
+        return None
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def _ws_args(workspace):
+    if workspace is None:
+        return None, 0
+    if workspace.device.type != "cuda" or not workspace.is_contiguous():
+        raise TypeError("workspace must be a contiguous CUDA tensor")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
 def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
             out_dtype=torch.float32, want_acc: bool = False, out: torch.Tensor = None,
-            act_bits: int = 8, acc: torch.Tensor = None):
+            act_bits: int = 8, acc: torch.Tensor = None, workspace: torch.Tensor = None):
     """Y = (X~ W~^T) gamma beta / (Q_b - 1); returns Y (and the int32 acc if
     asked, written to ``acc`` when that tensor is given).  w is a
     PackedTernary, PackedTernaryBase3 or PackedBinary; act_bits (4 or 8, the
-    width the codes were made with) applies to PackedBinary."""
+    width the codes were made with) applies to PackedBinary.  workspace: an
+    optional split workspace (decode_workspace) for T <= 16."""
     _need(Xq, torch.int8, "Xq")
     T = Xq.shape[0]
     dev = Xq.device
@@ -312,14 +348,15 @@ def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
     elif want_acc:
         acc = torch.empty((T, w.d_out), dtype=torch.int32, device=dev)
     fn, name = _entry(w, "bitlinear_forward")
+    wsp, wsn = _ws_args(workspace)
     if isinstance(w, PackedBinary):
         st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq), _ptr(beta),
-                _ptr(rowsum), T, act_bits, _ptr(out), od, _ptr(acc), _stream())
+                _ptr(rowsum), T, act_bits, _ptr(out), od, _ptr(acc), wsp, wsn, _stream())
     else:
         if act_bits != 8:
             raise ValueError("act_bits != 8 needs binary weights")
         st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(Xq), _ptr(beta),
-                _ptr(rowsum), T, _ptr(out), od, _ptr(acc), _stream())
+                _ptr(rowsum), T, _ptr(out), od, _ptr(acc), wsp, wsn, _stream())
     _check(st, name)
     return (out, acc) if want_acc else out
 
@@ -327,7 +364,8 @@ def forward(w, Xq: torch.Tensor, beta: torch.Tensor, rowsum: torch.Tensor,
 def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
            eps: float = 1e-5, norm_eps: float = 1e-5, out_dtype=torch.float32,
            out: torch.Tensor = None, scratch=None, static_weights: bool = False,
-           per_tensor: bool = False, act_bits: int = 8, inv_rms: torch.Tensor = None):
+           per_tensor: bool = False, act_bits: int = 8, inv_rms: torch.Tensor = None,
+           workspace: torch.Tensor = None):
     """The whole BitLinear forward from bf16 X: quantise, then product.
     w is a PackedTernary, PackedTernaryBase3 or PackedBinary; act_bits = 4
     (PackedBinary only) makes it the W1A4 forward.
@@ -337,7 +375,8 @@ def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
     before earlier work has finished).  per_tensor: one activation absmax for
     the whole X instead of one per token.  ``scratch`` = (Xq, beta, rowsum)
     receives the intermediates.  inv_rms: f32 [T] reciprocal RMS to use
-    instead of computing it.
+    instead of computing it.  workspace: an optional split workspace
+    (decode_workspace) for T <= 16.
     """
     _need(X, torch.bfloat16, "X")
     T = X.shape[0]
@@ -357,9 +396,10 @@ def linear(w, X: torch.Tensor, gain: torch.Tensor = None, rmsnorm: bool = True,
     flags = ((RMSNORM if rmsnorm else 0) | (STATIC_WEIGHTS if static_weights else 0)
              | (PER_TENSOR_ABSMAX if per_tensor else 0) | (ACT_4BIT if act_bits == 4 else 0))
     fn, name = _entry(w, "bitlinear_linear")
+    wsp, wsn = _ws_args(workspace)
     st = fn(_ptr(w.packed), _ptr(w.gamma), w.d_out, w.d_in, _ptr(X), T, _ptr(gain), flags, eps,
             norm_eps, _ptr(inv_rms), _ptr(Xq), _ptr(beta), _ptr(rowsum), _ptr(out), od,
-            _stream())
+            wsp, wsn, _stream())
     _check(st, name)
     return out
 
@@ -410,8 +450,11 @@ class LinearPlan:
         else:
             self._fn, self._name = _entry(w, "bitlinear_linear")
             self._pre = (w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in)
+            self._ws = decode_workspace(w.d_out, T, dev)   # the plan's own, as in the C plan
+            wsp, wsn = _ws_args(self._ws)
             self._post = (T, _ptr(gain), flags, eps, norm_eps, None, Xq.data_ptr(),
-                          beta.data_ptr(), rowsum.data_ptr(), out.data_ptr(), od, self._stream)
+                          beta.data_ptr(), rowsum.data_ptr(), out.data_ptr(), od, wsp, wsn,
+                          self._stream)
 
     def __call__(self, X: torch.Tensor) -> torch.Tensor:
         if X.dtype != torch.bfloat16 or tuple(X.shape) != self._shape or not X.is_contiguous():

@@ -19,26 +19,30 @@ bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_o
                              int64_t d_in, const int8_t *Xq, const float *beta,
                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
                              int32_t *acc_out, bool static_weights, int fmt, float qmax,
-                             cudaStream_t stream);
+                             void *ws, cudaStream_t stream);
 bool decode_can_fuse(int64_t T, int64_t d_in);
+size_t decode_workspace_bytes(int64_t d_out, int64_t T);
+int set_decode_split_mode(int mode);
+bool decode_rec_splits(const LaunchRec &rec);
 bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const uint16_t *X, int64_t T,
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
                                      const float *inv_rms_in, int8_t *Xq, float *beta,
                                      int32_t *rowsum, void *Y, int out_dtype,
-                                     bool static_weights, int fmt, float qmax,
+                                     bool static_weights, int fmt, float qmax, void *ws,
                                      cudaStream_t stream);
 bitlinear_status prepare_gemv(const void *packed, const float *gamma, int64_t d_out,
                               int64_t d_in, const int8_t *Xq, const float *beta,
                               const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
                               int32_t *acc_out, bool static_weights, int fmt, float qmax,
-                              LaunchRec *rec);
+                              void *ws, LaunchRec *rec);
 bitlinear_status prepare_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                       int64_t d_in, const uint16_t *X, int64_t T,
                                       const float *gain, bool rmsnorm, float eps,
                                       float norm_eps, const float *inv_rms_in, int8_t *Xq,
                                       float *beta, int32_t *rowsum, void *Y, int out_dtype,
-                                      bool static_weights, int fmt, float qmax, LaunchRec *rec);
+                                      bool static_weights, int fmt, float qmax, void *ws,
+                                      LaunchRec *rec);
 size_t decode_x_offset();
 bitlinear_status prepare_quant_act(const uint16_t *X, int64_t T, int64_t d_in,
                                    const float *norm_gain, uint32_t flags, float eps,
@@ -152,21 +156,33 @@ static bitlinear_status dispatch_forward(const void *packed, const float *gamma,
                                          int64_t d_out, int64_t d_in, const int8_t *Xq,
                                          const float *beta, const int32_t *rowsum, int64_t T,
                                          void *Y, int out_dtype, int32_t *acc_out,
-                                         bool static_weights, int fmt, float qmax,
+                                         bool static_weights, int fmt, float qmax, void *ws,
                                          cudaStream_t stream) {
     if (T <= 16 || fmt != kFmt2Bit)
         return launch_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                           acc_out, static_weights, fmt, qmax, stream);
+                           acc_out, static_weights, fmt, qmax, ws, stream);
     return launch_gemm_tc_pair(static_cast<const uint32_t *>(packed), gamma, d_out, d_in, Xq,
                                beta, rowsum, T, Y, out_dtype, acc_out, stream);
+}
+
+// The optional split workspace of the decode product: large enough for
+// (d_out, T) and 16-byte aligned.
+static bitlinear_status validate_workspace(int64_t d_out, int64_t T, const void *ws,
+                                           size_t ws_bytes) {
+    if (!ws) return BITLINEAR_OK;
+    if (ws_bytes < decode_workspace_bytes(d_out, T)) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned(ws, 16)) return BITLINEAR_ERR_MISALIGNED;
+    return BITLINEAR_OK;
 }
 
 static bitlinear_status forward_common(const void *packed, const float *gamma, int64_t d_out,
                                        int64_t d_in, const int8_t *Xq, const float *beta,
                                        const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                                       int32_t *acc_out, int fmt, float qmax,
-                                       cudaStream_t stream) {
+                                       int32_t *acc_out, int fmt, float qmax, void *ws,
+                                       size_t ws_bytes, cudaStream_t stream) {
     bitlinear_status st = validate_forward(packed, gamma, d_out, d_in, T, Y, out_dtype, acc_out);
+    if (st != BITLINEAR_OK) return st;
+    st = validate_workspace(d_out, T, ws, ws_bytes);
     if (st != BITLINEAR_OK) return st;
     if (fmt != kFmt2Bit && T > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     if (T == 0) return BITLINEAR_OK;
@@ -176,7 +192,7 @@ static bitlinear_status forward_common(const void *packed, const float *gamma, i
     st = check_device();
     if (st != BITLINEAR_OK) return st;
     return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                            acc_out, false, fmt, qmax, stream);
+                            acc_out, false, fmt, qmax, ws, stream);
 }
 
 // Argument checks of bitlinear_linear (and of a plan for it), X excluded:
@@ -207,10 +223,12 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
                                       const float *norm_gain, uint32_t flags, float eps,
                                       float norm_eps, const float *inv_rms_in, int8_t *Xq,
                                       float *beta, int32_t *rowsum, void *Y, int out_dtype,
-                                      int fmt, cudaStream_t stream) {
+                                      int fmt, void *ws, size_t ws_bytes, cudaStream_t stream) {
     bitlinear_status st = validate_linear(packed, gamma, d_out, d_in, T, norm_gain, flags, eps,
                                           norm_eps, inv_rms_in, Xq, beta, rowsum, Y, out_dtype,
                                           fmt);
+    if (st != BITLINEAR_OK) return st;
+    st = validate_workspace(d_out, T, ws, ws_bytes);
     if (st != BITLINEAR_OK || T == 0) return st;
     if (!X) return BITLINEAR_ERR_INVALID_ARG;
     if (!aligned(X, 16)) return BITLINEAR_ERR_MISALIGNED;
@@ -223,7 +241,7 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
     if (!per_tensor && decode_can_fuse(T, d_in))
         return launch_linear_fused(packed, gamma, d_out, d_in, X, T, norm_gain, rmsnorm, eps,
                                    norm_eps, inv_rms_in, Xq, beta, rowsum, Y, out_dtype,
-                                   static_weights, fmt, qmax, stream);
+                                   static_weights, fmt, qmax, ws, stream);
     // Quantiser, then the product as its programmatic dependent: with static
     // weights the product streams them while the codes are still being made.
     st = launch_quant_act(X, T, d_in, norm_gain,
@@ -232,7 +250,7 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
                           eps, norm_eps, inv_rms_in, Xq, beta, rowsum, nullptr, true, stream);
     if (st != BITLINEAR_OK) return st;
     return dispatch_forward(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                            nullptr, static_weights, fmt, qmax, stream);
+                            nullptr, static_weights, fmt, qmax, ws, stream);
 }
 
 }  // namespace bl
@@ -257,11 +275,20 @@ struct bitlinear_plan {
     int32_t *rowsum = nullptr;
     void *Y = nullptr;
     int out_dtype = 0;
+    void *ws = nullptr;       // owned split workspace of the decode product, or null
+    size_t ws_bytes = 0;
 };
 
 using namespace bl;
 
-extern "C" int bitlinear_version(void) { return 2; }
+extern "C" int bitlinear_version(void) { return 3; }
+
+extern "C" int bitlinear_set_decode_split(int mode) { return set_decode_split_mode(mode); }
+
+extern "C" size_t bitlinear_decode_workspace_bytes(int64_t d_out, int64_t T) {
+    if (d_out <= 0 || d_out % 16 || d_out > (1 << 22)) return 0;
+    return decode_workspace_bytes(d_out, T);
+}
 
 extern "C" const char *bitlinear_status_string(int status) {
     switch (status) {
@@ -279,35 +306,41 @@ extern "C" const char *bitlinear_status_string(int status) {
 extern "C" int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
                                  int64_t d_in, const int8_t *Xq, const float *beta,
                                  const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                                 int32_t *acc_out, cudaStream_t stream) {
+                                 int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
     return forward_common(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype, acc_out,
-                          kFmt2Bit, 127.0f, stream);
+                          kFmt2Bit, 127.0f, workspace, workspace_bytes, stream);
 }
 
 extern "C" int bitlinear_forward_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
                                        int64_t d_in, const int8_t *Xq, const float *beta,
                                        const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
-                                       int32_t *acc_out, cudaStream_t stream) {
+                                       int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                                       cudaStream_t stream) {
     return forward_common(packed3, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                          acc_out, kFmtBase3, 127.0f, stream);
+                          acc_out, kFmtBase3, 127.0f, workspace, workspace_bytes, stream);
 }
 
 extern "C" int bitlinear_forward_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
                                     int64_t d_in, const int8_t *Xq, const float *beta,
                                     const int32_t *rowsum, int64_t T, int act_bits, void *Y,
-                                    int out_dtype, int32_t *acc_out, cudaStream_t stream) {
+                                    int out_dtype, int32_t *acc_out, void *workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
     if (act_bits != 4 && act_bits != 8) return BITLINEAR_ERR_INVALID_ARG;
     return forward_common(packed1, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
-                          acc_out, kFmt1Bit, act_bits == 4 ? 7.0f : 127.0f, stream);
+                          acc_out, kFmt1Bit, act_bits == 4 ? 7.0f : 127.0f, workspace,
+                          workspace_bytes, stream);
 }
 
 extern "C" int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
                                 int64_t d_in, const uint16_t *X, int64_t T,
                                 const float *norm_gain, uint32_t flags, float eps, float norm_eps,
                                 const float *inv_rms_in, int8_t *Xq, float *beta,
-                                int32_t *rowsum, void *Y, int out_dtype, cudaStream_t stream) {
+                                int32_t *rowsum, void *Y, int out_dtype, void *workspace,
+                                size_t workspace_bytes, cudaStream_t stream) {
     return linear_common(packed, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps,
-                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmt2Bit, stream);
+                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmt2Bit, workspace,
+                         workspace_bytes, stream);
 }
 
 extern "C" int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma, int64_t d_out,
@@ -315,9 +348,11 @@ extern "C" int bitlinear_linear_base3(const uint8_t *packed3, const float *gamma
                                       const float *norm_gain, uint32_t flags, float eps,
                                       float norm_eps, const float *inv_rms_in, int8_t *Xq,
                                       float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                      void *workspace, size_t workspace_bytes,
                                       cudaStream_t stream) {
     return linear_common(packed3, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps,
-                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmtBase3, stream);
+                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmtBase3, workspace,
+                         workspace_bytes, stream);
 }
 
 extern "C" int bitlinear_linear_w1(const uint32_t *packed1, const float *gamma, int64_t d_out,
@@ -325,9 +360,11 @@ extern "C" int bitlinear_linear_w1(const uint32_t *packed1, const float *gamma, 
                                    const float *norm_gain, uint32_t flags, float eps,
                                    float norm_eps, const float *inv_rms_in, int8_t *Xq,
                                    float *beta, int32_t *rowsum, void *Y, int out_dtype,
+                                   void *workspace, size_t workspace_bytes,
                                    cudaStream_t stream) {
     return linear_common(packed1, gamma, d_out, d_in, X, T, norm_gain, flags, eps, norm_eps,
-                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmt1Bit, stream);
+                         inv_rms_in, Xq, beta, rowsum, Y, out_dtype, kFmt1Bit, workspace,
+                         workspace_bytes, stream);
 }
 
 extern "C" int bitlinear_dense_bf16_forward(const uint16_t *W, int64_t d_out, int64_t d_in,
@@ -425,6 +462,21 @@ extern "C" int bitlinear_linear_plan_create(const uint32_t *packed, const float 
     const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
     const bool rmsnorm = (flags & BITLINEAR_RMSNORM) != 0;
     const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
+    // A decode product gets its own zero-filled split workspace (kept only
+    // if the prepared launch uses it).
+    if (T >= 1 && T <= 16) {
+        p->ws_bytes = decode_workspace_bytes(d_out, T);
+        if (cudaMalloc(&p->ws, p->ws_bytes) != cudaSuccess) {
+            cudaGetLastError();
+            delete p;
+            return BITLINEAR_ERR_CUDA;
+        }
+        if (cudaMemset(p->ws, 0, p->ws_bytes) != cudaSuccess) {
+            cudaFree(p->ws);
+            delete p;
+            return BITLINEAR_ERR_CUDA;
+        }
+    }
     if (T == 0) {
         p->steps = 0;
     } else if (per_tensor) {
@@ -432,7 +484,7 @@ extern "C" int bitlinear_linear_plan_create(const uint32_t *packed, const float 
     } else if (decode_can_fuse(T, d_in)) {
         st = prepare_linear_fused(packed, gamma, d_out, d_in, nullptr, T, norm_gain, rmsnorm, eps,
                                   norm_eps, nullptr, Xq, beta, rowsum, Y, out_dtype,
-                                  static_weights, kFmt2Bit, 127.0f, &p->rec[0]);
+                                  static_weights, kFmt2Bit, 127.0f, p->ws, &p->rec[0]);
         p->x_field = decode_x_offset();
         p->steps = 1;
     } else {
@@ -442,10 +494,18 @@ extern "C" int bitlinear_linear_plan_create(const uint32_t *packed, const float 
         if (st == BITLINEAR_OK)
             st = T <= 16 ? prepare_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y,
                                         out_dtype, nullptr, static_weights, kFmt2Bit, 127.0f,
-                                        &p->rec[1])
+                                        p->ws, &p->rec[1])
                          : prepare_gemm_tc_pair(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y,
                                                 out_dtype, nullptr, &p->rec[1]);
         p->steps = 2;
+    }
+    const bool splits = (p->steps == 1 && decode_rec_splits(p->rec[0])) ||
+                        (p->steps == 2 && T <= 16 && decode_rec_splits(p->rec[1])) ||
+                        p->steps == -1;
+    if (p->ws && (st != BITLINEAR_OK || !splits)) {
+        cudaFree(p->ws);
+        p->ws = nullptr;
+        p->ws_bytes = 0;
     }
     if (st != BITLINEAR_OK) {
         delete p;
@@ -467,7 +527,7 @@ extern "C" int bitlinear_linear_plan_run(const bitlinear_plan *plan, const uint1
         return linear_common(plan->packed, plan->gamma, plan->d_out, plan->d_in, X, plan->T,
                              plan->norm_gain, plan->flags, plan->eps, plan->norm_eps, nullptr,
                              plan->Xq, plan->beta, plan->rowsum, plan->Y, plan->out_dtype,
-                             kFmt2Bit, stream);
+                             kFmt2Bit, plan->ws, plan->ws_bytes, stream);
     LaunchRec first = plan->rec[0];
     first.patch_ptr(0, plan->x_field, X);
     if (first.launch(stream) != cudaSuccess) return BITLINEAR_ERR_CUDA;
@@ -475,4 +535,13 @@ extern "C" int bitlinear_linear_plan_run(const bitlinear_plan *plan, const uint1
     return BITLINEAR_OK;
 }
 
-extern "C" void bitlinear_plan_destroy(bitlinear_plan *plan) { delete plan; }
+extern "C" void bitlinear_plan_destroy(bitlinear_plan *plan) {
+    if (plan && plan->ws) {
+        int prev = -1;
+        cudaGetDevice(&prev);
+        cudaSetDevice(plan->device);
+        cudaFree(plan->ws);
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+    delete plan;
+}

@@ -37,6 +37,14 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+// A GPU-scope relaxed 64-bit load (bypasses the non-coherent L1): a split
+// workspace word other CTAs update with atomics.
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // Bounded wait that also gives up once another role has aborted.
 __device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, const DeviceCtx &ctx,
                                          volatile int *abort_flag) {

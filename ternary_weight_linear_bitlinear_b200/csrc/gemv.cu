@@ -68,9 +68,31 @@
 // is sum c x, and W~ X~ = 2 sum c x - S.  The rescale divides by Q_b - 1 of
 // the activation codes (127, or 7 for 4-bit codes).
 //
+// Balanced split.  Without a workspace a CTA owns a run of whole groups, so
+// when the groups do not divide evenly over the resident CTAs (896 groups on
+// 296 CTAs: three or four each) the kernel ends with the CTAs that own one
+// more.  With a split workspace the (group, k-tile) units, group-major, are
+// cut into equal contiguous shares, one per resident CTA; a CTA's first and
+// last groups may then be shared with its neighbours ("segments" of
+// k-tiles).  A shared group's int32 partial sums meet in the workspace:
+// integer addition is exact, so the result does not depend on the split.
+// Each output has one 64-bit workspace word that describes itself: the sum of
+// the k-tile counts of the segments added so far (bits 45..63), their number
+// (bits 36..44) and the sum of their partial sums each biased by 2^25 (bits
+// 0..35; |partial| < 2 * 128 * 65536 < 2^25).  A segment adds
+// (k << 45) + (1 << 36) + (v + 2^25) with one atomic; whoever completes the
+// count to the group's k-tiles writes the output and zeroes the word.  No
+// counter, no fence, no waiting: a word is never seen half-updated.  A CTA's
+// first segment (shared with its left neighbour, which reaches that group
+// last) adds early and checks the returned word only at the CTA's end; its
+// last segment loads its words when it starts (the right neighbour has
+// usually added its part by then) and finalises from them without a round
+// trip, falling back to the atomic when they are not complete.
+
 // Every mbarrier wait is bounded; on expiry the CTA stops consuming, the
 // producer waits (bounded) for the copies it issued, and the error word is
 // set.
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -116,7 +138,27 @@ struct DecodeArgs {
     void *Y;
     int32_t *acc_out;
     int static_weights;
+    // Split workspace (see "Balanced split" above), or null: then every CTA
+    // owns whole groups.  One 64-bit word per output, T * 16R per group; zero
+    // before the launch, zero after it.
+    unsigned long long *split_ws;
 };
+
+// The split workspace word's fields.
+constexpr int kSplitKShift = 45;
+constexpr int kSplitPartsShift = 36;
+constexpr unsigned long long kSplitSumMask = (1ull << kSplitPartsShift) - 1;
+constexpr long long kSplitBias = 1ll << 25;
+
+__device__ __forceinline__ unsigned long long split_word(int k, int v) {
+    return ((unsigned long long)k << kSplitKShift) + (1ull << kSplitPartsShift) +
+           (unsigned long long)(v + kSplitBias);
+}
+__device__ __forceinline__ int split_k(unsigned long long w) { return (int)(w >> kSplitKShift); }
+__device__ __forceinline__ int split_sum(unsigned long long w) {
+    const long long parts = (long long)((w >> kSplitPartsShift) & 511u);
+    return (int)((long long)(w & kSplitSumMask) - parts * kSplitBias);
+}
 
 struct DecodePlan {
     int ks;            // k-blocks per slab
@@ -159,8 +201,15 @@ __device__ __forceinline__ void consumer_barrier() {
     asm volatile("bar.sync 2, %0;" ::"n"(kDecWarps * 32) : "memory");
 }
 
-template <int NT, int R, bool FUSED, bool OUT_BF16, int FMT>
-__global__ void __launch_bounds__(kDecThreads)
+// Resident CTAs per SM the register budget must allow: the one-tile-per-group
+// variants run many small CTAs per SM, and a programmatic dependent's CTAs
+// only overlap this grid's tail when both fit on the SM together.
+template <int NT, int R, int FMT>
+constexpr int dec_min_blocks() { return NT == 1 && R == 1 && FMT != kFmt1Bit ? 6 : 1; }
+
+// SPLIT: the balanced split (a.split_ws non-null); otherwise whole groups.
+template <int NT, int R, bool FUSED, bool OUT_BF16, int FMT, bool SPLIT>
+__global__ void __launch_bounds__(kDecThreads, dec_min_blocks<NT, R, FMT>())
 decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx ctx) {
     constexpr int TMAX = NT * 8;
     constexpr bool B3 = FMT == kFmtBase3;
@@ -185,11 +234,37 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     const int KB = a.kb_total, K = a.d_in, T = a.T;
     const int n_rt = a.d_out >> 4;
     const int n_groups = (n_rt + R - 1) / R;
-    const int grp0 = (int)(((long long)n_groups * blockIdx.x) / gridDim.x);
-    const int ngrp = (int)(((long long)n_groups * (blockIdx.x + 1)) / gridDim.x) - grp0;
-    const int ks = plan.ks, nslab = plan.nslab, stages = plan.stages;
+    const int ks = plan.ks, stages = plan.stages;
     const int stage_bytes = plan.stage_bytes;
-    const int units = ngrp * nslab;
+    // This CTA's share of the (group, k-tile) units, group-major: a run of
+    // whole groups, or with a split workspace an equal share of the units
+    // (the first U mod P CTAs one unit more).  32-bit: U < 2^27.
+    const int P = gridDim.x, c = blockIdx.x;
+    int u0, u1;
+    if (SPLIT) {
+        const int U = n_groups * KB, q = U / P, rem = U - q * P;
+        u0 = q * c + (c < rem ? c : rem);
+        u1 = u0 + q + (c < rem ? 1 : 0);
+    } else {
+        const int q = n_groups / P, rem = n_groups - q * P;
+        const int g0 = q * c + (c < rem ? c : rem);
+        u0 = g0 * KB;
+        u1 = (g0 + q + (c < rem ? 1 : 0)) * KB;
+    }
+    const int g_first = u0 / KB;
+    const int nseg = u1 > u0 ? (u1 - 1) / KB - g_first + 1 : 0;
+    // Segment s: k-tiles [seg_kb0(s), seg_kb1(s)) of group g_first + s.
+    auto seg_kb0 = [&](int sg) {
+        const int b = u0 - (g_first + sg) * KB;
+        return b > 0 ? b : 0;
+    };
+    auto seg_kb1 = [&](int sg) {
+        const int e = u1 - (g_first + sg) * KB;
+        return e < KB ? e : KB;
+    };
+    // Ring units: slabs of up to ks k-tiles of one segment, in order.
+    int units = 0;
+    for (int sg = 0; sg < nseg; ++sg) units += (seg_kb1(sg) - seg_kb0(sg) + ks - 1) / ks;
     // Dynamic shared memory: [bf16 X (fused)] [codes (fused)] [stages].
     const int xb_bytes = FUSED ? ((T * K * 2 + 127) & ~127) : 0;
     uint16_t *xb = reinterpret_cast<uint16_t *>(dsm);
@@ -212,41 +287,52 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     if (warp == kDecWarps) {
         // ------------------------------------------------------ producer ---
         if (lane == 0) {
-            // Unit (gi, sl): group grp0 + gi, slab sl; units run gi-major.
-            auto slab_kb = [&](int sl) { return KB - sl * ks < ks ? KB - sl * ks : ks; };
-            // Activation columns of a slab (the last base-3 tile may overhang d_in).
-            auto slab_cols = [&](int sl) {
-                const int c = slab_kb(sl) * kTileCols, left = K - sl * ks * kTileCols;
+            // Unit (sg, kb): k-tiles kb .. kb + nkb - 1 of segment sg.
+            auto unit_kb = [&](int sg, int kb) { return seg_kb1(sg) - kb < ks ? seg_kb1(sg) - kb : ks; };
+            auto next_unit = [&](int &sg, int &kb) {
+                kb += ks;
+                if (kb >= seg_kb1(sg)) {
+                    ++sg;
+                    kb = sg < nseg ? seg_kb0(sg) : 0;
+                }
+            };
+            // Activation columns of a unit (the last base-3 tile may overhang d_in).
+            auto unit_cols = [&](int sg, int kb) {
+                const int c = unit_kb(sg, kb) * kTileCols, left = K - kb * kTileCols;
                 return c < left ? c : left;
             };
-            auto issue_w = [&](int gi, int sl, int st) {
+            auto issue_w = [&](int sg, int kb, int st) {
                 const uint32_t bar = smem_u32(&full_bar[st]);
-                const int rt = (grp0 + gi) * R;
-                const int nkb = slab_kb(sl);
+                const int rt = (g_first + sg) * R;
+                const int nkb = unit_kb(sg, kb);
                 int nrow = 0;
                 #pragma unroll
                 for (int r = 0; r < R; ++r) nrow += rt + r < n_rt ? 1 : 0;
-                const uint32_t xbytes = FUSED ? 0u : (uint32_t)(T * slab_cols(sl));
+                const uint32_t xbytes = FUSED ? 0u : (uint32_t)(T * unit_cols(sg, kb));
                 mbar_arrive_expect_tx(bar, (uint32_t)(nrow * nkb * kTileBytes) + xbytes);
                 for (int r = 0; r < nrow; ++r)
                     bulk_g2s(ring_s + st * stage_bytes + r * ks * kTileBytes,
-                             a.packed + ((size_t)(rt + r) * KB + (size_t)sl * ks) * kTileBytes,
+                             a.packed + ((size_t)(rt + r) * KB + (size_t)kb) * kTileBytes,
                              (uint32_t)(nkb * kTileBytes), bar);
             };
-            auto issue_x = [&](int sl, int st) {
+            auto issue_x = [&](int sg, int kb, int st) {
                 if (FUSED) return;
                 const uint32_t bar = smem_u32(&full_bar[st]);
                 for (int t = 0; t < T; ++t)
                     bulk_g2s(ring_s + st * stage_bytes + R * ks * kTileBytes + t * ks * kTileCols,
-                             a.Xq + (size_t)t * K + (size_t)sl * ks * kTileCols,
-                             (uint32_t)slab_cols(sl), bar);
+                             a.Xq + (size_t)t * K + (size_t)kb * kTileCols,
+                             (uint32_t)unit_cols(sg, kb), bar);
             };
-            const int first = units < stages ? units : stages;
+            // With static weights the first unit's weights are requested
+            // before the dependency wait.  Only the first: a CTA's whole ring
+            // requested at once (by every CTA) arrives later as a whole, and
+            // the copies issued after the wait (activations) queue behind it.
+            const int first = units < 1 ? units : 1;
             if (a.static_weights) {
-                int gi = 0, sl = 0;
+                int sg = 0, kb = nseg > 0 ? seg_kb0(0) : 0;
                 for (int u = 0; u < first; ++u) {
-                    issue_w(gi, sl, u);
-                    if (++sl == nslab) { sl = 0; ++gi; }
+                    issue_w(sg, kb, u);
+                    next_unit(sg, kb);
                 }
             }
             pdl_wait_primary();
@@ -257,7 +343,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 mbar_arrive_expect_tx(xbar, (uint32_t)(T * K * 2));
                 bulk_g2s(smem_u32(xb), a.X, (uint32_t)(T * K * 2), xbar);
             }
-            int gi = 0, sl = 0, st = 0, round = 0, issued = 0;
+            int sg = 0, kb = nseg > 0 ? seg_kb0(0) : 0, st = 0, round = 0, issued = 0;
             for (int u = 0; u < units; ++u) {
                 if (round > 0) {
                     // Stage st was last used by unit u - stages: wait for its
@@ -265,13 +351,13 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                     if (!dec_wait(smem_u32(&empty_bar[st]), (uint32_t)(round - 1) & 1u, ctx,
                                   abort_flag))
                         break;
-                    issue_w(gi, sl, st);
-                } else if (!a.static_weights) {
-                    issue_w(gi, sl, st);
+                    issue_w(sg, kb, st);
+                } else if (!a.static_weights || u >= first) {
+                    issue_w(sg, kb, st);
                 }
-                issue_x(sl, st);
+                issue_x(sg, kb, st);
                 ++issued;
-                if (++sl == nslab) { sl = 0; ++gi; }
+                next_unit(sg, kb);
                 if (++st == stages) { st = 0; ++round; }
             }
             // Every copy issued must land before the CTA may exit.
@@ -295,6 +381,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
     pdl_launch_dependents();
     if (!a.static_weights) gamma = __ldg(a.gamma);
     const int g = lane >> 2, q = lane & 3;
+    float in_beta = 0.0f;   // product only: beta[t] and rowsum[t] of token t = threadIdx.x
+    int in_rowsum = 0;
     bool fast_quant = false;   // fused, no gain: codes made per warp, rowsum in the epilogue
     if constexpr (FUSED) {
         bool xok = dec_wait(smem_u32(&x_bar), 0, ctx, abort_flag);
@@ -359,19 +447,88 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
             }
             consumer_barrier();
         }
-    } else {
-        if (threadIdx.x < T) {
-            const int t = threadIdx.x;
-            s_yscale[t] = __fdiv_rn(__fmul_rn(gamma, a.beta[t]), a.qmax);
-            s_rowsum[t] = a.rowsum[t];
+    } else if (threadIdx.x < T) {
+        // Needed first by the first epilogue: loaded now, stored to shared
+        // memory after the first segment's MMAs, so that the load's latency
+        // (behind this CTA's weight stream) overlaps them.
+        in_beta = a.beta[threadIdx.x];
+        in_rowsum = a.rowsum[threadIdx.x];
+    }
+
+    // Fused: the CTAs hand back the intermediates once every warp's codes
+    // are complete.  Every CTA holds the same codes, so they are written in
+    // slices spread over the grid, and no single CTA lengthens it.
+    auto hand_back = [&]() {
+        if (blockIdx.x == 0 && threadIdx.x < T && a.rowsum_out) {
+            int sum = 0;
+            #pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) sum += qs.sum[w][threadIdx.x];
+            a.rowsum_out[threadIdx.x] = sum;
         }
+        if (a.Xq_out) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(xs);
+            uint4 *dst = reinterpret_cast<uint4 *>(a.Xq_out);
+            const int nv = (T * K) >> 4;
+            for (int v = blockIdx.x * kDecWarps * 32 + threadIdx.x; v < nv;
+                 v += gridDim.x * kDecWarps * 32)
+                dst[v] = src[v];
+        }
+    };
+    if (FUSED && fast_quant && nseg == 0) {   // a split share with no units
         consumer_barrier();
+        hand_back();
     }
 
     bool ok = true;
     int st = 0;
     uint32_t fph = 0;
-    for (int gi = 0; gi < ngrp; ++gi) {
+    constexpr int per_t = 16 * R;
+    // Outputs of a segment per consumer thread: i = threadIdx.x + 128 j.
+    constexpr int kEPT = (TMAX * per_t + kDecWarps * 32 - 1) / (kDecWarps * 32);
+    // Output (token t, row tile r, row) of group grp from sum c x over all of K.
+    auto emit = [&](int grp, int t, int r, int row, int v) {
+        int rsum;
+        if (FUSED && fast_quant) {
+            rsum = 0;
+            #pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) rsum += qs.sum[w][t];
+        } else {
+            rsum = s_rowsum[t];
+        }
+        // Offset codes: W~ = c - 1 (2-bit, base 3) or 2c - 1 (1 bit).
+        const int accv = W1 ? 2 * v - rsum : v - rsum;
+        const int o = (grp * R + r) * 16 + row;
+        const size_t yi = (size_t)t * a.d_out + o;
+        if (a.acc_out) a.acc_out[yi] = accv;
+        const float y = __fmul_rn((float)accv, s_yscale[t]);
+        if (OUT_BF16)
+            reinterpret_cast<__nv_bfloat16 *>(a.Y)[yi] = __float2bfloat16_rn(y);
+        else
+            reinterpret_cast<float *>(a.Y)[yi] = y;
+    };
+    // Split: the words of the last segment and of a shared first segment,
+    // loaded when the last segment starts.
+    const bool first_shared = SPLIT && nseg > 1 && seg_kb0(0) > 0;
+    unsigned long long pre_w[SPLIT ? kEPT : 1], first_w[SPLIT ? kEPT : 1];
+    for (int sg = 0; sg < nseg; ++sg) {
+        const int grp = g_first + sg;
+        const int kb0 = seg_kb0(sg), kb1 = seg_kb1(sg);
+        const bool part = SPLIT && (kb0 > 0 || kb1 < KB);   // shared with a neighbour
+        const bool last_part = part && sg == nseg - 1;
+        const int my_k = kb1 - kb0;
+        unsigned long long *gws = SPLIT ? a.split_ws + (size_t)grp * T * per_t : nullptr;
+        if constexpr (SPLIT) {
+            if (sg == nseg - 1) {
+                unsigned long long *gws0 = a.split_ws + (size_t)g_first * T * per_t;
+                #pragma unroll
+                for (int j = 0; j < kEPT; ++j) {
+                    const int idx = threadIdx.x + kDecWarps * 32 * j;
+                    const bool in = idx < T * per_t;
+                    pre_w[j] = last_part && in ? ld_relaxed_gpu_u64(gws + idx) : 0ull;
+                    first_w[j] = first_shared && in ? ld_relaxed_gpu_u64(gws0 + idx) : 0ull;
+                }
+            }
+        }
         int acc[R][NT][kSlots][4];
         #pragma unroll
         for (int r = 0; r < R; ++r)
@@ -382,15 +539,17 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                     #pragma unroll
                     for (int e = 0; e < 4; ++e) acc[r][nt][s][e] = 0;
 
-        for (int sl = 0; sl < nslab && ok; ++sl) {
+        for (int kbs = kb0; kbs < kb1 && ok; kbs += ks) {
             ok = dec_wait(smem_u32(&full_bar[st]), fph, ctx, abort_flag);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             const uint8_t *stage = ring + st * stage_bytes;
-            const int nkb = KB - sl * ks < ks ? KB - sl * ks : ks;
+            const int nkb = kb1 - kbs < ks ? kb1 - kbs : ks;
+            // Warp w multiplies the k-tiles kb = w (mod 4) (those it quantised).
+            const int kk0 = (warp - kbs) & (kDecWarps - 1);
             if constexpr (B3) {
-                for (int kk = warp; kk < nkb; kk += kDecWarps) {
+                for (int kk = kk0; kk < nkb; kk += kDecWarps) {
                     // This lane's 40 columns of the tile: 40q .. 40q+39.
-                    const int col0 = (sl * ks + kk) * 160 + 40 * q;
+                    const int col0 = (kbs + kk) * 160 + 40 * q;
                     uint32_t dg[R][10], dh[R][10];   // rows g and g + 8
                     #pragma unroll
                     for (int r = 0; r < R; ++r) {
@@ -426,9 +585,9 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                     }
                 }
             } else if constexpr (W1) {
-                for (int kk = warp; kk < nkb; kk += kDecWarps) {
+                for (int kk = kk0; kk < nkb; kk += kDecWarps) {
                     // This lane's 128 columns of the tile: 128q .. 128q+127.
-                    const int col0 = (sl * ks + kk) * 512 + 128 * q;
+                    const int col0 = (kbs + kk) * 512 + 128 * q;
                     uint32_t w0[R][4], w1[R][4];   // words 4q..4q+3 of rows g and g + 8
                     #pragma unroll
                     for (int r = 0; r < R; ++r) {
@@ -480,7 +639,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                     }
                 }
             } else
-            for (int kk = warp; kk < nkb; kk += kDecWarps) {
+            for (int kk = kk0; kk < nkb; kk += kDecWarps) {
                 uint32_t w0[R][4], w1[R][4];
                 #pragma unroll
                 for (int r = 0; r < R; ++r) {
@@ -496,7 +655,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                     const int t = nt * 8 + g;
                     const uint8_t *xsrc =
                         FUSED ? reinterpret_cast<const uint8_t *>(xs) + (size_t)t * K +
-                                    (size_t)(sl * ks + kk) * 256 + 64 * q
+                                    (size_t)(kbs + kk) * 256 + 64 * q
                               : stage + R * ks * 1024 + (t * ks + kk) * 256 + 64 * q;
                     #pragma unroll
                     for (int v = 0; v < 4; ++v) {
@@ -552,36 +711,24 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 }
                 red[warp][r][nt][lane] = make_int4(c[0], c[1], c[2], c[3]);
             }
-        consumer_barrier();
-        if (FUSED && fast_quant && gi == 0) {
-            // Every warp's codes are complete: the CTAs hand back the
-            // intermediates.  Every CTA holds the same codes, so they are
-            // written in slices spread over the grid, and no single CTA
-            // lengthens it.
-            if (blockIdx.x == 0 && threadIdx.x < T && a.rowsum_out) {
-                int sum = 0;
-                #pragma unroll
-                for (int w = 0; w < kDecWarps; ++w) sum += qs.sum[w][threadIdx.x];
-                a.rowsum_out[threadIdx.x] = sum;
-            }
-            if (a.Xq_out) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(xs);
-                uint4 *dst = reinterpret_cast<uint4 *>(a.Xq_out);
-                const int nv = (T * K) >> 4;
-                for (int v = blockIdx.x * kDecWarps * 32 + threadIdx.x; v < nv;
-                     v += gridDim.x * kDecWarps * 32)
-                    dst[v] = src[v];
-            }
+        if (!FUSED && sg == 0 && threadIdx.x < T) {
+            s_yscale[threadIdx.x] = __fdiv_rn(__fmul_rn(gamma, in_beta), a.qmax);
+            s_rowsum[threadIdx.x] = in_rowsum;
         }
+        consumer_barrier();
+        // Every warp's codes are complete (fused, after a barrier).
+        if (FUSED && fast_quant && sg == 0) hand_back();
 
-        // Epilogue of this group: output i -> (token t, row tile r, row), rows
-        // fastest, so consecutive threads store consecutive outputs.
-        const int rt0 = (grp0 + gi) * R;
-        const int per_t = 16 * R;
-        for (int idx = threadIdx.x; idx < T * per_t; idx += kDecWarps * 32) {
+        // Epilogue of this segment: output i -> (token t, row tile r, row),
+        // rows fastest, so consecutive threads store consecutive outputs.
+        // v is sum c x over this segment's k-tiles.
+        #pragma unroll
+        for (int j = 0; j < kEPT; ++j) {
+            const int idx = threadIdx.x + kDecWarps * 32 * j;
+            if (idx >= T * per_t) break;
             const int t = idx / per_t, rem = idx - t * per_t;
             const int r = rem >> 4, row = rem & 15;
-            if (rt0 + r >= n_rt) continue;
+            if (grp * R + r >= n_rt) continue;
             const int gg = row & 7, half = row >> 3;
             const int nt = t >> 3, tt = t & 7;
             const int src_lane = gg * 4 + (tt >> 1);
@@ -592,26 +739,45 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
                 const int *e = reinterpret_cast<const int *>(&red[w][r][nt][src_lane]);
                 v += e[reg];
             }
-            int rsum;
-            if (FUSED && fast_quant) {
-                rsum = 0;
-                #pragma unroll
-                for (int w = 0; w < kDecWarps; ++w) rsum += qs.sum[w][t];
-            } else {
-                rsum = s_rowsum[t];
+            if (!part) {
+                emit(grp, t, r, row, v);
+            } else if constexpr (SPLIT) {
+                if (last_part) {
+                    unsigned long long wd = pre_w[j];
+                    if (split_k(wd) + my_k != KB)
+                        wd = atomicAdd(gws + idx, split_word(my_k, v));   // not all in yet
+                    if (split_k(wd) + my_k == KB) {
+                        emit(grp, t, r, row, v + split_sum(wd));
+                        gws[idx] = 0ull;
+                    }
+                } else {
+                    atomicAdd(gws + idx, split_word(my_k, v));   // checked at the end
+                }
             }
-            // Offset codes: W~ = c - 1 (2-bit, base 3) or 2c - 1 (1 bit).
-            const int accv = W1 ? 2 * v - rsum : v - rsum;
-            const int o = (rt0 + r) * 16 + row;
-            const size_t yi = (size_t)t * a.d_out + o;
-            if (a.acc_out) a.acc_out[yi] = accv;
-            const float y = __fmul_rn((float)accv, s_yscale[t]);
-            if (OUT_BF16)
-                reinterpret_cast<__nv_bfloat16 *>(a.Y)[yi] = __float2bfloat16_rn(y);
-            else
-                reinterpret_cast<float *>(a.Y)[yi] = y;
         }
         consumer_barrier();
+    }
+    if constexpr (SPLIT) {
+        // A shared first segment (not also the last) added its part with no
+        // look at the result; its words, loaded after that addition, show
+        // whether it completed them (then this CTA writes those outputs: a
+        // neighbour whose own addition completed them first may write the
+        // same values too, which is harmless).
+        if (first_shared) {
+            unsigned long long *gws0 = a.split_ws + (size_t)g_first * T * per_t;
+            #pragma unroll
+            for (int j = 0; j < kEPT; ++j) {
+                const int idx = threadIdx.x + kDecWarps * 32 * j;
+                if (idx >= T * per_t) break;
+                const int t = idx / per_t, rem = idx - t * per_t;
+                const int r = rem >> 4, row = rem & 15;
+                if (g_first * R + r >= n_rt) continue;
+                if (split_k(first_w[j]) == KB) {
+                    emit(g_first, t, r, row, split_sum(first_w[j]));
+                    gws0[idx] = 0ull;
+                }
+            }
+        }
     }
 }
 
@@ -623,7 +789,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
 #define BL_DEC_WIDE_ROW_TILES (148 * 8) // from this many 16-row tiles on, 2 tiles per group
 #endif
 #ifndef BL_DEC_STAGE_BYTES
-#define BL_DEC_STAGE_BYTES 32768        // target bytes per pipeline stage
+#define BL_DEC_STAGE_BYTES 49152        // target bytes per pipeline stage
 #endif
 #ifndef BL_DEC_RING_BYTES
 #define BL_DEC_RING_BYTES 98304         // bytes of all stages of a CTA
@@ -635,10 +801,23 @@ decode_kernel(const __grid_constant__ DecodeArgs a, DecodePlan plan, DeviceCtx c
 #define BL_DEC_MIN_GROUPS 1             // at least this many groups per CTA
 #endif
 constexpr int kFusedMaxCodeBytes = BL_FUSED_MAX_CODE_BYTES;
+constexpr int kSmemPerSm = 228 * 1024;      // shared memory of an SM
+constexpr int kDecSmemReserve = 8 * 1024;   // per CTA: static shared memory + the 1 KiB reserve
+
+// When a call that has a split workspace splits its units (see "Balanced
+// split"): BITLINEAR_SPLIT_AUTO, _ALWAYS or _NEVER.
+static std::atomic<int> g_split_mode{BITLINEAR_SPLIT_AUTO};
+
+int set_decode_split_mode(int mode) {
+    if (mode != BITLINEAR_SPLIT_AUTO && mode != BITLINEAR_SPLIT_ALWAYS &&
+        mode != BITLINEAR_SPLIT_NEVER)
+        return BITLINEAR_ERR_INVALID_ARG;
+    g_split_mode.store(mode);
+    return BITLINEAR_OK;
+}
 
 template <int NT, int R, bool FUSED, bool OUT_BF16, int FMT>
-static cudaError_t prepare_decode_t(const DecodeArgs &args, const DeviceCtx &ctx,
-                                    LaunchRec *rec) {
+static cudaError_t prepare_decode_t(DecodeArgs args, const DeviceCtx &ctx, LaunchRec *rec) {
     constexpr int kTileBytes = FMT == kFmtBase3 ? 512 : 1024;
     constexpr int kTileCols = FMT == kFmtBase3 ? 160 : (FMT == kFmt1Bit ? 512 : 256);
     const int n_rt = args.d_out / 16;
@@ -655,9 +834,18 @@ static cudaError_t prepare_decode_t(const DecodeArgs &args, const DeviceCtx &ctx
     // multiplies exactly the k-blocks kb = w (mod 4) (those it quantised).
     if (plan.ks < KB) plan.ks = plan.ks >= kDecWarps ? plan.ks - plan.ks % kDecWarps : kDecWarps;
     if (plan.ks > KB) plan.ks = KB;
+    // Keep two CTAs per SM (eight MMA warps) where two stages of at least
+    // four k-tiles still fit beside the activations: one CTA of four MMA warps
+    // cannot keep up with the weight stream.
+    int ring_bytes = BL_DEC_RING_BYTES;
+    const int two_per_sm = kSmemPerSm / 2 - kDecSmemReserve - xb_bytes - plan.xs_bytes;
+    if (two_per_sm < ring_bytes && two_per_sm >= 2 * kDecWarps * per_kb) {
+        ring_bytes = two_per_sm;
+        while (plan.ks > kDecWarps && 2 * plan.ks * per_kb > ring_bytes) plan.ks -= kDecWarps;
+    }
     plan.nslab = (KB + plan.ks - 1) / plan.ks;
     plan.stage_bytes = plan.ks * per_kb;
-    plan.stages = BL_DEC_RING_BYTES / plan.stage_bytes;
+    plan.stages = ring_bytes / plan.stage_bytes;
     if (plan.stages > kDecMaxStages) plan.stages = kDecMaxStages;
     // No deeper than the units a CTA can get when up to 8 CTAs fit per SM.
     const int min_units = ((n_groups + 148 * 8 - 1) / (148 * 8)) * plan.nslab;
@@ -665,23 +853,50 @@ static cudaError_t prepare_decode_t(const DecodeArgs &args, const DeviceCtx &ctx
     if (plan.stages < 2) plan.stages = 2;
     const size_t smem =
         (size_t)xb_bytes + (size_t)plan.xs_bytes + (size_t)plan.stages * plan.stage_bytes;
-    auto kern = decode_kernel<NT, R, FUSED, OUT_BF16, FMT>;
-    cudaError_t e = ensure_dynamic_smem((const void *)kern, smem);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148, per_sm = 1;
+    int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem) !=
-            cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    int max_ctas = sms * per_sm / BL_DEC_CTA_FRACTION;
-    const int by_groups = (n_groups + BL_DEC_MIN_GROUPS - 1) / BL_DEC_MIN_GROUPS;
-    if (max_ctas > by_groups) max_ctas = by_groups;
-    if (max_ctas < sms) max_ctas = sms;
-    const int grid = n_groups < max_ctas ? n_groups : max_ctas;
+    // Resident CTAs per SM of a kernel variant with this shared memory.
+    auto prep = [&](const void *k, int *per_sm) {
+        cudaError_t e = ensure_dynamic_smem(k, smem);
+        if (e != cudaSuccess) return e;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, k, kDecThreads, smem) !=
+                cudaSuccess || *per_sm < 1)
+            *per_sm = 1;
+        return cudaSuccess;
+    };
+    // Split the units evenly (one share per resident CTA) when whole groups
+    // would not divide over the resident CTAs and every CTA still gets two
+    // groups' worth of units, so that a CTA's last segment usually finds its
+    // neighbour's part already added.
+    const int mode = g_split_mode.load();
+    bool split = false;
+    int per_sm = 1;
+    const void *kern = (const void *)decode_kernel<NT, R, FUSED, OUT_BF16, FMT, true>;
+    if (args.split_ws && mode != BITLINEAR_SPLIT_NEVER) {
+        cudaError_t e = prep(kern, &per_sm);
+        if (e != cudaSuccess) return e;
+        const int resident = sms * per_sm / BL_DEC_CTA_FRACTION;
+        split = mode == BITLINEAR_SPLIT_ALWAYS ||
+                (n_groups >= 2 * resident && n_groups % resident != 0);
+    }
+    int grid;
+    if (split) {
+        grid = sms * per_sm / BL_DEC_CTA_FRACTION;
+    } else {
+        args.split_ws = nullptr;
+        kern = (const void *)decode_kernel<NT, R, FUSED, OUT_BF16, FMT, false>;
+        cudaError_t e = prep(kern, &per_sm);
+        if (e != cudaSuccess) return e;
+        int max_ctas = sms * per_sm / BL_DEC_CTA_FRACTION;
+        const int by_groups = (n_groups + BL_DEC_MIN_GROUPS - 1) / BL_DEC_MIN_GROUPS;
+        if (max_ctas > by_groups) max_ctas = by_groups;
+        if (max_ctas < sms) max_ctas = sms;
+        grid = n_groups < max_ctas ? n_groups : max_ctas;
+    }
 
     *rec = LaunchRec();
-    rec->func = (const void *)kern;
+    rec->func = kern;
     rec->grid = dim3((unsigned)grid);
     rec->block = dim3(kDecThreads);
     rec->smem = smem;
@@ -746,6 +961,25 @@ static bitlinear_status prepare_decode(DecodeArgs args, bool fused, int out_dtyp
 
 size_t decode_x_offset() { return offsetof(DecodeArgs, X); }
 
+// Split workspace: one 64-bit word per output of 16 * (row tiles + 1) (one
+// spare tile: groups of two tiles may overhang d_out by one).
+size_t decode_workspace_bytes(int64_t d_out, int64_t T) {
+    if (T < 1 || T > 16 || d_out < 16) return 0;
+    const size_t bytes = 8 * (size_t)16 * (size_t)(d_out / 16 + 1) * (size_t)T;
+    return (bytes + 255) & ~(size_t)255;
+}
+
+static void set_split(DecodeArgs &a, void *ws) {
+    if (!ws || a.T < 1 || a.T > 16) return;
+    a.split_ws = static_cast<unsigned long long *>(ws);
+}
+
+bool decode_rec_splits(const LaunchRec &rec) {
+    DecodeArgs a;
+    std::memcpy(&a, rec.buf + rec.off[0], sizeof a);
+    return a.split_ws != nullptr;
+}
+
 bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, int fmt,
                                cudaStream_t stream) {
     LaunchRec rec;
@@ -757,7 +991,7 @@ bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, int f
 static DecodeArgs gemv_args(const void *packed, const float *gamma, int64_t d_out,
                             int64_t d_in, const int8_t *Xq, const float *beta,
                             const int32_t *rowsum, int64_t T, void *Y, int32_t *acc_out,
-                            bool static_weights, float qmax) {
+                            bool static_weights, float qmax, void *ws) {
     DecodeArgs a = {};
     a.packed = static_cast<const uint8_t *>(packed);
     a.gamma = gamma;
@@ -771,6 +1005,7 @@ static DecodeArgs gemv_args(const void *packed, const float *gamma, int64_t d_ou
     a.acc_out = acc_out;
     a.static_weights = static_weights ? 1 : 0;
     a.qmax = qmax;
+    set_split(a, ws);
     return a;
 }
 
@@ -778,9 +1013,9 @@ bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_o
                              int64_t d_in, const int8_t *Xq, const float *beta,
                              const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
                              int32_t *acc_out, bool static_weights, int fmt, float qmax,
-                             cudaStream_t stream) {
+                             void *ws, cudaStream_t stream) {
     return launch_decode(gemv_args(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, acc_out,
-                                   static_weights, qmax),
+                                   static_weights, qmax, ws),
                          false, out_dtype, fmt, stream);
 }
 
@@ -788,9 +1023,9 @@ bitlinear_status prepare_gemv(const void *packed, const float *gamma, int64_t d_
                               int64_t d_in, const int8_t *Xq, const float *beta,
                               const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
                               int32_t *acc_out, bool static_weights, int fmt, float qmax,
-                              LaunchRec *rec) {
+                              void *ws, LaunchRec *rec) {
     return prepare_decode(gemv_args(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, acc_out,
-                                    static_weights, qmax),
+                                    static_weights, qmax, ws),
                           false, out_dtype, fmt, rec);
 }
 
@@ -799,7 +1034,8 @@ bitlinear_status prepare_linear_fused(const void *packed, const float *gamma, in
                                       const float *gain, bool rmsnorm, float eps,
                                       float norm_eps, const float *inv_rms_in, int8_t *Xq,
                                       float *beta, int32_t *rowsum, void *Y, int out_dtype,
-                                      bool static_weights, int fmt, float qmax, LaunchRec *rec) {
+                                      bool static_weights, int fmt, float qmax, void *ws,
+                                      LaunchRec *rec) {
     DecodeArgs a = {};
     a.inv_rms_in = inv_rms_in;
     a.packed = static_cast<const uint8_t *>(packed);
@@ -819,6 +1055,7 @@ bitlinear_status prepare_linear_fused(const void *packed, const float *gamma, in
     a.Y = Y;
     a.static_weights = static_weights ? 1 : 0;
     a.qmax = qmax;
+    set_split(a, ws);
     return prepare_decode(a, true, out_dtype, fmt, rec);
 }
 
@@ -827,12 +1064,12 @@ bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
                                      const float *inv_rms_in, int8_t *Xq, float *beta,
                                      int32_t *rowsum, void *Y, int out_dtype,
-                                     bool static_weights, int fmt, float qmax,
+                                     bool static_weights, int fmt, float qmax, void *ws,
                                      cudaStream_t stream) {
     LaunchRec rec;
     bitlinear_status st = prepare_linear_fused(packed, gamma, d_out, d_in, X, T, gain, rmsnorm,
                                                eps, norm_eps, inv_rms_in, Xq, beta, rowsum, Y,
-                                               out_dtype, static_weights, fmt, qmax, &rec);
+                                               out_dtype, static_weights, fmt, qmax, ws, &rec);
     if (st != BITLINEAR_OK) return st;
     return rec.launch(stream) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.bitlinear_version() == 2
+    assert lib.bitlinear_version() == 3
     for code in range(0, 7):
         s = bl.status_string(code)
         assert s and s != "unknown status"
@@ -76,9 +76,10 @@ S0 = ctypes.c_void_p(0)
 
 
 def _fwd(lib, packed=0x10000, gamma=0x20000, d_out=64, d_in=256, xq=0x30000, beta=0x40000,
-         rowsum=0x50000, T=4, Y=0x60000, od=0, acc=None):
+         rowsum=0x50000, T=4, Y=0x60000, od=0, acc=None, ws=None, ws_bytes=0):
     return lib.bitlinear_forward(P(packed), P(gamma), d_out, d_in, P(xq), P(beta), P(rowsum), T,
-                                 P(Y), od, P(acc) if acc else None, S0)
+                                 P(Y), od, P(acc) if acc else None, P(ws) if ws else None,
+                                 ws_bytes, S0)
 
 
 def test_forward_validation(lib):
@@ -96,6 +97,35 @@ def test_forward_validation(lib):
     assert _fwd(lib, T=0, xq=0, beta=0, rowsum=0) == bl.OK
 
 
+def test_decode_workspace_rules(lib):
+    """The split workspace: one 8-byte word per output and token (one spare
+    16-row tile), rounded up to 256 bytes; only for 1 <= T <= 16; a workspace
+    that is too small or misaligned is refused before anything is
+    enqueued."""
+    nb = lib.bitlinear_decode_workspace_bytes
+    for d_out, T in ((64, 4), (28672, 1), (28672, 16), (6912, 8), (16, 1)):
+        n_rt = d_out // 16
+        want = 8 * 16 * (n_rt + 1) * T
+        assert nb(d_out, T) == (want + 255) // 256 * 256
+        assert bl.decode_workspace_bytes(d_out, T) == nb(d_out, T)
+    assert nb(64, 0) == 0 and nb(64, 17) == 0 and nb(24, 4) == 0 and nb(0, 4) == 0
+    need = nb(64, 4)
+    assert _fwd(lib, ws=0x70000, ws_bytes=need - 1) == bl.ERR_INVALID_ARG
+    assert _fwd(lib, ws=0x70008, ws_bytes=need) == bl.ERR_MISALIGNED
+    # T > 16 ignores the workspace's size (the prefill GEMM does not use it).
+    if not torch.cuda.is_available():
+        assert _fwd(lib, ws=0x70000, ws_bytes=need) == bl.ERR_DEVICE
+    lin = lib.bitlinear_linear
+    args = (P(0x10000), P(0x20000), 64, 256, P(0x30000), 4, None, 1, 1e-5, 1e-5, None,
+            P(0x40000), P(0x50000), P(0x60000), P(0x80000), 0)
+    assert lin(*args, P(0x70000), need - 4, S0) == bl.ERR_INVALID_ARG
+    assert lin(*args, P(0x70004), need, S0) == bl.ERR_MISALIGNED
+    assert lib.bitlinear_set_decode_split(3) == bl.ERR_INVALID_ARG
+    assert lib.bitlinear_set_decode_split(-1) == bl.ERR_INVALID_ARG
+    for mode in (bl.SPLIT_NEVER, bl.SPLIT_ALWAYS, bl.SPLIT_AUTO):
+        assert lib.bitlinear_set_decode_split(mode) == bl.OK
+
+
 def test_base3_sizes_and_validation(lib):
     """Five codes per byte on rows padded to 160 columns; base-3 entry points
     take 1 <= T <= 16 and validate like their 2-bit counterparts."""
@@ -107,7 +137,7 @@ def test_base3_sizes_and_validation(lib):
 
     def fwd(T=4, packed=0x10000, d_in=256, xq=0x30000):
         return f(P(packed), P(0x20000), 64, d_in, P(xq), P(0x40000), P(0x50000), T, P(0x60000),
-                 0, None, S0)
+                 0, None, None, 0, S0)
 
     assert fwd(T=17) == bl.ERR_UNSUPPORTED_SHAPE
     assert fwd(d_in=200) == bl.ERR_UNSUPPORTED_SHAPE
@@ -116,9 +146,11 @@ def test_base3_sizes_and_validation(lib):
     assert fwd(T=0, xq=0) == bl.OK
     lin = lib.bitlinear_linear_base3
     assert lin(P(0x10000), P(0x20000), 64, 256, P(0x30000), 17, None, 1, 1e-5, 1e-5, None,
-               P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0) == bl.ERR_UNSUPPORTED_SHAPE
+               P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, None, 0,
+               S0) == bl.ERR_UNSUPPORTED_SHAPE
     assert lin(P(0x10000), P(0x20000), 64, 256, P(0x30000), 4, None, 8, 1e-5, 1e-5, None,
-               P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0) == bl.ERR_INVALID_ARG
+               P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, None, 0,
+               S0) == bl.ERR_INVALID_ARG
     rp = lib.bitlinear_repack_base3
     assert rp(P(0x10000), 16, 128, P(0x20000), S0) == bl.ERR_UNSUPPORTED_SHAPE
     assert rp(P(0x10000), 16, 256, None, S0) == bl.ERR_INVALID_ARG
@@ -137,7 +169,7 @@ def test_w1_sizes_and_validation(lib):
 
     def fwd(T=4, bits=4, d_in=256, packed=0x10000):
         return f(P(packed), P(0x20000), 64, d_in, P(0x30000), P(0x40000), P(0x50000), T, bits,
-                 P(0x60000), 0, None, S0)
+                 P(0x60000), 0, None, None, 0, S0)
 
     assert fwd(T=17) == bl.ERR_UNSUPPORTED_SHAPE
     assert fwd(bits=5) == bl.ERR_INVALID_ARG
@@ -145,11 +177,12 @@ def test_w1_sizes_and_validation(lib):
     assert fwd(packed=0x10004) == bl.ERR_MISALIGNED
     assert fwd(T=0) == bl.OK
     args = (P(0x10000), P(0x20000), 64, 256, P(0x30000), 4, None)
-    tail = (1e-5, 1e-5, None, P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0)
+    tail = (1e-5, 1e-5, None, P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, None, 0, S0)
     assert lib.bitlinear_linear(*args, 1 | bl.ACT_4BIT, *tail) == bl.ERR_INVALID_ARG
     assert lib.bitlinear_linear_w1(*args, 16, *tail) == bl.ERR_INVALID_ARG
     # A supplied reciprocal RMS must be 4-byte aligned.
-    tail_r = (1e-5, 1e-5, P(0x80002), P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, S0)
+    tail_r = (1e-5, 1e-5, P(0x80002), P(0x40000), P(0x50000), P(0x60000), P(0x70000), 0, None, 0,
+              S0)
     assert lib.bitlinear_linear(*args, 1, *tail_r) == bl.ERR_MISALIGNED
     pk = lib.bitlinear_pack_weights_w1
     assert pk(P(0x10000), 16, 128, None, P(0x20000), 1 << 20, P(0x30000), P(0x40000),

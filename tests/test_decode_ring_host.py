@@ -5,8 +5,8 @@ ring of `stages` shared-memory stages.  One producer thread arms a stage's
 `full` barrier with the bytes it expects, then issues the weight copies and, for
 the product-only variant, the activation copies.  Four consumer warps wait on
 `full`, multiply, and arrive on `empty`.  With static weights the producer
-issues the first stages' weight copies before the dependency wait, and the main
-loop then adds only their activation copies, whose bytes the earlier arm already
+issues the first unit's weight copies before the dependency wait, and the main
+loop then adds only its activation copies, whose bytes the earlier arm already
 counted.  This model restates that loop and the kernel's parity arithmetic, runs
 it under random interleavings with copies landing in any order, and checks:
 - no deadlock;
@@ -22,13 +22,17 @@ DEC_WARPS = 4
 
 
 def test_model_constants_match_kernel_source():
-    """The model's warp count is the kernel's (csrc/gemv.cu)."""
+    """The model's warp count and prefetch rule are the kernel's (csrc/gemv.cu)."""
     import os
     import re
     path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
                         "ternary_weight_linear_bitlinear_b200", "csrc", "gemv.cu")
-    m = re.search(r"constexpr int kDecWarps = (\d+);", open(path).read())
+    src = open(path).read()
+    m = re.search(r"constexpr int kDecWarps = (\d+);", src)
     assert m and int(m.group(1)) == DEC_WARPS
+    # the number of units whose weights are requested before the dependency wait
+    assert "const int first = units < 1 ? units : 1;" in src
+    assert "} else if (!a.static_weights || u >= first) {" in src
 
 
 class Protocol(AssertionError):
@@ -122,7 +126,7 @@ class Ring:
                     self.full[st].copy_landed(u // S)
                 self.copies.append(land)
 
-        first = min(U, S)
+        first = min(U, 1)
         if self.static:
             for u in range(first):
                 issue_w(u, u)
@@ -132,7 +136,7 @@ class Ring:
             if rnd > 0:
                 yield self.empty[st], rnd - 1
                 issue_w(u, st)
-            elif not self.static:
+            elif not self.static or u >= first:
                 issue_w(u, st)
             issue_x(u, st)
             st += 1

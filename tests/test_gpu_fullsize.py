@@ -50,14 +50,17 @@ def run_problem(p: Problem, out_dtype, samples=512, check_packed=True, record=No
     xq_ref, beta_ref, rs_ref, rms_ref = oracle.quant_act(xb, eps=EPS)
     Xd = X.to(dev)
     T = p.tokens
+    ws = bl.decode_workspace(p.d_out, T, dev)   # the benchmark's split workspace (T <= 16)
 
     def call(inv_rms=None):
         sc = (Guarded((T, p.d_in), torch.int8), Guarded((T,), torch.float32),
               Guarded((T,), torch.int32))
         gy = Guarded((T, p.d_out), out_dtype)
         y = bl.linear(w, Xd, out=gy.t, scratch=tuple(x.t for x in sc), static_weights=True,
-                      inv_rms=inv_rms)
+                      inv_rms=inv_rms, workspace=ws)
         check_all(gy, *sc)
+        if ws is not None:
+            assert int(torch.count_nonzero(ws).item()) == 0
         return y, sc
 
     # The benchmarked call (static weights, its own reciprocal RMS), and the
@@ -69,7 +72,7 @@ def run_problem(p: Problem, out_dtype, samples=512, check_packed=True, record=No
     np.testing.assert_array_equal(sc_sup[2].t.cpu().numpy(), rs_ref)
     xq, beta, rowsum = (x.t for x in sc_sup)
     ga = Guarded((T, p.d_out), torch.int32)
-    _, acc = bl.forward(w, xq, beta, rowsum, out_dtype=out_dtype, acc=ga.t)
+    _, acc = bl.forward(w, xq, beta, rowsum, out_dtype=out_dtype, acc=ga.t, workspace=ws)
     check_all(ga)
     _, _, _, r_own = bl.quant_act(Xd)
     np.testing.assert_allclose(r_own.cpu().numpy(), rms_ref, rtol=1e-6)
