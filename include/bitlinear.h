@@ -246,7 +246,8 @@ int bitlinear_forward(const uint32_t *packed, const float *gamma, int64_t d_out,
 
 /* Bytes of the split workspace of a decode product with d_out outputs and T
  * tokens (1 <= T <= 16), or 0 for other T or an unsupported d_out:
- * 8 * 16 * (d_out / 16 + 1) * T rounded up to a multiple of 256. */
+ * 8 * T * R with R = 16 * (d_out / 16 + 1) rounded up to a multiple of 128,
+ * the total rounded up to a multiple of 256. */
 size_t bitlinear_decode_workspace_bytes(int64_t d_out, int64_t T);
 
 /* When decode calls given a split workspace split their units (process-wide;
@@ -260,6 +261,20 @@ size_t bitlinear_decode_workspace_bytes(int64_t d_out, int64_t T);
 #define BITLINEAR_SPLIT_ALWAYS 1
 #define BITLINEAR_SPLIT_NEVER 2
 int bitlinear_set_decode_split(int mode);
+
+/* Which product kernel decode calls (T <= 16) on 2-bit weights use
+ * (process-wide; calls and plans made afterwards follow it):
+ * BITLINEAR_DECODE_AUTO (default: by shape and T), BITLINEAR_DECODE_WARP_MMA
+ * (warp-level mma.sync on codes decoded in registers; the only one with the
+ * one-kernel quantise-and-multiply path) or BITLINEAR_DECODE_TCGEN05 (codes
+ * written to tensor memory, tcgen05.mma of 128 weight rows x 16 token slots;
+ * bitlinear_linear then runs the quantiser first).  The results are the same
+ * integers with every kernel.  Returns BITLINEAR_ERR_INVALID_ARG for another
+ * value. */
+#define BITLINEAR_DECODE_AUTO 0
+#define BITLINEAR_DECODE_WARP_MMA 1
+#define BITLINEAR_DECODE_TCGEN05 2
+int bitlinear_set_decode_kernel(int mode);
 
 /*
  * bitlinear_linear -- the whole BitLinear forward from bf16 activations:

@@ -56,6 +56,7 @@ SIGNATURES = {
                                  _vp, _vp, ctypes.c_size_t, _vp]),
     "bitlinear_decode_workspace_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bitlinear_set_decode_split": (_int, [_int]),
+    "bitlinear_set_decode_kernel": (_int, [_int]),
     "bitlinear_linear": (_int, [_vp, _vp, _i64, _i64, _vp, _i64, _vp, _u32, _f32, _f32, _vp,
                                 _vp, _vp, _vp, _vp, _int, _vp, ctypes.c_size_t, _vp]),
     "bitlinear_base3_bytes": (ctypes.c_size_t, [_i64, _i64]),
@@ -302,6 +303,15 @@ def set_decode_split(mode: int) -> None:
     """When decode calls with a split workspace split their units:
     SPLIT_AUTO (default), SPLIT_ALWAYS (tests) or SPLIT_NEVER; process-wide."""
     _check(lib().bitlinear_set_decode_split(mode), "bitlinear_set_decode_split")
+
+
+DECODE_AUTO, DECODE_WARP_MMA, DECODE_TCGEN05 = 0, 1, 2
+
+
+def set_decode_kernel(mode: int) -> None:
+    """Which product kernel 2-bit decode calls (T <= 16) use: DECODE_AUTO
+    (default), DECODE_WARP_MMA or DECODE_TCGEN05; process-wide."""
+    _check(lib().bitlinear_set_decode_kernel(mode), "bitlinear_set_decode_kernel")
 
 
 def decode_workspace_bytes(d_out: int, T: int) -> int:

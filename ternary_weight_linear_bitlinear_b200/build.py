@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libbitlinear.so")
-SOURCES = ["abi.cu", "pack.cu", "quant_act.cu", "gemv.cu", "gemm_tc.cu", "dense_bf16.cu",
+SOURCES = ["abi.cu", "pack.cu", "quant_act.cu", "gemv.cu", "gemv_tc.cu", "gemm_tc.cu", "dense_bf16.cu",
            "backward.cu"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -23,7 +23,13 @@ bitlinear_status launch_gemv(const void *packed, const float *gamma, int64_t d_o
 bool decode_can_fuse(int64_t T, int64_t d_in);
 size_t decode_workspace_bytes(int64_t d_out, int64_t T);
 int set_decode_split_mode(int mode);
-bool decode_rec_splits(const LaunchRec &rec);
+int set_decode_kernel(int mode);
+bool decode_use_tc(int64_t T, int64_t d_out, int64_t d_in);
+bitlinear_status prepare_decode_tc(const uint32_t *packed, const float *gamma, int64_t d_out,
+                                   int64_t d_in, const int8_t *Xq, const float *beta,
+                                   const int32_t *rowsum, int64_t T, void *Y, int out_dtype,
+                                   int32_t *acc_out, bool static_weights, void *ws,
+                                   LaunchRec *rec);
 bitlinear_status launch_linear_fused(const void *packed, const float *gamma, int64_t d_out,
                                      int64_t d_in, const uint16_t *X, int64_t T,
                                      const float *gain, bool rmsnorm, float eps, float norm_eps,
@@ -158,6 +164,14 @@ static bitlinear_status dispatch_forward(const void *packed, const float *gamma,
                                          void *Y, int out_dtype, int32_t *acc_out,
                                          bool static_weights, int fmt, float qmax, void *ws,
                                          cudaStream_t stream) {
+    if (T <= 16 && fmt == kFmt2Bit && qmax == 127.0f && decode_use_tc(T, d_out, d_in)) {
+        LaunchRec rec;
+        bitlinear_status st = prepare_decode_tc(static_cast<const uint32_t *>(packed), gamma,
+                                                d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
+                                                acc_out, static_weights, ws, &rec);
+        if (st != BITLINEAR_OK) return st;
+        return rec.launch(stream) == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+    }
     if (T <= 16 || fmt != kFmt2Bit)
         return launch_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y, out_dtype,
                            acc_out, static_weights, fmt, qmax, ws, stream);
@@ -238,7 +252,8 @@ static bitlinear_status linear_common(const void *packed, const float *gamma, in
     const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
     const bool rmsnorm = (flags & BITLINEAR_RMSNORM) != 0;
     const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
-    if (!per_tensor && decode_can_fuse(T, d_in))
+    if (!per_tensor && decode_can_fuse(T, d_in) &&
+        !(fmt == kFmt2Bit && decode_use_tc(T, d_out, d_in)))
         return launch_linear_fused(packed, gamma, d_out, d_in, X, T, norm_gain, rmsnorm, eps,
                                    norm_eps, inv_rms_in, Xq, beta, rowsum, Y, out_dtype,
                                    static_weights, fmt, qmax, ws, stream);
@@ -284,6 +299,8 @@ using namespace bl;
 extern "C" int bitlinear_version(void) { return 3; }
 
 extern "C" int bitlinear_set_decode_split(int mode) { return set_decode_split_mode(mode); }
+
+extern "C" int bitlinear_set_decode_kernel(int mode) { return set_decode_kernel(mode); }
 
 extern "C" size_t bitlinear_decode_workspace_bytes(int64_t d_out, int64_t T) {
     if (d_out <= 0 || d_out % 16 || d_out > (1 << 22)) return 0;
@@ -481,7 +498,7 @@ extern "C" int bitlinear_linear_plan_create(const uint32_t *packed, const float 
         p->steps = 0;
     } else if (per_tensor) {
         p->steps = -1;   // three launches with a folded beta: run as bitlinear_linear
-    } else if (decode_can_fuse(T, d_in)) {
+    } else if (decode_can_fuse(T, d_in) && !decode_use_tc(T, d_out, d_in)) {
         st = prepare_linear_fused(packed, gamma, d_out, d_in, nullptr, T, norm_gain, rmsnorm, eps,
                                   norm_eps, nullptr, Xq, beta, rowsum, Y, out_dtype,
                                   static_weights, kFmt2Bit, 127.0f, p->ws, &p->rec[0]);
@@ -492,17 +509,17 @@ extern "C" int bitlinear_linear_plan_create(const uint32_t *packed, const float 
                                norm_eps, nullptr, Xq, beta, rowsum, nullptr, true, &p->rec[0]);
         p->x_field = 0;
         if (st == BITLINEAR_OK)
-            st = T <= 16 ? prepare_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y,
+            st = T <= 16 && decode_use_tc(T, d_out, d_in)
+                     ? prepare_decode_tc(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y,
+                                         out_dtype, nullptr, static_weights, p->ws, &p->rec[1])
+                 : T <= 16 ? prepare_gemv(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y,
                                         out_dtype, nullptr, static_weights, kFmt2Bit, 127.0f,
                                         p->ws, &p->rec[1])
                          : prepare_gemm_tc_pair(packed, gamma, d_out, d_in, Xq, beta, rowsum, T, Y,
                                                 out_dtype, nullptr, &p->rec[1]);
         p->steps = 2;
     }
-    const bool splits = (p->steps == 1 && decode_rec_splits(p->rec[0])) ||
-                        (p->steps == 2 && T <= 16 && decode_rec_splits(p->rec[1])) ||
-                        p->steps == -1;
-    if (p->ws && (st != BITLINEAR_OK || !splits)) {
+    if (p->ws && st != BITLINEAR_OK) {
         cudaFree(p->ws);
         p->ws = nullptr;
         p->ws_bytes = 0;

@@ -808,6 +808,30 @@ constexpr int kDecSmemReserve = 8 * 1024;   // per CTA: static shared memory + t
 // split"): BITLINEAR_SPLIT_AUTO, _ALWAYS or _NEVER.
 static std::atomic<int> g_split_mode{BITLINEAR_SPLIT_AUTO};
 
+int decode_split_mode() { return g_split_mode.load(); }
+
+// Which decode product kernel T <= 16 calls on 2-bit weights use:
+// BITLINEAR_DECODE_AUTO, _WARP_MMA (mma.sync) or _TCGEN05.
+static std::atomic<int> g_decode_kernel{BITLINEAR_DECODE_AUTO};
+
+int set_decode_kernel(int mode) {
+    if (mode != BITLINEAR_DECODE_AUTO && mode != BITLINEAR_DECODE_WARP_MMA &&
+        mode != BITLINEAR_DECODE_TCGEN05)
+        return BITLINEAR_ERR_INVALID_ARG;
+    g_decode_kernel.store(mode);
+    return BITLINEAR_OK;
+}
+
+bool decode_use_tc(int64_t T, int64_t d_out, int64_t d_in) {
+    const int mode = g_decode_kernel.load();
+    if (mode == BITLINEAR_DECODE_TCGEN05) return true;
+    if (mode == BITLINEAR_DECODE_WARP_MMA) return false;
+    (void)T;
+    (void)d_out;
+    (void)d_in;
+    return false;
+}
+
 int set_decode_split_mode(int mode) {
     if (mode != BITLINEAR_SPLIT_AUTO && mode != BITLINEAR_SPLIT_ALWAYS &&
         mode != BITLINEAR_SPLIT_NEVER)
@@ -961,11 +985,14 @@ static bitlinear_status prepare_decode(DecodeArgs args, bool fused, int out_dtyp
 
 size_t decode_x_offset() { return offsetof(DecodeArgs, X); }
 
-// Split workspace: one 64-bit word per output of 16 * (row tiles + 1) (one
-// spare tile: groups of two tiles may overhang d_out by one).
+// Split workspace: one 64-bit word per token and row of 16 * (row tiles + 1)
+// rows rounded up to a multiple of 128 (groups of two 16-row tiles may
+// overhang d_out by one tile, the tensor-core kernel's 128-row blocks by up
+// to 112 rows).
 size_t decode_workspace_bytes(int64_t d_out, int64_t T) {
     if (T < 1 || T > 16 || d_out < 16) return 0;
-    const size_t bytes = 8 * (size_t)16 * (size_t)(d_out / 16 + 1) * (size_t)T;
+    const size_t rows = ((size_t)16 * (size_t)(d_out / 16 + 1) + 127) & ~(size_t)127;
+    const size_t bytes = 8 * rows * (size_t)T;
     return (bytes + 255) & ~(size_t)255;
 }
 
@@ -974,11 +1001,6 @@ static void set_split(DecodeArgs &a, void *ws) {
     a.split_ws = static_cast<unsigned long long *>(ws);
 }
 
-bool decode_rec_splits(const LaunchRec &rec) {
-    DecodeArgs a;
-    std::memcpy(&a, rec.buf + rec.off[0], sizeof a);
-    return a.split_ws != nullptr;
-}
 
 bitlinear_status launch_decode(DecodeArgs args, bool fused, int out_dtype, int fmt,
                                cudaStream_t stream) {

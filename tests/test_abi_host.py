@@ -98,15 +98,16 @@ def test_forward_validation(lib):
 
 
 def test_decode_workspace_rules(lib):
-    """The split workspace: one 8-byte word per output and token (one spare
-    16-row tile), rounded up to 256 bytes; only for 1 <= T <= 16; a workspace
-    that is too small or misaligned is refused before anything is
-    enqueued."""
+    """The split workspace: one 8-byte word per token and row of d_out plus a
+    spare 16-row tile, rounded up to 128 rows, the total to 256 bytes; only
+    for 1 <= T <= 16; a workspace that is too small or misaligned is refused
+    before anything is enqueued."""
     nb = lib.bitlinear_decode_workspace_bytes
-    for d_out, T in ((64, 4), (28672, 1), (28672, 16), (6912, 8), (16, 1)):
+    for d_out, T in ((64, 4), (28672, 1), (28672, 16), (6912, 8), (16, 1), (6928, 3)):
         n_rt = d_out // 16
-        want = 8 * 16 * (n_rt + 1) * T
-        assert nb(d_out, T) == (want + 255) // 256 * 256
+        rows = (16 * (n_rt + 1) + 127) // 128 * 128
+        want = (8 * rows * T + 255) // 256 * 256
+        assert nb(d_out, T) == want
         assert bl.decode_workspace_bytes(d_out, T) == nb(d_out, T)
     assert nb(64, 0) == 0 and nb(64, 17) == 0 and nb(24, 4) == 0 and nb(0, 4) == 0
     need = nb(64, 4)
@@ -124,6 +125,9 @@ def test_decode_workspace_rules(lib):
     assert lib.bitlinear_set_decode_split(-1) == bl.ERR_INVALID_ARG
     for mode in (bl.SPLIT_NEVER, bl.SPLIT_ALWAYS, bl.SPLIT_AUTO):
         assert lib.bitlinear_set_decode_split(mode) == bl.OK
+    assert lib.bitlinear_set_decode_kernel(3) == bl.ERR_INVALID_ARG
+    for mode in (bl.DECODE_WARP_MMA, bl.DECODE_TCGEN05, bl.DECODE_AUTO):
+        assert lib.bitlinear_set_decode_kernel(mode) == bl.OK
 
 
 def test_base3_sizes_and_validation(lib):

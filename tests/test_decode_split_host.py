@@ -46,6 +46,16 @@ def test_model_matches_kernel_source():
     assert "if (split_k(wd) + my_k != KB)" in src
     assert "if (split_k(wd) + my_k == KB) {" in src
     assert "if (split_k(first_w[j]) == KB) {" in src
+    # The tensor-core decode kernel uses the same word, partition and tests.
+    tc = open(SRC.replace("gemv.cu", "gemv_tc.cu")).read()
+    assert "constexpr int kSplitKShift = %d;" % K_SHIFT in tc
+    assert "constexpr int kSplitPartsShift = %d;" % PARTS_SHIFT in tc
+    assert "constexpr long long kSplitBias = 1ll << 25;" in tc
+    assert "const int U = n_mb * KB, q = U / P, rem = U - q * P;" in tc
+    assert "u0 = q * c + (c < rem ? c : rem);" in tc
+    assert "if (split_k(wd) + my_k != KB) wd = atomicAdd(w, split_word(my_k, vt));" in tc
+    assert "if (split_k(wd) + my_k == KB) {" in tc
+    assert "if (split_k(first_w[t]) == KB) {" in tc
 
 
 def segments(n_groups, KB, P, c):
@@ -195,17 +205,21 @@ def test_word_fields_hold_their_extremes():
 
 def ws_bytes(d_out, T):
     """bitlinear_decode_workspace_bytes, restated."""
-    b = 8 * 16 * (d_out // 16 + 1) * T
-    return (b + 255) // 256 * 256
+    rows = (16 * (d_out // 16 + 1) + 127) // 128 * 128
+    return (8 * rows * T + 255) // 256 * 256
 
 
-@pytest.mark.parametrize("d_out", [16, 32, 272, 6912, 18960, 28672])
+@pytest.mark.parametrize("d_out", [16, 32, 272, 6912, 6928, 18960, 28672])
 @pytest.mark.parametrize("T", [1, 8, 9, 16])
 def test_workspace_indices_in_bounds(d_out, T):
-    """Group g's words sit at [g T 16R, (g + 1) T 16R); every index the
-    kernel can form is inside the workspace."""
+    """Group g's words sit at [g T 16R, (g + 1) T 16R) (warp-MMA kernel), a
+    128-row block b's at [128 b T, 128 (b + 1) T) (tensor-core kernel); every
+    index either kernel can form is inside the workspace."""
     n_rt = d_out // 16
     for R in (1, 2):
         n_groups = (n_rt + R - 1) // R
         last = (n_groups - 1) * T * 16 * R + T * 16 * R - 1
         assert 8 * (last + 1) <= ws_bytes(d_out, T)
+    n_mb = (d_out + 127) // 128
+    last = ((n_mb - 1) * T + (T - 1)) * 128 + 127
+    assert 8 * (last + 1) <= ws_bytes(d_out, T)
