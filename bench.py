@@ -245,7 +245,7 @@ def capture(fn):
     return g
 
 
-DECODE_SOURCES = ("gemv.cu", "quant_common.cuh", "common.cuh")
+DECODE_SOURCES = ("gemv.cu", "quant_common.cuh", "common.cuh", "decode_common.cuh")
 GEMM_SOURCES = ("gemm_tc.cu", "common.cuh", "tc_common.cuh")
 
 
