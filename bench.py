@@ -619,54 +619,106 @@ def measure_e2e(run, steps):
     reads all its outputs back device -> host, inside the timed region.  The
     step is a LinearPlan call per layer (arguments bound once), run as a
     StepGraph (the step captured once as a CUDA graph, copies included, and
-    replayed) and, for comparison, eagerly."""
+    replayed): one step at a time on one stream, and double-buffered -- two
+    steps in flight on two streams with their own buffers, each step's kernels
+    ordered after the previous step's kernels (events), so that only the
+    copies of one step overlap the kernels of the other; eagerly for
+    comparison."""
     bl = run.bl
     dev = run.dev
     xs = [X for _, _, X, _, _, _ in run.layers]
     ys = [Y for _, _, _, _, Y, _ in run.layers]
     x_elems = [x.numel() for x in xs]
     y_elems = [y.numel() for y in ys]
-    host_x = torch.cat([x.reshape(-1) for x in xs]).cpu().pin_memory()
-    host_y = torch.empty(sum(y_elems), dtype=ys[0].dtype).pin_memory()
-    dev_x = torch.empty_like(host_x, device=dev)
-    dev_y = torch.empty(sum(y_elems), dtype=ys[0].dtype, device=dev)
-    x_views, y_views, ox, oy = [], [], 0, 0
-    for x, y, nx, ny in zip(xs, ys, x_elems, y_elems):
-        x_views.append(dev_x[ox:ox + nx].view(x.shape))
-        y_views.append(dev_y[oy:oy + ny].view(y.shape))
-        ox += nx
-        oy += ny
-    h2d = host_x.numel() * host_x.element_size()
-    d2h = host_y.numel() * host_y.element_size()
-    cs = torch.cuda.Stream()
-    plans = [bl.LinearPlan(w, X.shape[0], out=Y, scratch=scratch, static_weights=True, stream=cs)
-             for (_, w, _, scratch, _, _), X, Y in zip(run.layers, x_views, y_views)]
 
-    def one():
-        dev_x.copy_(host_x, non_blocking=True)
-        for plan, X in zip(plans, x_views):
-            plan(X)
-        host_y.copy_(dev_y, non_blocking=True)
+    class Lane:
+        """Pinned host X and Y, device buffers, scratch and plans of one step."""
+
+        def __init__(self, stream):
+            self.s = stream
+            self.host_x = torch.cat([x.reshape(-1) for x in xs]).cpu().pin_memory()
+            self.host_y = torch.empty(sum(y_elems), dtype=ys[0].dtype).pin_memory()
+            self.dev_x = torch.empty_like(self.host_x, device=dev)
+            self.dev_y = torch.empty(sum(y_elems), dtype=ys[0].dtype, device=dev)
+            self.x_views, y_views, ox, oy = [], [], 0, 0
+            for x, y, nx, ny in zip(xs, ys, x_elems, y_elems):
+                self.x_views.append(self.dev_x[ox:ox + nx].view(x.shape))
+                y_views.append(self.dev_y[oy:oy + ny].view(y.shape))
+                ox += nx
+                oy += ny
+            self.plans = []
+            for (p, w, X, _, _, _), Yv in zip(run.layers, y_views):
+                T = X.shape[0]
+                scratch = (torch.empty((T, p.d_in), dtype=torch.int8, device=dev),
+                           torch.empty(T, dtype=torch.float32, device=dev),
+                           torch.empty(T, dtype=torch.int32, device=dev))
+                self.plans.append(bl.LinearPlan(w, T, out=Yv, scratch=scratch,
+                                                static_weights=True, stream=stream))
+            self.graph = None
+            self.g_in = self.g_calls = self.g_out = None
+            self.done = torch.cuda.Event()   # this step's kernels finished
+
+        def copy_in(self):
+            self.dev_x.copy_(self.host_x, non_blocking=True)
+
+        def calls(self):
+            for plan, X in zip(self.plans, self.x_views):
+                plan(X)
+
+        def copy_out(self):
+            self.host_y.copy_(self.dev_y, non_blocking=True)
+
+        def one(self):
+            self.copy_in()
+            self.calls()
+            self.copy_out()
+
+    lanes = [Lane(torch.cuda.Stream()), Lane(torch.cuda.Stream())]
+    h2d = lanes[0].host_x.numel() * lanes[0].host_x.element_size()
+    d2h = lanes[0].host_y.numel() * lanes[0].host_y.element_size()
+    s0, s1 = lanes[0].s, lanes[1].s
 
     def timed(fn):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        a.record(cs)
-        for _ in range(steps):
-            fn()
-        b.record(cs)
+        a.record(s0)
+        s1.wait_stream(s0)
+        for i in range(steps):
+            fn(i)
+        s0.wait_stream(s1)
+        b.record(s0)
         b.synchronize()
         return a.elapsed_time(b) / steps
 
-    with torch.cuda.stream(cs):
-        one()
+    with torch.cuda.stream(s0):
+        lanes[0].one()
         torch.cuda.synchronize()
-        ms_eager = timed(one)
-        step = bl.StepGraph(one, stream=cs)
-        step()
-        ms_graph = timed(step)
-    return ms_graph, ms_eager, h2d, d2h
+        ms_eager = timed(lambda i: lanes[0].one())
+    for lane in lanes:
+        lane.graph = bl.StepGraph(lane.one, stream=lane.s)
+        lane.g_in = bl.StepGraph(lane.copy_in, stream=lane.s)
+        lane.g_calls = bl.StepGraph(lane.calls, stream=lane.s)
+        lane.g_out = bl.StepGraph(lane.copy_out, stream=lane.s)
+        lane.graph()
+    torch.cuda.synchronize()
 
+    def replay(lane):
+        with torch.cuda.stream(lane.s):
+            lane.graph()
+
+    def pipelined(i):
+        lane, prev = lanes[i % 2], lanes[(i + 1) % 2]
+        with torch.cuda.stream(lane.s):
+            lane.g_in()
+            if i > 0:
+                lane.s.wait_event(prev.done)   # kernels one step after another
+            lane.g_calls()
+            lane.done.record(lane.s)
+            lane.g_out()
+
+    ms_graph = timed(lambda i: replay(lanes[0]))
+    ms_pipe = timed(pipelined)
+    return ms_pipe, ms_graph, ms_eager, h2d, d2h
 
 
 # -------------------------------------------------------- CPU oracle ---
@@ -889,8 +941,9 @@ def main():
             extras["prefill"]["ms_gemm"])
         sampler.mark(False)
 
-    e2e_ms, e2e_eager_ms, h2d, d2h = measure_e2e(run, max(3, min(args.steps, 20)))
+    e2e_ms, e2e_serial_ms, e2e_eager_ms, h2d, d2h = measure_e2e(run, max(4, min(args.steps, 20)))
     e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_serial_ms = max_over_ranks(e2e_serial_ms, world)
     e2e_eager_ms = max_over_ranks(e2e_eager_ms, world)
     sampler.stop()
     status = run.bl.device_error(clear=True)
@@ -935,12 +988,18 @@ def main():
             "e2e": {"value": round(replica_value(nb["step"], world, e2e_ms), 3),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 4),
+                    "one_step_at_a_time": {
+                        "value": round(replica_value(nb["step"], world, e2e_serial_ms), 3),
+                        "ms_per_step": round(e2e_serial_ms, 4)},
                     "eager": {"value": round(replica_value(nb["step"], world, e2e_eager_ms), 3),
                               "ms_per_step": round(e2e_eager_ms, 4)},
                     "how": "public Python API: a LinearPlan per layer (bitlinear_linear with "
                            "bound arguments), the step replayed as a StepGraph (CUDA graph of "
                            "the copies and the calls); every step one copy of all its X in "
-                           "from pinned host memory and one of all its Y out"},
+                           "from pinned host memory and one of all its Y out; double-buffered: "
+                           "two steps in flight on two streams with their own buffers, each "
+                           "step's kernels after the previous step's kernels, so only copies "
+                           "overlap kernels"},
             "gpu_launches": (1 if one_kernel else 2) * len(run.layers) * args.steps,
             "clocks": clocks,
             "device_error": run.bl.status_string(status),
