@@ -114,8 +114,11 @@ struct __align__(8) Barriers {
     int abort_flag;
 };
 static_assert(sizeof(Barriers) <= 1024, "barrier block");
+// Epilogue staging for the tensor-map store of Y: per epilogue warp 4 KiB, two
+// 32 x 32 bf16 chunks (64-byte swizzle) or one fp32 chunk (128-byte swizzle).
+constexpr int kStageY = 4096;
 constexpr int kSmemBytes = kStages * kStage + kPSlots * kPUnit + 1024 /* barriers */ +
-                           1024 /* alignment slack */;
+                           kEpiWarps * kStageY + 1024 /* alignment slack */;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 // ------------------------------------------------------------- cluster ---
@@ -204,6 +207,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(pair::kThreads, 1)
 gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                    const __grid_constant__ CUtensorMap map_y,
                     const float *__restrict__ gamma_ptr, int d_out, int d_in,
                     const float *__restrict__ beta, const int32_t *__restrict__ rowsum, int T,
                     void *__restrict__ Y, int32_t *__restrict__ acc_out, DeviceCtx ctx) {
@@ -213,6 +217,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *p_ring = smem + kStages * kStage;
     Barriers *bars = reinterpret_cast<Barriers *>(p_ring + kPSlots * kPUnit);
+    uint8_t *y_stage = p_ring + kPSlots * kPUnit + 1024;   // 1024-byte aligned
     const uint32_t smem_base = smem_u32(smem);
     auto stage_x = [&](int s) { return smem_base + s * kStage; };   // token half; codes at + kBTile
 
@@ -457,6 +462,13 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
         const int quarter = warp & 3;
         const uint32_t lane_field = (uint32_t)(quarter * 32) << 16;
         const float gamma = *gamma_ptr;
+        // Without acc_out, each 32-row chunk of the warp's 32 tokens goes
+        // through shared memory (row = token, swizzled so the lanes' 16-byte
+        // writes do not conflict) and out with one tensor-map store, which
+        // writes whole lines and clips tokens past T and rows past d_out.
+        const bool staged = acc_out == nullptr;
+        const uint32_t ystage = smem_u32(y_stage) + (uint32_t)(quarter * kStageY);
+        int nchunk = 0;
         int i = 0;
         for (int tile = pair_id; tile < num_tiles; tile += num_pairs, ++i) {
             const int m0 = (tile % m_tiles) * 2 * kBM;
@@ -476,6 +488,56 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem_base + lane_field + buf * kAccCols + c * 32, v);
                 tmem_wait_ld();
+                if (staged) {
+                    // bf16: two 2 KiB buffers, at most one store still reading;
+                    // fp32: one 4 KiB buffer, no store still reading.
+                    const uint32_t sb = ystage + (OUT_BF16 ? (uint32_t)(nchunk & 1) * 2048u : 0u);
+                    if (lane == 0) {
+                        if (OUT_BF16) bulk_wait_read_1();
+                        else bulk_wait_read_0();
+                    }
+                    __syncwarp();
+                    float y[32];
+                    #pragma unroll
+                    for (int e = 0; e < 32; ++e) y[e] = __fmul_rn((float)((int)v[e] - rs), sc);
+                    if (OUT_BF16) {
+                        // row = lane, 64 bytes: chunk k at k ^ ((lane >> 1) & 3)
+                        #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            uint32_t pw[4];
+                            #pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __nv_bfloat162 h =
+                                    __floats2bfloat162_rn(y[8 * k + 2 * e], y[8 * k + 2 * e + 1]);
+                                pw[e] = *reinterpret_cast<const uint32_t *>(&h);
+                            }
+                            const uint32_t at = sb + (uint32_t)lane * 64u +
+                                                (((uint32_t)k ^ (((uint32_t)lane >> 1) & 3u)) << 4);
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(at),
+                                         "r"(pw[0]), "r"(pw[1]), "r"(pw[2]), "r"(pw[3])
+                                         : "memory");
+                        }
+                    } else {
+                        // row = lane, 128 bytes: chunk k at k ^ (lane & 7)
+                        #pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t at = sb + (uint32_t)lane * 128u +
+                                                (((uint32_t)k ^ ((uint32_t)lane & 7u)) << 4);
+                            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(at),
+                                         "f"(y[4 * k]), "f"(y[4 * k + 1]), "f"(y[4 * k + 2]),
+                                         "f"(y[4 * k + 3])
+                                         : "memory");
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&map_y, sb, o0, t - lane);
+                        bulk_commit_group();
+                    }
+                    ++nchunk;
+                    continue;
+                }
                 if (!live) continue;
                 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -515,6 +577,9 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
             __syncwarp();
             if (lane == 0) signal_leader(&bars->acc_empty[buf]);
         }
+        // Every staged store has completed before the CTA may exit.
+        if (staged && lane == 0) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -576,6 +641,22 @@ bitlinear_status prepare_gemm_tc_pair(const uint32_t *packed, const float *gamma
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BITLINEAR_ERR_CUDA;
     }
+    CUtensorMap map_y;
+    {
+        // Y [T][d_out]; boxes of 32 tokens x 32 outputs, the swizzle of the
+        // epilogue's staging (64-byte rows for bf16, 128-byte rows for fp32).
+        const cuuint64_t esz = bf ? 2 : 4;
+        const cuuint64_t dims[2] = {(cuuint64_t)d_out, (cuuint64_t)T};
+        const cuuint64_t strides[1] = {(cuuint64_t)d_out * esz};
+        const cuuint32_t box[2] = {32, 32};
+        const cuuint32_t estr[2] = {1, 1};
+        if (encode(&map_y, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   bf ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BITLINEAR_ERR_CUDA;
+    }
     auto kern = bf ? gemm_tc_pair_kernel<true> : gemm_tc_pair_kernel<false>;
     if (ensure_dynamic_smem((const void *)kern, kSmemBytes) != cudaSuccess)
         return BITLINEAR_ERR_CUDA;
@@ -591,6 +672,7 @@ bitlinear_status prepare_gemm_tc_pair(const uint32_t *packed, const float *gamma
     rec->pdl = true;
     rec->push(map_x);
     rec->push(map_w);
+    rec->push(map_y);
     rec->push(gamma);
     rec->push((int)d_out);
     rec->push((int)d_in);

@@ -135,6 +135,10 @@ __device__ __forceinline__ void bulk_commit_group() {
 __device__ __forceinline__ void bulk_wait_read_1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
+// No committed store group is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 // Every committed store group has completed.
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");

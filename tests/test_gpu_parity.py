@@ -334,6 +334,37 @@ def test_gemm_many_tiles_matches_oracle(d_out, d_in, T, out_dtype):
     forward_case(d_out, d_in, T, out_dtype)
 
 
+# Without acc_out the prefill GEMM's epilogue stages each 32 x 32 chunk in
+# shared memory and writes it with a tensor-map store (clipped at T and
+# d_out); with acc_out it writes both outputs directly.
+STAGED_CASES = [
+    (16, 256, 17, torch.float32),        # one 16-row tile; 17 tokens
+    (48, 768, 100, torch.bfloat16),
+    (144, 512, 300, torch.float32),      # a chunk straddling d_out (144 = 4.5 x 32)
+    (272, 768, 600, torch.bfloat16),
+    (4112, 256, 1100, torch.bfloat16),   # last row tile of 16 rows
+    (4096, 512, 1201, torch.float32),
+    (8192, 256, 1800, torch.float32),    # up to four pair tiles per pair
+]
+
+
+@pytest.mark.parametrize("d_out,d_in,T,out_dtype", STAGED_CASES)
+def test_gemm_staged_store_matches_oracle(d_out, d_in, T, out_dtype):
+    W, X = draw(Problem("gs", d_in, d_out, T, 0.02, 0.01, 50.0, 7))
+    o = oracle_side(W, X)
+    w = bl.PackedTernary(to_dev(oracle.pack(o["wq"]).view(np.int32)),
+                         torch.tensor([o["gamma"]], device=dev()), d_out, d_in)
+    xq, beta, rs = to_dev(o["xq"]), to_dev(o["beta"]), to_dev(o["rowsum"])
+    gy = Guarded((T, d_out), out_dtype)
+    y = bl.forward(w, xq, beta, rs, out=gy.t)
+    check_all(gy)
+    acc_ref = oracle.int_matmul(o["wq"], o["xq"])
+    check_y(y, acc_ref, o["gamma"], o["beta"], out_dtype == torch.bfloat16)
+    y2, acc = bl.forward(w, xq, beta, rs, out_dtype=out_dtype, want_acc=True)
+    assert torch.equal(y, y2)
+    np.testing.assert_array_equal(acc.cpu().numpy(), acc_ref)
+
+
 def test_forward_zero_inputs():
     for T in (1, 40):
         d_out, d_in = 64, 512
