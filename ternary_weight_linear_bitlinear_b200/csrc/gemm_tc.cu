@@ -114,9 +114,12 @@ struct __align__(8) Barriers {
     int abort_flag;
 };
 static_assert(sizeof(Barriers) <= 1024, "barrier block");
-// Epilogue staging for the tensor-map store of Y: per epilogue warp 4 KiB, two
-// 32 x 32 bf16 chunks (64-byte swizzle) or one fp32 chunk (128-byte swizzle).
-constexpr int kStageY = 4096;
+// Epilogue staging for the tensor-map store of Y: per epilogue warp 2 KiB, one
+// box of 32 tokens x 64 bytes (32 bf16 or 16 fp32 outputs, 64-byte swizzle).
+// Small enough that a quantiser CTA still fits beside this CTA on its SM, so
+// that under a programmatic launch this CTA's prologue overlaps the
+// quantiser (measured: 4 KiB per warp lost that overlap).
+constexpr int kStageY = 2048;
 constexpr int kSmemBytes = kStages * kStage + kPSlots * kPUnit + 1024 /* barriers */ +
                            kEpiWarps * kStageY + 1024 /* alignment slack */;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
@@ -468,7 +471,6 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
         // writes whole lines and clips tokens past T and rows past d_out.
         const bool staged = acc_out == nullptr;
         const uint32_t ystage = smem_u32(y_stage) + (uint32_t)(quarter * kStageY);
-        int nchunk = 0;
         int i = 0;
         for (int tile = pair_id; tile < num_tiles; tile += num_pairs, ++i) {
             const int m0 = (tile % m_tiles) * 2 * kBM;
@@ -489,53 +491,43 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
                 tmem_ld_32x32b_x32(tmem_base + lane_field + buf * kAccCols + c * 32, v);
                 tmem_wait_ld();
                 if (staged) {
-                    // bf16: two 2 KiB buffers, at most one store still reading;
-                    // fp32: one 4 KiB buffer, no store still reading.
-                    const uint32_t sb = ystage + (OUT_BF16 ? (uint32_t)(nchunk & 1) * 2048u : 0u);
-                    if (lane == 0) {
-                        if (OUT_BF16) bulk_wait_read_1();
-                        else bulk_wait_read_0();
-                    }
-                    __syncwarp();
                     float y[32];
                     #pragma unroll
                     for (int e = 0; e < 32; ++e) y[e] = __fmul_rn((float)((int)v[e] - rs), sc);
-                    if (OUT_BF16) {
+                    // bf16: one box of the 32 outputs; fp32: two boxes of 16.
+                    constexpr int kBoxes = OUT_BF16 ? 1 : 2;
+                    #pragma unroll
+                    for (int h = 0; h < kBoxes; ++h) {
+                        if (lane == 0) bulk_wait_read_0();   // the buffer's last store has read it
+                        __syncwarp();
                         // row = lane, 64 bytes: chunk k at k ^ ((lane >> 1) & 3)
                         #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             uint32_t pw[4];
-                            #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const __nv_bfloat162 h =
-                                    __floats2bfloat162_rn(y[8 * k + 2 * e], y[8 * k + 2 * e + 1]);
-                                pw[e] = *reinterpret_cast<const uint32_t *>(&h);
+                            if (OUT_BF16) {
+                                #pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const __nv_bfloat162 hh = __floats2bfloat162_rn(
+                                        y[8 * k + 2 * e], y[8 * k + 2 * e + 1]);
+                                    pw[e] = *reinterpret_cast<const uint32_t *>(&hh);
+                                }
+                            } else {
+                                #pragma unroll
+                                for (int e = 0; e < 4; ++e) pw[e] = __float_as_uint(y[16 * h + 4 * k + e]);
                             }
-                            const uint32_t at = sb + (uint32_t)lane * 64u +
+                            const uint32_t at = ystage + (uint32_t)lane * 64u +
                                                 (((uint32_t)k ^ (((uint32_t)lane >> 1) & 3u)) << 4);
                             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(at),
                                          "r"(pw[0]), "r"(pw[1]), "r"(pw[2]), "r"(pw[3])
                                          : "memory");
                         }
-                    } else {
-                        // row = lane, 128 bytes: chunk k at k ^ (lane & 7)
-                        #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const uint32_t at = sb + (uint32_t)lane * 128u +
-                                                (((uint32_t)k ^ ((uint32_t)lane & 7u)) << 4);
-                            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(at),
-                                         "f"(y[4 * k]), "f"(y[4 * k + 1]), "f"(y[4 * k + 2]),
-                                         "f"(y[4 * k + 3])
-                                         : "memory");
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&map_y, ystage, o0 + 16 * h, t - lane);
+                            bulk_commit_group();
                         }
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&map_y, sb, o0, t - lane);
-                        bulk_commit_group();
-                    }
-                    ++nchunk;
                     continue;
                 }
                 if (!live) continue;
@@ -643,16 +635,16 @@ bitlinear_status prepare_gemm_tc_pair(const uint32_t *packed, const float *gamma
     }
     CUtensorMap map_y;
     {
-        // Y [T][d_out]; boxes of 32 tokens x 32 outputs, the swizzle of the
-        // epilogue's staging (64-byte rows for bf16, 128-byte rows for fp32).
+        // Y [T][d_out]; boxes of 32 tokens x 64 bytes (32 bf16 or 16 fp32
+        // outputs), the 64-byte swizzle of the epilogue's staging.
         const cuuint64_t esz = bf ? 2 : 4;
         const cuuint64_t dims[2] = {(cuuint64_t)d_out, (cuuint64_t)T};
         const cuuint64_t strides[1] = {(cuuint64_t)d_out * esz};
-        const cuuint32_t box[2] = {32, 32};
+        const cuuint32_t box[2] = {bf ? 32u : 16u, 32};
         const cuuint32_t estr[2] = {1, 1};
         if (encode(&map_y, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                    2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   bf ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BITLINEAR_ERR_CUDA;
