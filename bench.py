@@ -1013,18 +1013,27 @@ def main():
 
 
 def reference_arm(args, warmup):
-    """The CPU oracle timed on this host: each step is a bounded sample
-    (one BitLinear forward of the workload's shape), same metric and unit."""
+    """The CPU oracle timed on this host, same metric and unit.  A step is as
+    many BitLinear forwards of the workload as the GPU arm's step (LAYERS,
+    cycling through the workload's layers), unless K such steps would take
+    more than about two minutes on this host; then fewer forwards per step,
+    as config.forwards_per_step says."""
     import oracle
     wl = WORKLOADS[args.workload]
     prepared = _oracle_prepared(args.workload)
     threads = oracle.threads(parallel=True)
-    for i in range(warmup):
+    per_step = max(1, LAYERS // len(prepared)) * len(prepared)
+    t1 = time.perf_counter()
+    for i in range(max(warmup, 1)):
         p, wq, g, xb = prepared[i % len(prepared)]
         oracle_layer_step(p, wq, g, xb, parallel=True)
+    one = (time.perf_counter() - t1) / max(warmup, 1)
+    budget_s = 120.0
+    if args.steps * per_step * one > budget_s:
+        per_step = max(1, int(budget_s / (args.steps * one)))
     nbytes = 0
     t0 = time.perf_counter()
-    for i in range(args.steps):
+    for i in range(args.steps * per_step):
         p, wq, g, xb = prepared[i % len(prepared)]
         oracle_layer_step(p, wq, g, xb, parallel=True)
         nbytes += decode_bytes(p)["step"]
@@ -1035,14 +1044,14 @@ def reference_arm(args, warmup):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": warmup,
         "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": args.workload, "forwards_per_step": 1,
+        "config": {"workload": args.workload, "forwards_per_step": per_step,
                    "tokens": wl.problems[0].tokens, "d_in": wl.problems[0].d_in,
                    "d_out": wl.problems[0].d_out},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle", "host_cpus": len(os.sched_getaffinity(0)),
-                         "sample": "each step one BitLinear forward of the workload by the "
+                         "sample": "each step %d BitLinear forwards of the workload by the "
                                    "plain C oracle, its product split over %d OpenMP threads"
-                                   % threads},
+                                   % (per_step, threads)},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
