@@ -157,6 +157,10 @@ QA_CASES = [
     (5, 1024, 0.01, 50.0, True, True),
     (2048, 4096, 0.0, 1.0, True, False),
     (1, 65536, 0.001, 100.0, True, False),
+    # More tokens than the GPU holds quantiser CTAs at once (several waves).
+    (2400, 768, 0.01, 50.0, True, True),
+    (2411, 256, 0.01, 50.0, False, False),
+    (2400, 8448, 0.005, 100.0, True, False),   # 1056 vectors: a short last batch
 ]
 
 
@@ -212,7 +216,7 @@ def test_quant_act_special_tokens():
 PER_TENSOR_CASES = [
     # (T, K, rmsnorm, gain)
     (1, 512, True, False), (5, 512, True, True), (40, 1024, False, False),
-    (300, 4096, True, False), (1100, 256, True, False),
+    (300, 4096, True, False), (1100, 256, True, False), (2400, 512, True, True),
 ]
 
 
@@ -523,6 +527,7 @@ PLAN_CASES = [
     (6912, 2560, 1, bl.RMSNORM | bl.STATIC_WEIGHTS),     # fused quantiser + GEMV
     (272, 4096, 12, bl.RMSNORM),                           # quantiser, then GEMV
     (512, 1024, 300, bl.RMSNORM | bl.STATIC_WEIGHTS),     # quantiser, then prefill GEMM
+    (272, 512, 2400, bl.RMSNORM),                          # several quantiser waves, then GEMM
     (272, 1024, 5, bl.RMSNORM | bl.PER_TENSOR_ABSMAX),     # run as bitlinear_linear
     (144, 512, 3, 0),                                      # no RMSNorm
 ]
