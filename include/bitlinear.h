@@ -311,10 +311,14 @@ int bitlinear_linear(const uint32_t *packed, const float *gamma, int64_t d_out,
  * stream; same rules and errors), checks the device, prepares the launches
  * and returns a plan in *plan (NULL on error).  The plan is a small host
  * object owned by the caller; it keeps the pointers it was given, which must
- * stay valid while it is used, and, when its decode product splits its
- * units (see bitlinear_forward), owns a split workspace in device memory
- * (bitlinear_decode_workspace_bytes(d_out, T) bytes; BITLINEAR_ERR_CUDA if
- * it cannot be allocated).
+ * stay valid while it is used, and, for 1 <= T <= 16, owns a split
+ * workspace in device memory (bitlinear_decode_workspace_bytes(d_out, T)
+ * bytes, used when its decode product splits its units, see
+ * bitlinear_forward).  The workspace is zero-filled before plan_create
+ * returns (it waits for that fill alone), so a first run on any stream finds
+ * it ready; BITLINEAR_ERR_CUDA if it cannot be allocated or filled.  As it
+ * allocates device memory, plan_create may not be called while a stream
+ * capture is in progress.
  * flags: BITLINEAR_RMSNORM, BITLINEAR_STATIC_WEIGHTS,
  * BITLINEAR_PER_TENSOR_ABSMAX (2-bit weights only, as bitlinear_linear).
  *

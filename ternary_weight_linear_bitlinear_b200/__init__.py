@@ -461,6 +461,9 @@ class LinearPlan:
             self._fn, self._name = _entry(w, "bitlinear_linear")
             self._pre = (w.packed.data_ptr(), w.gamma.data_ptr(), w.d_out, w.d_in)
             self._ws = decode_workspace(w.d_out, T, dev)   # the plan's own, as in the C plan
+            if self._ws is not None and stream is not None:
+                # zero-filled on the current stream: runs on `stream` come after it
+                stream.wait_stream(torch.cuda.current_stream(self._ws.device))
             wsp, wsn = _ws_args(self._ws)
             self._post = (T, _ptr(gain), flags, eps, norm_eps, None, Xq.data_ptr(),
                           beta.data_ptr(), rowsum.data_ptr(), out.data_ptr(), od, wsp, wsn,

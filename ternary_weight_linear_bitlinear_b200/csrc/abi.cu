@@ -479,8 +479,10 @@ extern "C" int bitlinear_linear_plan_create(const uint32_t *packed, const float 
     const bool static_weights = (flags & BITLINEAR_STATIC_WEIGHTS) != 0;
     const bool rmsnorm = (flags & BITLINEAR_RMSNORM) != 0;
     const bool per_tensor = (flags & BITLINEAR_PER_TENSOR_ABSMAX) != 0;
-    // A decode product gets its own zero-filled split workspace (kept only
-    // if the prepared launch uses it).
+    // A decode plan owns a split workspace, used by its launches when they
+    // split.  It is zeroed on a private stream and waited for here, so that a
+    // first run on any stream (one that does not wait for the legacy default
+    // stream included) finds it zero.
     if (T >= 1 && T <= 16) {
         p->ws_bytes = decode_workspace_bytes(d_out, T);
         if (cudaMalloc(&p->ws, p->ws_bytes) != cudaSuccess) {
@@ -488,7 +490,14 @@ extern "C" int bitlinear_linear_plan_create(const uint32_t *packed, const float 
             delete p;
             return BITLINEAR_ERR_CUDA;
         }
-        if (cudaMemset(p->ws, 0, p->ws_bytes) != cudaSuccess) {
+        cudaStream_t zs = nullptr;
+        bool zeroed = cudaStreamCreateWithFlags(&zs, cudaStreamNonBlocking) == cudaSuccess;
+        if (zeroed)
+            zeroed = cudaMemsetAsync(p->ws, 0, p->ws_bytes, zs) == cudaSuccess &&
+                     cudaStreamSynchronize(zs) == cudaSuccess;
+        if (zs) cudaStreamDestroy(zs);
+        if (!zeroed) {
+            cudaGetLastError();
             cudaFree(p->ws);
             delete p;
             return BITLINEAR_ERR_CUDA;
