@@ -22,7 +22,14 @@
  *     keep the pointers they were given and own a small workspace).
  *   - All work is enqueued on `stream` (0 = legacy default stream); no entry
  *     point synchronises except bitlinear_device_error and
- *     bitlinear_get_last_device_error.
+ *     bitlinear_get_last_device_error, and bitlinear_linear_plan_create,
+ *     which waits for the zero fill of the plan's own workspace.
+ *   - Per device the library remembers the address of its device error word
+ *     and the shared-memory limits it has raised.  A device reset
+ *     (cudaDeviceReset) in the process invalidates them: after one, the
+ *     library must not be used on that device again (plans made before it
+ *     included).  bitlinear_pack_weights_noalloc alone looks its address up
+ *     again.
  *   - Shapes: d_out (output features, N) is a positive multiple of 16,
  *     d_in (input features, K) a positive multiple of 256 and at most 65536,
  *     T (tokens) is 0 .. 1048576.  T = 0 is a no-op that returns
