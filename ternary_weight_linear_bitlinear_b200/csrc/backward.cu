@@ -100,8 +100,6 @@ dequant_kernel(const int8_t *__restrict__ xq, const float *__restrict__ beta, in
     }
 }
 
-static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
-
 struct BackwardLayout {
     size_t wt, xh, total;   // byte offsets of the two bf16 operands, total bytes
 };
