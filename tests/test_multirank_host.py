@@ -8,8 +8,6 @@ import subprocess
 import sys
 import time
 
-import pytest
-
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 WORKER = os.path.join(ROOT, "tests", "multirank_worker.py")
 
