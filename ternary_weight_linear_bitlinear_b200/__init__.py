@@ -321,12 +321,15 @@ def decode_workspace_bytes(d_out: int, T: int) -> int:
 
 def decode_workspace(d_out: int, T: int, device=None):
     """A zero-filled split workspace for decode products with d_out outputs
-    and up to T tokens (None when T > 16).  The kernels leave it zero, so one
-    workspace serves every call on one stream; calls that may overlap on the
-    GPU need their own."""
+    and up to T tokens (None when T > 16), on `device` (default: the current
+    CUDA device), zeroed on that device's current stream.  The kernels leave
+    it zero, so one workspace serves every call on one stream; calls that may
+    overlap on the GPU need their own."""
     n = decode_workspace_bytes(d_out, min(max(T, 1), 16)) if T <= 16 else 0
     if n == 0:
         return None
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
